@@ -1,0 +1,395 @@
+/*
+ * attn_oracle.c -- plain, slow, fp64 CPU oracle for exact attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA library under exact_io_aware_sm_b200/.
+ *
+ * What it computes is the plain definition, with S and P materialised:
+ *
+ *   Scaled dot-product attention, "Attention Mechanism Optimization for
+ *   Efficient LLM Inference" (pyy0715.github.io), section "Background: Scaled
+ *   Dot-Product Attention", equation Attention(Q,K,V) = softmax(QK^T/sqrt(d_k))V,
+ *   and its "Kernel Fusion" table: S = QK^T * scale, P = softmax(S), O = PV,
+ *   each a full pass.  FlashAttention returns exactly this result
+ *   ("FlashAttention: memory-saving exact attention", base.kaita.kr, section 3,
+ *   Theorem 1), so the oracle is the definition written out, not the tiled
+ *   algorithm.
+ *
+ *   Safe softmax (max subtraction): same FlashAttention page, section 2 step 1;
+ *   the inference page's softmax equation in section "Tiling".
+ *
+ *   GQA head mapping: query heads form contiguous groups that share one KV
+ *   head (inference page, section "Grouped-Query Attention", mapping diagram),
+ *   so hkv = hq / (Hq / Hkv).
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *   - the mask is boolean, applied as -inf on the scaled logits;
+ *   - causal alignment is bottom-right: key j allowed for query i iff
+ *     j <= i + (Nkv - Nq);
+ *   - a row with no allowed key has O = 0 and LSE = -inf;
+ *   - LSE is the natural log-sum-exp of the scaled logits, m + ln(l);
+ *   - BLOCK masks are 16x16-granular: allowed iff block_map[i/16][j/16] != 0;
+ *   - the frame rule: query frame f sees key frames {0, f-1, f} (a set).
+ *
+ * Inputs are read element by element and converted to double from exactly the
+ * stored value (bf16 bit patterns, fp32 or fp64).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORA_MASK_NONE 0
+#define ORA_MASK_CAUSAL 1
+#define ORA_MASK_BLOCK 2
+
+#define ORA_BF16 0
+#define ORA_F32 1
+#define ORA_F64 2
+
+#define ORA_GRAIN 16 /* block-map granularity (rows and columns) */
+
+static double ld(const void *p, int dtype, size_t idx) {
+  if (dtype == ORA_BF16) {
+    uint32_t u = (uint32_t)((const uint16_t *)p)[idx] << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+  }
+  if (dtype == ORA_F32) return (double)((const float *)p)[idx];
+  return ((const double *)p)[idx];
+}
+
+/* Element mask, from its definition (no tiles involved). */
+int ora_allowed(int mask_kind, const uint8_t *block_map, int Nq, int Nkv, int i, int j) {
+  if (i < 0 || i >= Nq || j < 0 || j >= Nkv) return 0;
+  if (mask_kind == ORA_MASK_NONE) return 1;
+  if (mask_kind == ORA_MASK_CAUSAL) return j <= i + (Nkv - Nq);
+  if (mask_kind == ORA_MASK_BLOCK) {
+    int nbc = (Nkv + ORA_GRAIN - 1) / ORA_GRAIN;
+    return block_map[(size_t)(i / ORA_GRAIN) * nbc + (j / ORA_GRAIN)] != 0;
+  }
+  return 0;
+}
+
+/*
+ * One query row against keys [0, nkeys) of one (b, hkv) slice.
+ * q_at(t), k_at(j,t), v_at(j,t) are expressed through base offsets and strides
+ * (in elements).  Writes o[0..d) (fp64) and *lse.
+ */
+static void one_row(const void *q, size_t q_off, const void *k, const void *v, size_t kv_off,
+                    size_t kv_row_stride, int nkeys, int d, double scale, int dtype,
+                    int mask_kind, const uint8_t *block_map, int Nq, int Nkv, int qi,
+                    double *S, double *o, double *lse) {
+  /* S = scale * q k^T for allowed keys, -inf otherwise (materialised row). */
+  double m = -INFINITY;
+  for (int j = 0; j < nkeys; ++j) {
+    if (mask_kind >= 0 && !ora_allowed(mask_kind, block_map, Nq, Nkv, qi, j)) {
+      S[j] = -INFINITY;
+      continue;
+    }
+    double acc = 0.0;
+    for (int t = 0; t < d; ++t)
+      acc += ld(q, dtype, q_off + t) * ld(k, dtype, kv_off + (size_t)j * kv_row_stride + t);
+    S[j] = scale * acc;
+    if (S[j] > m) m = S[j];
+  }
+  for (int t = 0; t < d; ++t) o[t] = 0.0;
+  if (m == -INFINITY) { /* no allowed key */
+    *lse = -INFINITY;
+    return;
+  }
+  /* P = exp(S - m) (materialised in place), l = sum P. */
+  double l = 0.0;
+  for (int j = 0; j < nkeys; ++j) {
+    S[j] = (S[j] == -INFINITY) ? 0.0 : exp(S[j] - m);
+    l += S[j];
+  }
+  /* O = P V / l. */
+  for (int j = 0; j < nkeys; ++j) {
+    if (S[j] == 0.0) continue;
+    for (int t = 0; t < d; ++t)
+      o[t] += S[j] * ld(v, dtype, kv_off + (size_t)j * kv_row_stride + t);
+  }
+  for (int t = 0; t < d; ++t) o[t] /= l;
+  *lse = m + log(l);
+}
+
+/*
+ * Prefill attention for a list of rows.
+ * Layouts (contiguous): q [B,Nq,Hq,d], k/v [B,Nkv,Hkv,d].
+ * rows: nrows triples (b, hq, i).  o: [nrows][d] fp64, lse: [nrows] fp64.
+ * Returns 0, or -1 on bad arguments.
+ */
+int ora_attn_rows(const void *q, const void *k, const void *v, int dtype, int B, int Hq, int Hkv,
+                  int Nq, int Nkv, int d, double scale, int mask_kind, const uint8_t *block_map,
+                  const int32_t *rows, int nrows, double *o, double *lse) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || Nq < 0 || Nkv < 0) return -1;
+  if (mask_kind == ORA_MASK_BLOCK && !block_map) return -1;
+  int G = Hq / Hkv;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double *S = (double *)malloc(sizeof(double) * (size_t)(Nkv > 0 ? Nkv : 1));
+#pragma omp for schedule(dynamic, 4)
+    for (int r = 0; r < nrows; ++r) {
+      int b = rows[3 * r], hq = rows[3 * r + 1], i = rows[3 * r + 2];
+      if (b < 0 || b >= B || hq < 0 || hq >= Hq || i < 0 || i >= Nq) {
+        bad = 1;
+        continue;
+      }
+      int hkv = hq / G;
+      size_t q_off = (((size_t)b * Nq + i) * Hq + hq) * d;
+      size_t kv_off = ((size_t)b * Nkv * Hkv + hkv) * d;
+      one_row(q, q_off, k, v, kv_off, (size_t)Hkv * d, Nkv, d, scale, dtype, mask_kind, block_map,
+              Nq, Nkv, i, S, o + (size_t)r * d, lse + r);
+    }
+    free(S);
+  }
+  return bad ? -1 : 0;
+}
+
+/* Every row: o [B,Nq,Hq,d] fp64, lse [B,Hq,Nq] fp64. */
+int ora_attn_fwd(const void *q, const void *k, const void *v, int dtype, int B, int Hq, int Hkv,
+                 int Nq, int Nkv, int d, double scale, int mask_kind, const uint8_t *block_map,
+                 double *o, double *lse) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || Nq < 0 || Nkv < 0) return -1;
+  if (mask_kind == ORA_MASK_BLOCK && !block_map) return -1;
+  int G = Hq / Hkv;
+  long total = (long)B * Hq * Nq;
+#pragma omp parallel
+  {
+    double *S = (double *)malloc(sizeof(double) * (size_t)(Nkv > 0 ? Nkv : 1));
+#pragma omp for schedule(dynamic, 16)
+    for (long r = 0; r < total; ++r) {
+      int i = (int)(r % Nq);
+      int hq = (int)((r / Nq) % Hq);
+      int b = (int)(r / ((long)Nq * Hq));
+      int hkv = hq / G;
+      size_t q_off = (((size_t)b * Nq + i) * Hq + hq) * d;
+      size_t kv_off = ((size_t)b * Nkv * Hkv + hkv) * d;
+      one_row(q, q_off, k, v, kv_off, (size_t)Hkv * d, Nkv, d, scale, dtype, mask_kind, block_map,
+              Nq, Nkv, i, S, o + q_off, lse + ((size_t)b * Hq + hq) * Nq + i);
+    }
+    free(S);
+  }
+  return 0;
+}
+
+/*
+ * Single-token decode over a KV cache (inference page, section "Decode":
+ * the new query attends to every cached K_1..K_t, V_1..V_t).
+ * q [B,Hq,d]; caches [B,Lmax,Hkv,d]; seqlens[B] (host) in [0, Lmax].
+ * o [B,Hq,d] fp64, lse [B,Hq] fp64.  No mask beyond the cache length.
+ */
+int ora_decode(const void *q, const void *kc, const void *vc, int dtype, const int32_t *seqlens,
+               int B, int Hq, int Hkv, int Lmax, int d, double scale, double *o, double *lse) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || Lmax < 0) return -1;
+  for (int b = 0; b < B; ++b)
+    if (seqlens[b] < 0 || seqlens[b] > Lmax) return -1;
+  int G = Hq / Hkv;
+#pragma omp parallel
+  {
+    double *S = (double *)malloc(sizeof(double) * (size_t)(Lmax > 0 ? Lmax : 1));
+#pragma omp for schedule(dynamic, 1)
+    for (int r = 0; r < B * Hq; ++r) {
+      int b = r / Hq, hq = r % Hq, hkv = hq / G;
+      size_t q_off = ((size_t)b * Hq + hq) * d;
+      size_t kv_off = ((size_t)b * Lmax * Hkv + hkv) * d;
+      one_row(q, q_off, kc, vc, kv_off, (size_t)Hkv * d, seqlens[b], d, scale, dtype,
+              -1 /* no mask */, NULL, 1, seqlens[b], 0, S, o + q_off, lse + r);
+    }
+    free(S);
+  }
+  return 0;
+}
+
+/*
+ * Online (block-wise) softmax statistics of one vector, for checking the
+ * merge rule against the pages' worked examples ("FlashAttention" page,
+ * section 2: per-block max m and sum l, merged with e^(m_block - m_all);
+ * inference page, section "Online-Softmax": m_new = max(m_old, max B),
+ * d_new = d_old * exp(m_old - m_new) + sum exp(B - m_new)).
+ * bounds[0..nb]: block b covers x[bounds[b] .. bounds[b+1]).
+ * Outputs per block: m_blk, l_blk (the block alone), m_run, l_run (merged
+ * through block b), resc (the factor exp(m_run[b-1] - m_run[b]) applied to
+ * the old sum; 1 for b = 0).
+ */
+int ora_online_softmax(const double *x, const int *bounds, int nb, double *m_blk, double *l_blk,
+                       double *m_run, double *l_run, double *resc) {
+  double m = -INFINITY, l = 0.0;
+  for (int b = 0; b < nb; ++b) {
+    int lo = bounds[b], hi = bounds[b + 1];
+    if (hi < lo) return -1;
+    double mb = -INFINITY;
+    for (int j = lo; j < hi; ++j)
+      if (x[j] > mb) mb = x[j];
+    double lb = 0.0;
+    for (int j = lo; j < hi; ++j) lb += exp(x[j] - mb);
+    m_blk[b] = mb;
+    l_blk[b] = lb;
+    double mn = mb > m ? mb : m;
+    double r = (b == 0 || m == -INFINITY) ? 1.0 : exp(m - mn);
+    double lnew = (b == 0 ? 0.0 : l * r) + (mb == -INFINITY ? 0.0 : lb * exp(mb - mn));
+    resc[b] = r;
+    m = mn;
+    l = lnew;
+    m_run[b] = m;
+    l_run[b] = l;
+  }
+  return 0;
+}
+
+/*
+ * Merge of partial results over disjoint key sets (the same rule as above,
+ * written for normalised partial outputs): given S partials (O_s [d], lse_s),
+ * lse = log sum_s exp(lse_s) and O = sum_s exp(lse_s - lse) O_s.
+ * A partial with lse_s = -inf contributes nothing.
+ */
+int ora_merge_partials(const double *o_parts, const double *lse_parts, int nparts, int d,
+                       double *o, double *lse) {
+  double m = -INFINITY;
+  for (int s = 0; s < nparts; ++s)
+    if (lse_parts[s] > m) m = lse_parts[s];
+  for (int t = 0; t < d; ++t) o[t] = 0.0;
+  if (m == -INFINITY) {
+    *lse = -INFINITY;
+    return 0;
+  }
+  double sum = 0.0;
+  for (int s = 0; s < nparts; ++s) sum += exp(lse_parts[s] - m);
+  double L = m + log(sum);
+  for (int s = 0; s < nparts; ++s) {
+    if (lse_parts[s] == -INFINITY) continue;
+    double w = exp(lse_parts[s] - L);
+    for (int t = 0; t < d; ++t) o[t] += w * o_parts[(size_t)s * d + t];
+  }
+  *lse = L;
+  return 0;
+}
+
+/*
+ * Frame-aligned element mask (TPU attention guide, aibase.it, step 3: the
+ * live region follows frame boundaries; query frame f attends to its own
+ * frame, the previous frame and the reference frame 0).
+ */
+int ora_frame_allowed(int frame_len, int i, int j) {
+  int fi = i / frame_len, fj = j / frame_len;
+  return fj == 0 || fj == fi || fj == fi - 1;
+}
+
+/*
+ * 16x16 block map of the frame mask, by brute force over elements.  Fails
+ * (-1) unless every 16x16 block is uniformly allowed or disallowed.
+ * out: [ceil(N/16)][ceil(N/16)] with N = n_frames * frame_len.
+ */
+int ora_frame_block_map(int n_frames, int frame_len, uint8_t *out) {
+  if (n_frames <= 0 || frame_len <= 0) return -1;
+  long N = (long)n_frames * frame_len;
+  int nb = (int)((N + ORA_GRAIN - 1) / ORA_GRAIN);
+  for (int bi = 0; bi < nb; ++bi)
+    for (int bj = 0; bj < nb; ++bj) {
+      int any = 0, all = 1;
+      for (int i = bi * ORA_GRAIN; i < (bi + 1) * ORA_GRAIN && i < N; ++i)
+        for (int j = bj * ORA_GRAIN; j < (bj + 1) * ORA_GRAIN && j < N; ++j) {
+          int a = ora_frame_allowed(frame_len, i, j);
+          any |= a;
+          all &= a;
+        }
+      if (any && !all) return -1;
+      out[(size_t)bi * nb + bj] = (uint8_t)any;
+    }
+  return 0;
+}
+
+/*
+ * Tile classification by brute force over elements: 0 empty (no element
+ * allowed), 1 full (every element of the tile inside [0,Nq)x[0,Nkv) allowed),
+ * 2 partial.  out: [ceil(Nq/tq)][ceil(Nkv/tk)].
+ */
+int ora_classify(int mask_kind, const uint8_t *block_map, int Nq, int Nkv, int tq, int tk,
+                 uint8_t *out) {
+  if (tq <= 0 || tk <= 0 || Nq < 0 || Nkv < 0) return -1;
+  if (mask_kind == ORA_MASK_BLOCK && !block_map) return -1;
+  int nti = (Nq + tq - 1) / tq, ntj = (Nkv + tk - 1) / tk;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int ti = 0; ti < nti; ++ti)
+    for (int tj = 0; tj < ntj; ++tj) {
+      long cnt = 0, tot = 0;
+      for (int i = ti * tq; i < (ti + 1) * tq && i < Nq; ++i)
+        for (int j = tj * tk; j < (tj + 1) * tk && j < Nkv; ++j) {
+          cnt += ora_allowed(mask_kind, block_map, Nq, Nkv, i, j);
+          ++tot;
+        }
+      out[(size_t)ti * ntj + tj] = (uint8_t)(cnt == 0 ? 0 : (cnt == tot ? 1 : 2));
+    }
+  return 0;
+}
+
+/* Number of allowed (query, key) pairs, by brute force. */
+long long ora_count_allowed(int mask_kind, const uint8_t *block_map, int Nq, int Nkv) {
+  long long c = 0;
+#pragma omp parallel for reduction(+ : c) schedule(static)
+  for (int i = 0; i < Nq; ++i)
+    for (int j = 0; j < Nkv; ++j) c += ora_allowed(mask_kind, block_map, Nq, Nkv, i, j);
+  return c;
+}
+
+/*
+ * Check a tile schedule for one mask.  qtiles: nq x (row0, nrows, first, count),
+ * kvtiles: nk x (col0, ncols, partial).  A tile's columns may run past Nkv
+ * (padding), but every listed key must be < Nkv or the tile must be marked
+ * partial.  Conditions checked:
+ *   (1) the Q tiles partition [0, Nq) (in any order, no overlap, no gap);
+ *   (2) within one Q tile the KV tiles are pairwise disjoint;
+ *   (3) for every row of the Q tile, the union of its KV tiles, clipped to
+ *       the allowed set, is exactly the row's allowed set (coverage);
+ *   (4) every tile not marked partial is fully allowed for all its rows and
+ *       columns (including columns < Nkv only).
+ * Returns 0 when valid, or a positive code naming the first failed condition.
+ */
+int ora_check_schedule(int mask_kind, const uint8_t *block_map, int Nq, int Nkv,
+                       const int32_t *qtiles, int nq, const int32_t *kvtiles, int nk) {
+  uint8_t *rowseen = (uint8_t *)calloc((size_t)(Nq > 0 ? Nq : 1), 1);
+  uint8_t *colseen = (uint8_t *)malloc((size_t)(Nkv > 0 ? Nkv : 1) + 4096);
+  int rc = 0;
+  for (int t = 0; t < nq && !rc; ++t) {
+    int r0 = qtiles[4 * t], nr = qtiles[4 * t + 1], f = qtiles[4 * t + 2], c = qtiles[4 * t + 3];
+    if (nr <= 0 || r0 < 0 || r0 + nr > Nq || f < 0 || c < 0 || f + c > nk) {
+      rc = 1;
+      break;
+    }
+    for (int i = r0; i < r0 + nr; ++i) {
+      if (rowseen[i]) rc = 1;
+      rowseen[i] = 1;
+    }
+    if (rc) break;
+    memset(colseen, 0, (size_t)(Nkv > 0 ? Nkv : 1));
+    for (int u = f; u < f + c && !rc; ++u) {
+      int c0 = kvtiles[3 * u], nc = kvtiles[3 * u + 1], part = kvtiles[3 * u + 2];
+      if (c0 < 0 || nc <= 0) {
+        rc = 2;
+        break;
+      }
+      for (int j = c0; j < c0 + nc && j < Nkv; ++j) {
+        if (colseen[j]) rc = 2;
+        colseen[j] = 1;
+      }
+      if (!part) {
+        if (c0 + nc > Nkv) rc = 4;
+        for (int i = r0; i < r0 + nr && !rc; ++i)
+          for (int j = c0; j < c0 + nc && !rc; ++j)
+            if (!ora_allowed(mask_kind, block_map, Nq, Nkv, i, j)) rc = 4;
+      }
+    }
+    for (int i = r0; i < r0 + nr && !rc; ++i)
+      for (int j = 0; j < Nkv && !rc; ++j)
+        if (ora_allowed(mask_kind, block_map, Nq, Nkv, i, j) && !colseen[j]) rc = 3;
+  }
+  for (int i = 0; i < Nq && !rc; ++i)
+    if (!rowseen[i]) rc = 1;
+  free(rowseen);
+  free(colseen);
+  return rc;
+}
