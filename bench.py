@@ -1,0 +1,539 @@
+"""Benchmark: exact attention on B200 through the C-ABI library.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gpt2|long|frame|decode] [--no-extra]
+
+Headline (one JSON line on rank 0): prefill attention TFLOP/s on the GPT-2
+shaped causal workload (B=8, H=12, N=1024, d=64, bf16).  One step is one
+attn_fwd call (tile plan lookup, TMA/tcgen05 kernel: S = QK^T, mask on
+partial tiles, online softmax, PV, O and LSE out).  The same line carries the
+decode workload (B=64, Hq=32, Hkv=8, d=128, lengths U[1024, 8192]) in KV GB/s
+and, unless --no-extra, the long-context GQA and frame block-sparse prefill
+workloads, each with its own roofline fraction.
+
+FLOPs are algorithmic: 4*d per allowed (query, key) pair.  Bytes for decode
+are algorithmic: the K and V rows below each sequence's length, read once.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
+device synchronise on both sides; each step is bracketed by CUDA events on the
+launching stream, and L2 is flushed (a 256 MiB write) before every prefill
+step; the decode cache (1.26 GB) is larger than L2.  Multi-GPU: one process
+per GPU, each rank runs its own copy of the workload (weak scaling), the
+reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+MIB = 1 << 20
+
+# ------------------------------------------------------------------ workloads
+WORKLOADS = {
+    "tiny": dict(kind="prefill", B=1, Hq=2, Hkv=2, N=256, d=64, mask="none", dtype="f32", seed=1001,
+                 desc="tiny non-causal fp32: B=1, H=2, N=256, d=64"),
+    "gpt2": dict(kind="prefill", B=8, Hq=12, Hkv=12, N=1024, d=64, mask="causal", dtype="bf16", seed=1002,
+                 desc="GPT-2 causal prefill: B=8, H=12, N=1024, d=64, bf16"),
+    "long": dict(kind="prefill", B=1, Hq=32, Hkv=8, N=16384, d=128, mask="causal", dtype="bf16", seed=1003,
+                 desc="long-context GQA causal prefill: B=1, Hq=32, Hkv=8, N=16384, d=128, bf16"),
+    "frame": dict(kind="prefill", B=1, Hq=24, Hkv=24, N=24960, d=128, mask="frame", frames=24, frame_len=1040,
+                  dtype="bf16", seed=1004,
+                  desc="frame block-sparse: B=1, H=24, 24 frames x 1040 tokens, d=128, bf16"),
+    "decode": dict(kind="decode", B=64, Hq=32, Hkv=8, Lmax=8192, d=128, dtype="bf16", seed=1005, len_seed=2005,
+                   desc="GQA decode: B=64, Hq=32, Hkv=8, d=128, lengths U[1024,8192]"),
+}
+
+
+def allowed_pairs(w) -> int:
+    """Allowed (query, key) pairs per head of a prefill workload."""
+    N = w["N"]
+    if w["mask"] == "none":
+        return N * N
+    if w["mask"] == "causal":
+        return N * (N + 1) // 2
+    F, L = w["frames"], w["frame_len"]
+    live = 1 + (2 if F > 1 else 0) + 3 * max(0, F - 2)  # key frames {0, f-1, f}
+    return live * L * L
+
+
+def prefill_flops(w) -> int:
+    return 4 * w["d"] * allowed_pairs(w) * w["B"] * w["Hq"]
+
+
+def decode_kv_bytes(lens, Hkv, d, elem=2) -> int:
+    return int(np.sum(lens)) * Hkv * d * elem * 2
+
+
+def attention_matrix_elements(N, H, B) -> int:
+    """Elements of S (or P) for B*H heads of N x N (FlashAttention page, section 1)."""
+    return N * N * H * B
+
+
+def kv_cache_bytes_per_token(layers, heads, head_dim, elem=2) -> int:
+    """K and V for one token (inference page, "Actual KV Cache Size")."""
+    return 2 * elem * layers * heads * head_dim
+
+
+def io_elements(N, d, M):
+    """HBM accesses in elements: standard ~N^2, tiled ~N^2 d^2 / M (FlashAttention page, section 5)."""
+    return N * N, N * N * d * d / M
+
+
+# ------------------------------------------------------------------ peaks / traffic
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_sha(fn):
+    with open(os.path.join(ROOT, "exact_io_aware_sm_b200", "csrc", fn), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(key):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(key)
+    if not e or e.get("source_sha") != kernel_source_sha(e["source"]):
+        return None
+    return e["dram_bytes_per_launch"]
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read only)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, util))
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0, "source": "nvml" if self.ok else "unavailable"}
+        loaded = [m for m, u in self.samples if u > 0] or [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank works on its own batch (weak scaling): distinct seeds."""
+    return seed + 100000 * rank
+
+
+# ------------------------------------------------------------------ inputs
+def host_prefill_inputs(w, seed):
+    dt = w["dtype"]
+    B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
+    q = synthetic.tensor(seed, synthetic.TID_Q, (B, N, Hq, d), dt)
+    k = synthetic.tensor(seed, synthetic.TID_K, (B, N, Hkv, d), dt)
+    v = synthetic.tensor(seed, synthetic.TID_V, (B, N, Hkv, d), dt)
+    return q, k, v
+
+
+def to_torch(x, device=None, pin=False):
+    import torch
+    t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if x.dtype == np.uint16 else torch.from_numpy(x)
+    if pin:
+        return t.pin_memory()
+    return t.to(device) if device is not None else t
+
+
+def mask_of(w):
+    import exact_io_aware_sm_b200 as eio
+    if w["mask"] == "none":
+        return eio.MASK_NONE, None
+    if w["mask"] == "causal":
+        return eio.MASK_CAUSAL, None
+    return eio.MASK_BLOCK, eio.frame_block_map(w["frames"], w["frame_len"])
+
+
+# ------------------------------------------------------------------ timing core
+def time_steps(step, K, W, world, flush=None):
+    """W warm-ups, then K steps each bracketed by events on the current stream."""
+    import torch
+    for _ in range(W):
+        if flush:
+            flush()
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(K):
+        if flush:
+            flush()
+        starts[i].record()
+        step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - t0
+    ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return sum(ms) / K, wall
+
+
+def make_flush():
+    import torch
+    buf = torch.empty(256 * MIB, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        buf.fill_(1)
+    return flush
+
+
+def bench_prefill(w, args, world, rank, peaks, with_e2e=True):
+    import torch
+
+    import exact_io_aware_sm_b200 as eio
+    seed = rank_seed(w["seed"], rank)
+    q, k, v = host_prefill_inputs(w, seed)
+    tq, tk, tv = (to_torch(x, "cuda") for x in (q, k, v))
+    mk, bm = mask_of(w)
+    scale = 1.0 / math.sqrt(w["d"])
+    o = torch.empty_like(tq)
+    lse = torch.empty((w["B"], w["Hq"], w["N"]), dtype=torch.float32, device="cuda")
+
+    def step():
+        eio.attn_fwd(tq, tk, tv, o=o, lse=lse, scale=scale, mask_kind=mk, block_map=bm)
+
+    flush = make_flush()
+    ms, wall = time_steps(step, args.steps, args.warmup, world, flush)
+    eio.sync_status()
+    ms = max_over_ranks(ms, world)
+    flops = prefill_flops(w)
+    tflops = world * flops / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    out = {
+        "ms_per_step": ms, "tflops": tflops, "flops_per_step": flops,
+        "roofline": {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak,
+                     "unit": "TFLOP/s", "frac": flops / (ms * 1e-3) / 1e12 / peak,
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "kernel": "prefill_bf16_kernel",
+                     "traffic": recorded_traffic(f"prefill_{args_key(w)}")},
+        "gpu_launches": args.steps,
+        "wall_s": wall,
+    }
+    # attainable at this arithmetic intensity: min(peak, AI * HBM)
+    alg_bytes = q.nbytes + k.nbytes + v.nbytes + q.nbytes + lse.numel() * 4  # Q, K, V in; O, LSE out
+    ai = flops / alg_bytes
+    out["roofline"]["attainable_tflops"] = min(peak, ai * peaks["hbm_gbs"] / 1e3)
+    out["roofline"]["alg_bytes"] = int(alg_bytes)
+    if with_e2e:
+        hq_, hk_, hv_ = (to_torch(x, pin=True) for x in (q, k, v))
+        ho = torch.empty(tq.shape, dtype=tq.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            tq.copy_(hq_, non_blocking=True)
+            tk.copy_(hk_, non_blocking=True)
+            tv.copy_(hv_, non_blocking=True)
+            eio.attn_fwd(tq, tk, tv, o=o, lse=lse, scale=scale, mask_kind=mk, block_map=bm)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        ems, _ = time_steps(e2e_step, max(3, args.steps // 4), 2, world, flush)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(ems, world)
+        out["e2e"] = {"value": world * flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "ms_per_step": ems,
+                      "h2d_bytes_per_step": int(q.nbytes + k.nbytes + v.nbytes),
+                      "d2h_bytes_per_step": int(ho.numel() * ho.element_size() + hl.numel() * 4)}
+    del tq, tk, tv, o, lse
+    torch.cuda.empty_cache()
+    return out
+
+
+def args_key(w):
+    return f"{w['mask']}_d{w['d']}_n{w['N']}"
+
+
+def bench_decode(w, args, world, rank, peaks, with_e2e=True):
+    import torch
+
+    import exact_io_aware_sm_b200 as eio
+    seed = rank_seed(w["seed"], rank)
+    B, Hq, Hkv, Lmax, d = w["B"], w["Hq"], w["Hkv"], w["Lmax"], w["d"]
+    lens = synthetic.seqlens(w["len_seed"], B)
+    q = synthetic.tensor(seed, synthetic.TID_Q, (B, Hq, d))
+    kc = synthetic.kv_cache(seed, synthetic.TID_K, B, Lmax, Hkv, d, lens)
+    vc = synthetic.kv_cache(seed, synthetic.TID_V, B, Lmax, Hkv, d, lens)
+    tq, tk, tv = to_torch(q, "cuda"), to_torch(kc, "cuda"), to_torch(vc, "cuda")
+    del kc, vc
+    tl = torch.from_numpy(lens).cuda()
+    scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(tq)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+
+    def step():
+        eio.attn_decode(tq, tk, tv, tl, o=o, lse=lse, scale=scale)
+
+    steps = max(args.steps, 20)
+    ms, wall = time_steps(step, steps, args.warmup, world)
+    eio.sync_status()
+    ms = max_over_ranks(ms, world)
+    kvb = decode_kv_bytes(lens, Hkv, d)
+    alg = kvb + q.nbytes * 2 + B * Hq * 4
+    gbs = world * alg / (ms * 1e-3) / 1e9
+    peak = peaks["hbm_gbs"]
+    out = {
+        "metric": "decode KV GB/s", "value": gbs, "unit": "GB/s", "ms_per_step": ms,
+        "config": {"workload": w["desc"], "sum_len": int(lens.sum()), "kv_bytes": kvb,
+                   "l2": "cache (1.26 GB) larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": alg / (ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": alg / (ms * 1e-3) / 1e9 / peak, "peak_source": f"{peaks['source']} copy",
+                     "kernel": "decode_split_kernel + decode_combine_kernel (one call)",
+                     "traffic": recorded_traffic("decode")},
+        "gpu_launches": 2 * steps, "steps": steps, "wall_s": wall,
+    }
+    if with_e2e:
+        # A decode step's input is the new query; the cache stays resident.
+        hq_ = to_torch(q, pin=True)
+        ho = torch.empty(tq.shape, dtype=tq.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            tq.copy_(hq_, non_blocking=True)
+            eio.attn_decode(tq, tk, tv, tl, o=o, lse=lse, scale=scale)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        ems, _ = time_steps(e2e_step, steps, 3, world)
+        ems = max_over_ranks(ems, world)
+        out["e2e"] = {"value": world * alg / (ems * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ems,
+                      "h2d_bytes_per_step": int(q.nbytes), "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4)}
+    del tq, tk, tv
+    torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_prefill_sample(w, seed, batch_elems):
+    """Run the fp64 oracle on `batch_elems` batch elements of the workload;
+    returns (seconds, flops)."""
+    import oracle
+    B = w["B"]
+    w1 = dict(w, B=1)
+    q, k, v = host_prefill_inputs(w, seed)
+    mk, bm = mask_of(w)
+    kinds = {"none": oracle.MASK_NONE, "causal": oracle.MASK_CAUSAL}
+    ok = kinds.get(w["mask"], oracle.MASK_BLOCK)
+    t0 = time.perf_counter()
+    for b in range(min(batch_elems, B)):
+        oracle.attn_fwd(q[b:b + 1], k[b:b + 1], v[b:b + 1], 1.0 / math.sqrt(w["d"]), ok, bm)
+    dt = time.perf_counter() - t0
+    return dt, prefill_flops(w1) * min(batch_elems, B)
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm, on the same metric and workload."""
+    w = WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    seed = w["seed"]
+    steps = []
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        oracle_prefill_sample(w, seed, 1)
+    for _ in range(args.steps):
+        dt, fl = oracle_prefill_sample(w, seed, 1)
+        steps.append((dt, fl))
+    ms = 1e3 * sum(s[0] for s in steps) / len(steps)
+    tflops = steps[0][1] / (ms * 1e-3) / 1e12
+    line = {
+        "impl": "reference", "metric": "prefill attn TFLOP/s", "value": tflops, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w["desc"], "sample": "one batch element (1 of 8) per step"},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": "one batch element of the GPT-2 causal workload per step"},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gpt2", choices=["gpt2", "long", "frame"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the decode / other prefill workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import torch
+
+    import exact_io_aware_sm_b200 as eio
+    from exact_io_aware_sm_b200 import build as ebuild
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    ebuild.build()
+    eio.lib()
+    peaks = measured_peaks()
+    w = WORKLOADS[args.workload]
+
+    sampler = ClockSampler(torch.cuda.current_device())
+    with sampler:
+        head = bench_prefill(w, args, world, rank, peaks)
+        extra = {}
+        if not args.no_extra:
+            extra["decode"] = bench_decode(WORKLOADS["decode"], args, world, rank, peaks)
+            for name in ("long", "frame"):
+                if name == args.workload:
+                    continue
+                wx = WORKLOADS[name]
+                r = bench_prefill(wx, argparse.Namespace(steps=max(5, args.steps // 5), warmup=3),
+                                  world, rank, peaks, with_e2e=False)
+                extra[name] = {"metric": "prefill attn TFLOP/s", "value": r["tflops"], "unit": "TFLOP/s",
+                               "ms_per_step": r["ms_per_step"], "config": {"workload": wx["desc"]},
+                               "roofline": r["roofline"], "gpu_launches": r["gpu_launches"]}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        dt, fl = oracle_prefill_sample(w, rank_seed(w["seed"], 0), w["B"])
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"the whole workload ({w['B']} batch elements), fp64, {dt:.2f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": "prefill attn TFLOP/s", "value": head["tflops"], "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w["desc"], "parallelism": f"replicas x{world} (independent batches)",
+                       "l2": "flushed before every step (256 MiB write)",
+                       "flops_per_step_per_gpu": head["flops_per_step"]},
+            "roofline": head["roofline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+            "clocks": sampler.summary(), "cpu_baseline": cpu,
+        }
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

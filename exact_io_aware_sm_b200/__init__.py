@@ -1,0 +1,182 @@
+"""Python binding of libattn_b200.so (exact, IO-aware attention on B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of the shared library.  PyTorch supplies device memory and streams.
+There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+
+Entry points mirror include/attn.h:
+
+    attn_fwd(q, k, v, ...)            prefill, [B, N, H, d] tensors
+    attn_decode(q, k_cache, v_cache, seqlens, ...)
+    frame_block_map(n_frames, frame_len)
+    classify(mask_kind, block_map, Nq, Nkv, tq, tk)
+    plan(mask_kind, block_map, Nq, Nkv)
+    sync_status(stream=None)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
+
+ATTN_OK = 0
+STATUS_NAMES = {
+    0: "ATTN_OK", 1: "ATTN_ERR_NULL", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_ALIGN",
+    4: "ATTN_ERR_UNSUPPORTED", 5: "ATTN_ERR_MASK", 6: "ATTN_ERR_CUDA",
+    7: "ATTN_ERR_DEVICE_TIMEOUT", 8: "ATTN_ERR_WORKSPACE", 9: "ATTN_ERR_DEVICE_ARG",
+}
+MASK_NONE, MASK_CAUSAL, MASK_BLOCK = 0, 1, 2
+BF16, F32 = 0, 1
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, detail: str):
+        self.code = code
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {detail}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libattn_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m exact_io_aware_sm_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, I, P]
+        L.attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P]
+        L.attn_frame_block_map.argtypes = [I, I, P]
+        L.attn_classify.argtypes = [I, P, I, I, I, I, P]
+        L.attn_plan.argtypes = [I, P, I, I, P, I, P, I, P, P]
+        L.attn_sync_status.argtypes = [P]
+        L.attn_last_error_detail.argtypes = [ctypes.c_char_p, I]
+        L.attn_shutdown.argtypes = []
+        L.attn_version.restype = ctypes.c_char_p
+        for fn in (L.attn_fwd, L.attn_decode, L.attn_frame_block_map, L.attn_classify, L.attn_plan,
+                   L.attn_sync_status, L.attn_last_error_detail, L.attn_shutdown):
+            fn.restype = I
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    buf = ctypes.create_string_buffer(512)
+    lib().attn_last_error_detail(buf, 512)
+    return buf.value.decode()
+
+
+def _check(rc: int) -> None:
+    if rc != ATTN_OK:
+        raise AttnError(rc, last_error())
+
+
+def _np_ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _bm(block_map):
+    return None if block_map is None else np.ascontiguousarray(block_map, dtype=np.uint8)
+
+
+def attn_fwd(q, k, v, o=None, lse=None, scale=None, mask_kind=MASK_NONE, block_map=None,
+             stream=None, want_lse=True):
+    """Prefill attention.  q [B,Nq,Hq,d], k/v [B,Nkv,Hkv,d] CUDA tensors
+    (bf16, or fp32 for the exact fp32 path).  Returns (o, lse) with o like q
+    and lse fp32 [B,Hq,Nq] (None if want_lse is False and lse is None)."""
+    import torch
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    B, Nq, Hq, d = q.shape
+    Nkv, Hkv = k.shape[1], k.shape[2]
+    if q.dtype == torch.bfloat16:
+        dt = BF16
+    elif q.dtype == torch.float32:
+        dt = F32
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    bm = _bm(block_map)
+    _check(lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                          None if lse is None else lse.data_ptr(), B, Hq, Hkv, Nq, Nkv, d,
+                          float(scale), mask_kind, _np_ptr(bm), dt, _stream_ptr(stream)))
+    return o, lse
+
+
+def attn_decode(q, k_cache, v_cache, seqlens, o=None, lse=None, scale=None, stream=None,
+                want_lse=True):
+    """Single-token decode.  q [B,Hq,d] bf16; caches [B,Lmax,Hkv,d] bf16;
+    seqlens int32 [B] on the device."""
+    import torch
+    B, Hq, d = q.shape
+    Lmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(lib().attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+                             o.data_ptr(), None if lse is None else lse.data_ptr(), B, Hq, Hkv, Lmax,
+                             d, float(scale), _stream_ptr(stream)))
+    return o, lse
+
+
+def frame_block_map(n_frames: int, frame_len: int) -> np.ndarray:
+    nb = (n_frames * frame_len + 15) // 16
+    out = np.zeros((nb, nb), np.uint8)
+    _check(lib().attn_frame_block_map(n_frames, frame_len, _np_ptr(out)))
+    return out
+
+
+def classify(mask_kind, block_map, Nq, Nkv, tq, tk) -> np.ndarray:
+    out = np.zeros(((Nq + tq - 1) // tq, (Nkv + tk - 1) // tk), np.uint8)
+    bm = _bm(block_map)
+    _check(lib().attn_classify(mask_kind, _np_ptr(bm), Nq, Nkv, tq, tk, _np_ptr(out)))
+    return out
+
+
+def plan(mask_kind, block_map, Nq, Nkv):
+    """The tile schedule attn_fwd runs: (qtiles [n,4], kvtiles [m,3]) int32."""
+    bm = _bm(block_map)
+    nq, nk = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().attn_plan(mask_kind, _np_ptr(bm), Nq, Nkv, None, 0, None, 0,
+                           ctypes.byref(nq), ctypes.byref(nk)))
+    qt = np.zeros((nq.value, 4), np.int32)
+    kt = np.zeros((nk.value, 3), np.int32)
+    _check(lib().attn_plan(mask_kind, _np_ptr(bm), Nq, Nkv, _np_ptr(qt), nq.value, _np_ptr(kt),
+                           nk.value, ctypes.byref(nq), ctypes.byref(nk)))
+    return qt, kt
+
+
+def sync_status(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel latched a device error."""
+    _check(lib().attn_sync_status(_stream_ptr(stream)))
+
+
+def shutdown() -> None:
+    lib().attn_shutdown()
+
+
+def version() -> str:
+    return lib().attn_version().decode()

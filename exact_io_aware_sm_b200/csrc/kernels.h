@@ -1,0 +1,62 @@
+// kernels.h -- launchers shared between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace eio {
+
+// Device error codes latched by kernels (same values as attn_status).
+constexpr int kErrDeviceTimeout = 7;
+constexpr int kErrDeviceArg = 9;
+
+struct PrefillArgs {
+  const int4* qtiles;   // (row0, nrows, first_kv, n_kv)
+  const int4* kvtiles;  // (col0, ncols, partial, 0)
+  const int* order;     // Q-tile visit order
+  void* o;              // [B, Nq, Hq, d] bf16
+  float* lse;           // [B, Hq, Nq] or nullptr
+  int* err;
+  int B, Hq, Hkv, Nq, Nkv, n_qtiles;
+  float scale_log2;  // scale * log2(e)
+  int causal, causal_off;
+};
+
+// bf16 tensor-core prefill (tcgen05 / TMA).  d in {64, 128}.
+cudaError_t launch_prefill_bf16(int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                                const CUtensorMap& tv, const PrefillArgs& a, cudaStream_t s);
+int prefill_bf16_smem_bytes(int d);
+
+struct PrefillF32Args {
+  const float* q;
+  const float* k;
+  const float* v;
+  float* o;
+  float* lse;
+  const uint8_t* block_map;  // device, or nullptr
+  int B, Hq, Hkv, Nq, Nkv, mask_kind;
+  float scale;
+};
+cudaError_t launch_prefill_f32(int d, const PrefillF32Args& a, cudaStream_t s);
+
+// Split-KV decode.
+constexpr int kDecodeChunk = 512;
+struct DecodeArgs {
+  const void* q;    // [B, Hq, d] bf16
+  const void* kc;   // [B, Lmax, Hkv, d] bf16
+  const void* vc;
+  const int32_t* seqlens;
+  void* o;          // [B, Hq, d] bf16
+  float* lse;       // [B, Hq] or nullptr
+  float* opart;     // [B, Hq, nsplit, d]
+  float* lpart;     // [B, Hq, nsplit]  (log2 domain)
+  int* err;
+  int B, Hq, Hkv, Lmax, nsplit;
+  float scale_log2;
+};
+cudaError_t launch_decode(int d, int G, const DecodeArgs& a, cudaStream_t s);
+size_t decode_partial_floats(int B, int Hq, int Lmax, int d);
+
+}  // namespace eio

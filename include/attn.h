@@ -1,0 +1,187 @@
+/*
+ * attn.h -- C ABI of libattn_b200.so: exact, IO-aware attention on B200 (sm_100a).
+ *
+ * The library computes scaled dot-product attention
+ *
+ *     O = softmax(Q K^T * scale + mask) V        (per head; LSE written alongside)
+ *
+ * exactly, FlashAttention-style: Q, K and V are tiled through shared memory and
+ * tensor memory with an online softmax (running row max m and sum l, with the
+ * accumulator rescaled when m grows), so the N x N score matrix S and the
+ * probability matrix P never reach HBM.
+ *
+ * Sources for what is computed:
+ *   - SDPA definition: "Attention Mechanism Optimization for Efficient LLM
+ *     Inference", section "Background: Scaled Dot-Product Attention".
+ *   - Tiling, online softmax, exactness (Theorem 1) and block-sparse skipping:
+ *     "FlashAttention: memory-saving exact attention", sections 2, 3 and 6.
+ *   - GQA head grouping (contiguous groups share one KV head) and the decode
+ *     step over a KV cache: the inference page, sections "Grouped-Query
+ *     Attention" and "Two Phases of Inference / Decode".
+ *   - Frame-aligned block-sparse masks and the removal of partial tiles:
+ *     "TPU attention optimisation guide" (aibase.it), step 3.
+ *
+ * Conventions shared by every call
+ *   - Every function returns an attn_status code; no call aborts or exits.
+ *     attn_last_error_detail() gives the text of the last failure on the
+ *     calling thread.
+ *   - Tensors are contiguous and row-major in the layouts stated per call.
+ *     Device pointers must be 16-byte aligned.  The caller owns every buffer;
+ *     the library never frees or reallocates caller memory.
+ *   - Streams: "stream" is a cudaStream_t passed as void* (NULL = legacy
+ *     default stream).  Compute calls are asynchronous on that stream.
+ *     Argument errors are returned at once, before any launch.  Errors that a
+ *     kernel detects (a bounded wait that ran out, a cache length outside
+ *     [0, Lmax]) are latched in a device word and returned by a later
+ *     attn_sync_status().
+ *   - Workspace: the library owns a per-device workspace (tile schedules,
+ *     split-KV partials, error word).  It grows on demand with cudaMalloc and
+ *     is released by attn_shutdown().  A call that must grow it synchronises
+ *     the device.
+ *   - Masks.  NONE: every key allowed.  CAUSAL: key j allowed for query i iff
+ *     j <= i + (Nkv - Nq) (bottom-right alignment).  BLOCK: allowed iff
+ *     block_map[i/16][j/16] != 0, a host uint8 array of
+ *     [ceil(Nq/16)][ceil(Nkv/16)].  A row with no allowed key gets O = 0 and
+ *     LSE = -inf.
+ *   - LSE is ln(sum_j exp(scale * q_i . k_j)) over the allowed j, in fp32.
+ *   - GQA: Hq % Hkv == 0; query head h reads KV head h / (Hq / Hkv).
+ */
+#ifndef EXACT_IO_AWARE_SM_B200_ATTN_H
+#define EXACT_IO_AWARE_SM_B200_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_NULL = 1,            /* a required pointer is NULL */
+  ATTN_ERR_SHAPE = 2,           /* a size is out of range or inconsistent */
+  ATTN_ERR_ALIGN = 3,           /* a device pointer is not 16-byte aligned */
+  ATTN_ERR_UNSUPPORTED = 4,     /* head dim / dtype / device not supported */
+  ATTN_ERR_MASK = 5,            /* bad mask kind or missing block map */
+  ATTN_ERR_CUDA = 6,            /* a CUDA runtime or driver call failed */
+  ATTN_ERR_DEVICE_TIMEOUT = 7,  /* a kernel's bounded wait ran out */
+  ATTN_ERR_WORKSPACE = 8,       /* workspace allocation failed */
+  ATTN_ERR_DEVICE_ARG = 9       /* a kernel found a bad device-side argument (seqlens) */
+} attn_status;
+
+typedef enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_BLOCK = 2 } attn_mask_kind;
+
+typedef enum { ATTN_BF16 = 0, ATTN_F32 = 1 } attn_dtype;
+
+/* Block-map granularity (rows and columns). */
+#define ATTN_MAP_GRAIN 16
+
+/*
+ * attn_fwd -- prefill attention over full Q, K, V.
+ *
+ * Passage: FlashAttention page, section 3 (the fused tiled forward pass) and
+ * section 6 (block-sparse: tiles that the block mask zeroes are skipped); the
+ * causal mask; GQA sharing of K/V.
+ *
+ *   q      device, [B, Nq, Hq, d]   (dtype)
+ *   k, v   device, [B, Nkv, Hkv, d] (dtype)
+ *   o      device, [B, Nq, Hq, d]   (dtype; written)
+ *   lse    device, [B, Hq, Nq] fp32 (written); may be NULL to skip
+ *   scale  logit scale, typically 1/sqrt(d)
+ *   mask_kind  attn_mask_kind
+ *   block_map  host uint8 [ceil(Nq/16)][ceil(Nkv/16)] for ATTN_MASK_BLOCK,
+ *              ignored (may be NULL) otherwise.  Read during the call only.
+ *   dtype  ATTN_BF16: tensor-core path (tcgen05, fp32 accumulation, P rounded
+ *          to bf16 for the PV product).  d in {64, 128}.
+ *          ATTN_F32: fp32 inputs and output, exact fp32 CUDA-core path for
+ *          small problems.  d in {32, 64, 128}.
+ * Limits: B, Hq, Hkv >= 1; Nq, Nkv >= 1; B*Hq*ceil(Nq/16) < 2^31.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, MASK, CUDA, WORKSPACE.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Nq, int Nkv, int d, float scale, int mask_kind, const uint8_t* block_map,
+             int dtype, void* stream);
+
+/*
+ * attn_decode -- single-token decode over a KV cache (split-KV + LSE combine).
+ *
+ * Passage: the inference page, section "Decode" (the new query attends to
+ * every cached key/value) and section "Why Decode is Memory-bound"; the
+ * combine uses the block merge rule of the FlashAttention page, section 2.
+ *
+ *   q         device, [B, Hq, d] bf16 (the newest token's query per sequence)
+ *   k_cache   device, [B, Lmax, Hkv, d] bf16
+ *   v_cache   device, [B, Lmax, Hkv, d] bf16
+ *   seqlens   device, int32 [B]; sequence b attends to cache rows
+ *             0 .. seqlens[b]-1.  Rows at or above seqlens[b] are never read.
+ *             A value outside [0, Lmax] latches ATTN_ERR_DEVICE_ARG and that
+ *             sequence gets O = 0, LSE = -inf; 0 gives O = 0, LSE = -inf.
+ *   o         device, [B, Hq, d] bf16 (written)
+ *   lse       device, [B, Hq] fp32 (written); may be NULL
+ * Limits: d == 128 or 64; 1 <= Lmax; Hq / Hkv <= 8.
+ * Scratch: fp32 partials in the library workspace, B*Hq*ceil(Lmax/chunk)*(d+1)
+ * floats (chunk = 512 keys).
+ */
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                void* o, float* lse, int B, int Hq, int Hkv, int Lmax, int d, float scale,
+                void* stream);
+
+/*
+ * attn_frame_block_map -- block map of the frame-aligned video mask.
+ *
+ * Passage: TPU attention guide, step 3 (the mask's live region follows frame
+ * boundaries; each query frame attends to its own frame, the previous frame
+ * and the reference frame 0).  Query frame f sees key frames {0, f-1, f}.
+ *   out  host, uint8 [nb][nb], nb = ceil(n_frames*frame_len/16)
+ * Requires frame_len % 16 == 0 (so that no 16x16 block straddles frames);
+ * else ATTN_ERR_SHAPE.
+ */
+int attn_frame_block_map(int n_frames, int frame_len, uint8_t* out);
+
+/*
+ * attn_classify -- full / empty / partial class of every tile of a grid.
+ *
+ * Passage: TPU attention guide, step 3 (measure the share of partial blocks
+ * among live blocks; find a tile size that splits the mask into tiles fully
+ * inside or outside it).
+ *   out  host, uint8 [ceil(Nq/tq)][ceil(Nkv/tk)]: 0 empty, 1 full, 2 partial.
+ *        Edge tiles are judged on their elements inside [0,Nq) x [0,Nkv).
+ */
+int attn_classify(int mask_kind, const uint8_t* block_map, int Nq, int Nkv, int tq, int tk,
+                  uint8_t* out);
+
+/*
+ * attn_plan -- the tile schedule attn_fwd would run for a mask (host only).
+ *
+ * Q tiles hold at most 128 rows and never mix rows with different block-map
+ * rows, so under a BLOCK mask every KV tile is full (no predicate); under a
+ * CAUSAL mask the diagonal tiles are partial; a KV tile that runs past Nkv is
+ * partial.  Empty tiles are never listed.
+ *   qtiles   host int32 [qcap][4]: (row0, nrows, first_kv, n_kv), or NULL
+ *   kvtiles  host int32 [kvcap][3]: (col0, ncols, partial), or NULL
+ *            ncols is a multiple of 16 and at most 128.
+ *   *n_q, *n_kv  receive the counts (always written).
+ * Returns ATTN_ERR_SHAPE if a capacity is too small (counts still written).
+ */
+int attn_plan(int mask_kind, const uint8_t* block_map, int Nq, int Nkv, int32_t* qtiles, int qcap,
+              int32_t* kvtiles, int kvcap, int* n_q, int* n_kv);
+
+/*
+ * attn_sync_status -- synchronise `stream` and return (and clear) the error
+ * word latched by kernels on the current device (ATTN_OK if none).
+ */
+int attn_sync_status(void* stream);
+
+/* Copy the text of the last failure on this thread into buf (NUL-terminated). */
+int attn_last_error_detail(char* buf, int len);
+
+/* Release every workspace the library holds (all devices).  Idempotent. */
+int attn_shutdown(void);
+
+/* Library version string, e.g. "exact_io_aware_sm_b200 0.1". */
+const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_IO_AWARE_SM_B200_ATTN_H */

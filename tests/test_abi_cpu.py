@@ -1,0 +1,188 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+* libattn_b200.so loads and exports every function declared in include/attn.h;
+* block maps, tile classes and tile schedules are bit-exact with the oracle's
+  brute-force element enumeration;
+* argument errors come back as status codes before any device work.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_sm_b200 as eio
+import oracle
+from exact_io_aware_sm_b200 import build as ebuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_lib():
+    ebuild.build()
+    return eio.lib()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(attn_[a-z0-9_]+)\s*\(",
+                                text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert "attn_fwd" in names and "attn_decode" in names and len(names) >= 8
+    L = ctypes.CDLL(eio.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+    assert eio.version().startswith("exact_io_aware_sm_b200")
+
+
+def test_frame_block_map_bit_exact():
+    for F, L in [(24, 1040), (3, 16), (5, 48), (2, 1040), (7, 112)]:
+        assert np.array_equal(eio.frame_block_map(F, L), oracle.frame_block_map(F, L))
+    with pytest.raises(eio.AttnError) as ei:
+        eio.frame_block_map(4, 1000)  # not a multiple of 16
+    assert ei.value.code == 2
+
+
+def _random_map(rng, nbr, nbc, p):
+    return (rng.random((nbr, nbc)) < p).astype(np.uint8)
+
+
+CLASSIFY_CASES = [
+    (oracle.MASK_NONE, None, 300, 200, 128, 128),
+    (oracle.MASK_CAUSAL, None, 1024, 1024, 128, 128),
+    (oracle.MASK_CAUSAL, None, 1000, 1300, 128, 64),
+    (oracle.MASK_CAUSAL, None, 1300, 1000, 100, 37),
+    (oracle.MASK_CAUSAL, None, 17, 5, 16, 16),
+]
+
+
+@pytest.mark.parametrize("case", CLASSIFY_CASES)
+def test_classify_matches_oracle(case):
+    kind, bm, Nq, Nkv, tq, tk = case
+    assert np.array_equal(eio.classify(kind, bm, Nq, Nkv, tq, tk),
+                          oracle.classify(kind, bm, Nq, Nkv, tq, tk))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_classify_block_maps_match_oracle(seed):
+    rng = np.random.default_rng(seed)
+    Nq, Nkv = int(rng.integers(1, 700)), int(rng.integers(1, 700))
+    bm = _random_map(rng, (Nq + 15) // 16, (Nkv + 15) // 16, rng.uniform(0.1, 0.9))
+    for tq, tk in [(128, 128), (16, 16), (64, 32), (48, 80), (7, 129)]:
+        assert np.array_equal(eio.classify(oracle.MASK_BLOCK, bm, Nq, Nkv, tq, tk),
+                              oracle.classify(oracle.MASK_BLOCK, bm, Nq, Nkv, tq, tk))
+
+
+def test_classify_frame_config():
+    bm = eio.frame_block_map(24, 1040)
+    for t in (128, 16):
+        assert np.array_equal(eio.classify(oracle.MASK_BLOCK, bm, 24960, 24960, t, t),
+                              oracle.classify(oracle.MASK_BLOCK, bm, 24960, 24960, t, t))
+
+
+PLAN_CASES = [
+    (oracle.MASK_NONE, 256, 256),
+    (oracle.MASK_NONE, 250, 77),
+    (oracle.MASK_CAUSAL, 1024, 1024),
+    (oracle.MASK_CAUSAL, 300, 300),
+    (oracle.MASK_CAUSAL, 200, 333),
+    (oracle.MASK_CAUSAL, 333, 200),
+    (oracle.MASK_CAUSAL, 1, 1),
+]
+
+
+@pytest.mark.parametrize("case", PLAN_CASES)
+def test_plan_is_a_valid_schedule(case):
+    kind, Nq, Nkv = case
+    qt, kt = eio.plan(kind, None, Nq, Nkv)
+    assert oracle.check_schedule(kind, None, Nq, Nkv, qt, kt) == 0
+    assert np.all(kt[:, 1] % 16 == 0) and np.all(kt[:, 1] <= 128) and np.all(qt[:, 1] <= 128)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_plan_block_maps_valid_and_predicate_free(seed):
+    rng = np.random.default_rng(10 + seed)
+    Nq, Nkv = int(rng.integers(1, 600)), int(rng.integers(1, 600))
+    bm = _random_map(rng, (Nq + 15) // 16, (Nkv + 15) // 16, rng.uniform(0.05, 0.95))
+    if seed % 2:
+        bm = np.repeat(bm[::4], 4, axis=0)[: bm.shape[0]]  # runs of identical rows
+    qt, kt = eio.plan(oracle.MASK_BLOCK, bm, Nq, Nkv)
+    assert oracle.check_schedule(oracle.MASK_BLOCK, bm, Nq, Nkv, qt, kt) == 0
+    # only a tile running past Nkv may need a predicate
+    for c0, nc, part in kt:
+        assert part == (1 if c0 + nc > Nkv else 0)
+
+
+def test_plan_frame_config_has_no_partial_tiles():
+    bm = eio.frame_block_map(24, 1040)
+    qt, kt = eio.plan(oracle.MASK_BLOCK, bm, 24960, 24960)
+    assert oracle.check_schedule(oracle.MASK_BLOCK, bm, 24960, 24960, qt, kt) == 0
+    assert kt[:, 2].sum() == 0
+    assert len(qt) == 24 * 9  # 8 tiles of 128 rows and one of 16 per 1040-row frame
+    # live (query row, key) pairs visited == allowed pairs: nothing padded on the key side
+    visited = sum(int(r[1]) * int(kt[r[2]:r[2] + r[3], 1].sum()) for r in qt)
+    assert visited == 69 * 1040 * 1040
+
+
+def test_plan_causal_counts():
+    qt, kt = eio.plan(oracle.MASK_CAUSAL, None, 16384, 16384)
+    assert len(qt) == 128 and len(kt) == 128 * 129 // 2
+    assert kt[:, 2].sum() == 128  # one diagonal tile per Q tile
+
+
+# ---------------------------------------------------------------- errors
+FAKE = 0x10000  # never dereferenced: every case fails validation first
+
+
+def _fwd(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=2, Hkv=2, Nq=16, Nkv=16, d=64,
+                scale=0.125, mask=0, bm=None, dtype=0, stream=None)
+    args.update(kw)
+    return eio.lib().attn_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"],
+                              args["Hq"], args["Hkv"], args["Nq"], args["Nkv"], args["d"],
+                              args["scale"], args["mask"], args["bm"], args["dtype"], args["stream"])
+
+
+def test_argument_errors():
+    assert _fwd(q=None) == 1
+    assert _fwd(Hq=3, Hkv=2) == 2
+    assert _fwd(Nq=0) == 2
+    assert _fwd(scale=0.0) == 2
+    assert _fwd(scale=float("nan")) == 2
+    assert _fwd(q=FAKE + 8) == 3
+    assert _fwd(d=96) == 4
+    assert _fwd(dtype=7) == 4
+    assert _fwd(mask=2) == 5
+    assert _fwd(mask=9) == 5
+    L = eio.lib()
+    assert L.attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 12, 4, 64, 128, 0.1, None) == 4  # G = 3
+    assert L.attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 4, 64, 96, 0.1, None) == 4
+    assert L.attn_decode(FAKE, FAKE, FAKE, None, FAKE, None, 1, 8, 4, 64, 128, 0.1, None) == 1
+    assert L.attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 4, 0, 128, 0.1, None) == 2
+    assert L.attn_classify(0, None, 10, 10, 0, 16, FAKE) == 2
+    assert L.attn_classify(2, None, 10, 10, 16, 16, FAKE) == 5
+
+
+def test_last_error_detail_text():
+    assert _fwd(q=FAKE + 4) == 3
+    assert "aligned" in eio.last_error()
+    assert _fwd(Hq=3, Hkv=2) == 2
+    assert "multiple" in eio.last_error()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_no_device_is_an_error_not_a_crash():
+    # valid arguments, no GPU: reported as a CUDA error, nothing dereferenced
+    assert _fwd() == 6
+    assert eio.lib().attn_shutdown() == 0

@@ -1,0 +1,300 @@
+"""GPU parity: the CUDA library against the fp64 oracle, element by element.
+
+Tolerances (fixed by the benchmark spec for bf16 inputs, applied to the fp32
+case as well): O max-abs error <= 2e-2 and mean-abs error <= 2e-3, LSE within
+1e-3; rows without any allowed key must give O = 0 and LSE = -inf exactly.
+Small shapes are compared on every element; the full-size workloads on
+sampled rows (the oracle computes those one by one), plus properties that hold
+at any size (determinism, masked keys carry no weight, GQA == repeated MHA).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_sm_b200 as eio
+import oracle
+import synthetic
+
+pytestmark = pytest.mark.gpu
+
+O_MAX, O_MEAN, LSE_TOL = 2e-2, 2e-3, 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from exact_io_aware_sm_b200 import build
+    build.build()
+    eio.lib()
+    yield
+    eio.sync_status()
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def host_f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def check(o_gpu, lse_gpu, o_ref, lse_ref, where=""):
+    o = host_f64(o_gpu).reshape(o_ref.shape)
+    err = np.abs(o - o_ref)
+    assert np.isfinite(o).all(), f"{where}: non-finite output"
+    assert err.max() <= O_MAX, f"{where}: O max-abs {err.max():.3e}"
+    assert err.mean() <= O_MEAN, f"{where}: O mean-abs {err.mean():.3e}"
+    if lse_gpu is not None:
+        lg = lse_gpu.cpu().numpy().astype(np.float64).reshape(lse_ref.shape)
+        ninf = np.isneginf(lse_ref)
+        assert np.array_equal(np.isneginf(lg), ninf), f"{where}: -inf LSE rows differ"
+        if (~ninf).any():
+            le = np.abs(lg[~ninf] - lse_ref[~ninf])
+            assert le.max() <= LSE_TOL, f"{where}: LSE err {le.max():.3e}"
+    return err.max(), err.mean()
+
+
+def make_inputs(seed, B, Hq, Hkv, Nq, Nkv, d, dtype="bf16"):
+    q = synthetic.tensor(seed, synthetic.TID_Q, (B, Nq, Hq, d), dtype)
+    k = synthetic.tensor(seed, synthetic.TID_K, (B, Nkv, Hkv, d), dtype)
+    v = synthetic.tensor(seed, synthetic.TID_V, (B, Nkv, Hkv, d), dtype)
+    return q, k, v
+
+
+def run_fwd(q, k, v, scale, kind, bm):
+    if q.dtype == np.uint16:
+        tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    else:
+        tq, tk, tv = (torch.from_numpy(x).cuda() for x in (q, k, v))
+    o, lse = eio.attn_fwd(tq, tk, tv, scale=scale, mask_kind=kind, block_map=bm)
+    eio.sync_status()
+    return o, lse
+
+
+def random_block_map(seed, Nq, Nkv, p=0.5):
+    rng = np.random.default_rng(seed)
+    return (rng.random(((Nq + 15) // 16, (Nkv + 15) // 16)) < p).astype(np.uint8)
+
+
+SMALL = [
+    # B, Hq, Hkv, Nq, Nkv, d, mask
+    (1, 2, 2, 256, 256, 64, "none"),
+    (1, 2, 2, 256, 256, 128, "none"),
+    (2, 4, 4, 300, 300, 64, "causal"),
+    (1, 8, 2, 517, 517, 128, "causal"),
+    (1, 4, 1, 200, 333, 128, "causal"),
+    (1, 2, 2, 333, 200, 64, "causal"),
+    (1, 2, 2, 1, 1, 64, "none"),
+    (1, 2, 1, 1, 77, 128, "none"),
+    (3, 3, 3, 17, 5, 64, "none"),
+    (2, 3, 1, 130, 257, 64, "none"),
+    (1, 4, 2, 400, 300, 128, "block"),
+    (2, 2, 2, 250, 250, 64, "block"),
+    (1, 2, 2, 240, 240, 128, "frame48"),
+    (1, 2, 2, 3120, 3120, 128, "frame1040"),
+    (1, 2, 2, 3120, 3120, 64, "frame1040"),
+]
+
+
+def mask_args(kind, Nq, Nkv, seed):
+    if kind == "none":
+        return eio.MASK_NONE, None
+    if kind == "causal":
+        return eio.MASK_CAUSAL, None
+    if kind == "block":
+        return eio.MASK_BLOCK, random_block_map(seed, Nq, Nkv, 0.45)
+    L = int(kind[len("frame"):])
+    return eio.MASK_BLOCK, eio.frame_block_map(Nq // L, L)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[f"{c[-1]}-{c[3]}x{c[4]}-d{c[5]}-g{c[1]//c[2]}" for c in SMALL])
+def test_prefill_small_all_elements(case):
+    B, Hq, Hkv, Nq, Nkv, d, kind = case
+    seed = 7000 + SMALL.index(case)
+    q, k, v = make_inputs(seed, B, Hq, Hkv, Nq, Nkv, d)
+    mk, bm = mask_args(kind, Nq, Nkv, seed)
+    scale = 1 / math.sqrt(d)
+    o, lse = run_fwd(q, k, v, scale, mk, bm)
+    ro, rl = oracle.attn_fwd(q, k, v, scale, mk, bm)
+    check(o, lse, ro, rl, str(case))
+
+
+def test_config1_tiny_fp32():
+    """B=1, H=2, N=256, d=64, fp32 inputs, no mask (all elements)."""
+    q, k, v = make_inputs(1001, 1, 2, 2, 256, 256, 64, "f32")
+    o, lse = run_fwd(q, k, v, 1 / 8, eio.MASK_NONE, None)
+    ro, rl = oracle.attn_fwd(q, k, v, 1 / 8, eio.MASK_NONE)
+    mx, mean = check(o, lse, ro, rl, "config1")
+    assert mx < 1e-5  # exact fp32 arithmetic
+
+
+@pytest.mark.parametrize("case", [(2, 4, 4, 100, 100, 64, 0), (1, 4, 2, 64, 200, 128, 1),
+                                  (1, 2, 1, 40, 40, 32, 2)])
+def test_fp32_masks(case):
+    B, Hq, Hkv, Nq, Nkv, d, kind = case
+    q, k, v = make_inputs(1100 + kind, B, Hq, Hkv, Nq, Nkv, d, "f32")
+    bm = random_block_map(5, Nq, Nkv) if kind == 2 else None
+    o, lse = run_fwd(q, k, v, 0.2, kind, bm)
+    ro, rl = oracle.attn_fwd(q, k, v, 0.2, kind, bm)
+    check(o, lse, ro, rl, str(case))
+
+
+def sampled_rows(rng, B, Hq, Nq, special, n):
+    rows = [(int(rng.integers(B)), int(rng.integers(Hq)), int(i)) for i in rng.integers(0, Nq, n)]
+    rows += [(b, h, i) for i in special for b, h in [(0, 0), (B - 1, Hq - 1)]]
+    return np.array(rows, np.int32)
+
+
+def check_rows(o, lse, ref_o, ref_l, rows, where):
+    og = host_f64(o)
+    lg = lse.cpu().numpy().astype(np.float64)
+    got_o = np.stack([og[b, i, h] for b, h, i in rows])
+    got_l = np.array([lg[b, h, i] for b, h, i in rows])
+    err = np.abs(got_o - ref_o)
+    assert err.max() <= O_MAX and err.mean() <= O_MEAN, f"{where}: {err.max():.3e} {err.mean():.3e}"
+    assert np.abs(got_l - ref_l).max() <= LSE_TOL, f"{where}: LSE {np.abs(got_l - ref_l).max():.3e}"
+
+
+def test_config2_gpt2_causal_full_size():
+    B, H, N, d = 8, 12, 1024, 64
+    q, k, v = make_inputs(1002, B, H, H, N, N, d)
+    o, lse = run_fwd(q, k, v, 1 / 8, eio.MASK_CAUSAL, None)
+    rows = sampled_rows(np.random.default_rng(2), B, H, N, [0, 1, 127, 128, 129, 511, 1023], 400)
+    ro, rl = oracle.attn_rows(q, k, v, 1 / 8, rows, oracle.MASK_CAUSAL)
+    check_rows(o, lse, ro, rl, rows, "config2")
+
+
+def test_config3_long_gqa_causal_full_size():
+    B, Hq, Hkv, N, d = 1, 32, 8, 16384, 128
+    q, k, v = make_inputs(1003, B, Hq, Hkv, N, N, d)
+    o, lse = run_fwd(q, k, v, 1 / math.sqrt(128), eio.MASK_CAUSAL, None)
+    rows = sampled_rows(np.random.default_rng(3), B, Hq, N, [0, 127, 128, 8191, 16383], 160)
+    ro, rl = oracle.attn_rows(q, k, v, 1 / math.sqrt(128), rows, oracle.MASK_CAUSAL)
+    check_rows(o, lse, ro, rl, rows, "config3")
+
+
+def test_config4_frame_block_sparse_full_size():
+    F, L, H, d = 24, 1040, 24, 128
+    N = F * L
+    q, k, v = make_inputs(1004, 1, H, H, N, N, d)
+    bm = eio.frame_block_map(F, L)
+    o, lse = run_fwd(q, k, v, 1 / math.sqrt(128), eio.MASK_BLOCK, bm)
+    special = [0, 1023, 1024, 1039, 1040, 2079, 2080, 3119, 3120, 12345, N - 17, N - 16, N - 1]
+    rows = sampled_rows(np.random.default_rng(4), 1, H, N, special, 120)
+    ro, rl = oracle.attn_rows(q, k, v, 1 / math.sqrt(128), rows, oracle.MASK_BLOCK, bm)
+    check_rows(o, lse, ro, rl, rows, "config4")
+
+
+# ------------------------------------------------------------------ decode
+def run_decode(q, kc, vc, lens, scale):
+    o, lse = eio.attn_decode(dev_bf16(q), dev_bf16(kc), dev_bf16(vc),
+                             torch.from_numpy(np.asarray(lens, np.int32)).cuda(), scale=scale)
+    eio.sync_status()
+    return o, lse
+
+
+DECODE_SMALL = [
+    # B, Hq, Hkv, Lmax, d, lens
+    (4, 8, 8, 600, 128, [1, 15, 16, 17]),
+    (3, 8, 4, 1100, 128, [511, 512, 513]),
+    (2, 16, 2, 2000, 128, [1025, 2000]),
+    (2, 8, 1, 700, 64, [700, 3]),
+    (5, 4, 2, 64, 64, [64, 1, 33, 2, 63]),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_SMALL)
+def test_decode_small(case):
+    B, Hq, Hkv, Lmax, d, lens = case
+    lens = np.array(lens, np.int32)
+    seed = 2100 + DECODE_SMALL.index(case)
+    q = synthetic.tensor(seed, synthetic.TID_Q, (B, Hq, d))
+    kc = synthetic.kv_cache(seed, synthetic.TID_K, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)  # NaN past len
+    vc = synthetic.kv_cache(seed, synthetic.TID_V, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
+    o, lse = run_decode(q, kc, vc, lens, 1 / math.sqrt(d))
+    ro, rl = oracle.decode(q, kc, vc, lens, 1 / math.sqrt(d))
+    check(o, lse, ro, rl, str(case))
+
+
+def test_decode_zero_length_and_bad_length():
+    B, Hq, Hkv, Lmax, d = 3, 4, 4, 64, 128
+    q = synthetic.tensor(5, 1, (B, Hq, d))
+    lens = np.array([0, 64, 5], np.int32)
+    kc = synthetic.kv_cache(5, 2, B, Lmax, Hkv, d, lens)
+    vc = synthetic.kv_cache(5, 3, B, Lmax, Hkv, d, lens)
+    o, lse = run_decode(q, kc, vc, lens, 0.1)
+    ro, rl = oracle.decode(q, kc, vc, lens, 0.1)
+    check(o, lse, ro, rl, "zero-length")
+    # a length above Lmax is latched as a device argument error; that row reads nothing
+    bad = np.array([3, 65, 5], np.int32)
+    o2, l2 = eio.attn_decode(dev_bf16(q), dev_bf16(kc), dev_bf16(vc), torch.from_numpy(bad).cuda(), scale=0.1)
+    with pytest.raises(eio.AttnError) as ei:
+        eio.sync_status()
+    assert ei.value.code == 9
+    assert torch.all(o2[1].float() == 0) and torch.isneginf(l2[1]).all()
+    eio.sync_status()  # cleared
+
+
+def test_config5_gqa_decode_full_size():
+    B, Hq, Hkv, Lmax, d = 64, 32, 8, 8192, 128
+    lens = synthetic.seqlens(2005, B)
+    q = synthetic.tensor(1005, synthetic.TID_Q, (B, Hq, d))
+    kc = synthetic.kv_cache(1005, synthetic.TID_K, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
+    vc = synthetic.kv_cache(1005, synthetic.TID_V, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
+    o, lse = run_decode(q, kc, vc, lens, 1 / math.sqrt(d))
+    ro, rl = oracle.decode(q, kc, vc, lens, 1 / math.sqrt(d))
+    check(o, lse, ro, rl, "config5")
+
+
+# ------------------------------------------------------------------ properties
+def test_masked_keys_carry_no_weight_bitwise():
+    """Causal: keys a row must not see changed to 1e4 -> bit-identical output.
+    Block map: keys in blocks no query may see set to NaN (never loaded)."""
+    B, H, N, d = 1, 2, 384, 128
+    q, k, v = make_inputs(31, B, H, H, N, N, d)
+    o1, l1 = run_fwd(q, k, v, 0.09, eio.MASK_CAUSAL, None)
+    k2, v2 = k.copy(), v.copy()
+    big = synthetic.f32_to_bf16_bits(np.float32([1e4, -1e4]))
+    k2[0, 200:] = big[0]
+    v2[0, 200:] = big[1]
+    # rows < 200 cannot see keys >= 200
+    o2, l2 = run_fwd(q, k2, v2, 0.09, eio.MASK_CAUSAL, None)
+    assert torch.equal(o1[:, :200], o2[:, :200]) and torch.equal(l1[:, :, :200], l2[:, :, :200])
+
+    bm = np.ones((N // 16, N // 16), np.uint8)
+    bm[:, 5:9] = 0  # key blocks 5..8 seen by nobody
+    o3, l3 = run_fwd(q, k, v, 0.09, eio.MASK_BLOCK, bm)
+    k3, v3 = k.copy(), v.copy()
+    k3[0, 80:144] = 0x7FC0
+    v3[0, 80:144] = 0x7FC0
+    o4, l4 = run_fwd(q, k3, v3, 0.09, eio.MASK_BLOCK, bm)
+    assert torch.equal(o3, o4) and torch.equal(l3, l4)
+
+
+def test_deterministic():
+    q, k, v = make_inputs(41, 2, 4, 2, 700, 700, 128)
+    a = run_fwd(q, k, v, 0.1, eio.MASK_CAUSAL, None)
+    b = run_fwd(q, k, v, 0.1, eio.MASK_CAUSAL, None)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_gqa_equals_repeated_mha_bitwise():
+    q, k, v = make_inputs(51, 1, 8, 2, 300, 300, 64)
+    o1, l1 = run_fwd(q, k, v, 0.12, eio.MASK_CAUSAL, None)
+    kr, vr = np.repeat(k, 4, axis=2), np.repeat(v, 4, axis=2)
+    o2, l2 = run_fwd(q, kr, vr, 0.12, eio.MASK_CAUSAL, None)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_constant_v_rows():
+    B, H, N, d = 1, 2, 300, 128
+    q, k, _ = make_inputs(61, B, H, H, N, N, d)
+    c = synthetic.normal(62, 1, d)
+    v = np.broadcast_to(c, (B, N, H, d)).copy()
+    o, _ = run_fwd(q, k, v, 0.1, eio.MASK_CAUSAL, None)
+    cf = synthetic.bf16_bits_to_f32(c).astype(np.float64)
+    err = np.abs(host_f64(o) - cf).max()
+    assert err <= 8e-3 * max(1.0, np.abs(cf).max())
