@@ -465,7 +465,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="gpt2", choices=["gpt2", "long", "frame"])
+    ap.add_argument("--workload", default="gpt2", choices=["gpt2", "long", "frame", "decode"])
     ap.add_argument("--no-extra", action="store_true", help="skip the decode / other prefill workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -493,6 +493,20 @@ def main():
     w = WORKLOADS[args.workload]
 
     sampler = ClockSampler(torch.cuda.current_device())
+    if args.workload == "decode":
+        with sampler:
+            d = bench_decode(w, args, world, rank, peaks)
+        if rank == 0:
+            line = {"metric": d["metric"], "value": d["value"], "unit": d["unit"], "n_gpus": world,
+                    "steps": d["steps"], "warmup": args.warmup, "ms_per_step": d["ms_per_step"],
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                    "data": "synthetic", "config": d["config"], "roofline": d["roofline"], "e2e": d["e2e"],
+                    "gpu_launches": d["gpu_launches"], "clocks": sampler.summary(), "cpu_baseline": None}
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     with sampler:
         head = bench_prefill(w, args, world, rank, peaks)
         extra = {}
