@@ -211,6 +211,8 @@ int check_mask_args(int mask_kind, const uint8_t* block_map) {
 
 }  // namespace
 
+void eio::set_error_detail(const char* msg) { std::snprintf(g_err, sizeof g_err, "%s", msg); }
+
 extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,

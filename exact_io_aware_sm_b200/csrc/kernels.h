@@ -59,4 +59,7 @@ struct DecodeArgs {
 cudaError_t launch_decode(int d, int G, const DecodeArgs& a, cudaStream_t s);
 size_t decode_partial_floats(int B, int Hq, int Lmax, int d);
 
+// Sets the text returned by attn_last_error_detail() on this thread.
+void set_error_detail(const char* msg);
+
 }  // namespace eio

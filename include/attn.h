@@ -177,6 +177,42 @@ int attn_last_error_detail(char* buf, int len);
 /* Release every workspace the library holds (all devices).  Idempotent. */
 int attn_shutdown(void);
 
+/* Size of the fixed device array that attn_decode_noalloc uses as scratch. */
+#define ATTN_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
+
+/*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate.
+ *
+ * The source pages have no counterpart for this entry point.
+ *
+ * Some callers cannot let a library call cudaMalloc: a host framework that
+ * owns all device memory through its own pool, a serving process whose memory
+ * budget is fixed at start-up, or a caller that cannot take the device-wide
+ * synchronisation cudaMalloc / cudaFree may cause.  This variant computes the
+ * same decode as attn_decode (same arguments, layouts and kernels) but keeps
+ * its scratch (the per-split fp32 partials and an error word) in one fixed
+ * file-scope device array of ATTN_NOALLOC_SCRATCH_BYTES.  Every GPU that loads
+ * the library holds that array until the process exits.  The call itself
+ * performs no cudaMalloc, cudaFree or other allocating call.
+ *
+ *   Scratch needed: 256 + 4 * B*Hq*ceil(Lmax/512)*(d+1) bytes; a shape that
+ *   needs more than ATTN_NOALLOC_SCRATCH_BYTES returns ATTN_ERR_WORKSPACE
+ *   (attn_last_error_detail says how much it needed), before any GPU work.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, and the array keeps
+ *   the previous call's contents (each call clears the error word and writes
+ *   every partial it reads).  Calls that overlap on the GPU (different
+ *   streams, or other host threads) race on the array: order them.
+ *   Errors: as attn_decode for arguments.  A seqlens entry outside [0, Lmax]
+ *   gives that sequence O = 0 and LSE = -inf; this variant does not report it
+ *   through attn_sync_status.
+ */
+int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Lmax, int d, float scale, void* stream);
+
 /* Library version string, e.g. "exact_io_aware_sm_b200 0.1". */
 const char* attn_version(void);
 
