@@ -57,6 +57,33 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pair arithmetic (sm_100): one instruction for two lanes of work.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -271,49 +298,63 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t sr[128];
       const uint32_t sbase = tmem + lane_off + static_cast<uint32_t>((j & 1) * 128);
+      const bool full = nc == 128 && !kt.z;
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        if (c * 16 < nc) tmem_ld16(sbase + c * 16, sr + c * 16);
+        for (int c = 0; c < 4; ++c) tmem_ld32(sbase + c * 32, sr + c * 32);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (c * 16 < nc) tmem_ld16(sbase + c * 16, sr + c * 16);
+      }
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[j & 1]);
 
-      // Predicate: only on partial tiles (and columns past the tile width).
-      float mx = -INFINITY;
-      if (kt.z) {
-        const int c0 = kt.x;
-        int lim = min(nc, a.Nkv - c0);  // allowed iff c < lim
-        if (a.causal) lim = min(lim, grow + a.causal_off + 1 - c0);
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float x = c < lim ? __uint_as_float(sr[c]) : -INFINITY;
-          sr[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+      // Predicate: only on partial tiles and on columns past a narrow tile.
+      if (!full) {
+        int lim = nc;  // allowed iff c < lim
+        if (kt.z) {
+          const int c0 = kt.x;
+          lim = min(lim, a.Nkv - c0);
+          if (a.causal) lim = min(lim, grow + a.causal_off + 1 - c0);
         }
-      } else {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float x = c < nc ? __uint_as_float(sr[c]) : -INFINITY;
-          sr[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
       }
+      // Row max: four independent chains of 3-input max.
+      float mx4[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        float m = __uint_as_float(sr[t * 32]);
+#pragma unroll
+        for (int c = 1; c < 31; c += 2)
+          m = max3f(m, __uint_as_float(sr[t * 32 + c]), __uint_as_float(sr[t * 32 + c + 1]));
+        mx4[t] = fmaxf(m, __uint_as_float(sr[t * 32 + 31]));
+      }
+      const float mx = max3f(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
       const float mx_s = mx * sl2;
       const bool upd = mx_s > m_b + kRescaleThreshold;
       const float m_new = upd ? mx_s : m_b;
       const float alpha = upd ? ex2(m_b - m_new) : 1.0f;
       const float base = (m_new == -INFINITY) ? 0.f : m_new;
 
-      float sum = 0.f;
+      // p = 2^(s * scale*log2e - base), packed two at a time; row sum in
+      // four independent pairs of accumulators.
+      float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
       uint32_t pk[64];
 #pragma unroll
       for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl2, -base));
-        const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, -base));
-        sum += p0 + p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+        const float2 t = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                               make_float2(sl2, sl2), make_float2(-base, -base));
+        const float2 p = make_float2(ex2(t.x), ex2(t.y));
+        acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], p);
+        pk[c >> 1] = pack_bf16x2(p.x, p.y);
       }
+      const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+      const float sum = s01.x + s01.y;
 
       // P buffer and O are free once PV_{j-1} has completed.
       if (j > 0) {
