@@ -43,13 +43,17 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // ------------------------------------------------------------------ workspace
 struct DevPlan {
-  int mask_kind, Nq, Nkv;
+  int mask_kind, Nq, Nkv, rows_mode;
   std::vector<uint8_t> map;  // copy of the host block map (BLOCK only)
   int n_q = 0, n_kv = 0;
   int4* d_q = nullptr;
   int4* d_kv = nullptr;
   int* d_order = nullptr;
   uint8_t* d_map = nullptr;  // device copy of the block map (fp32 path)
+  int n_pairs = 0;
+  int4* d_pairs = nullptr;   // tensor-core path: Q-tile pairs, their KV lists, visit order
+  int4* d_pkv = nullptr;
+  int* d_porder = nullptr;
 };
 
 struct DevWs {
@@ -68,6 +72,12 @@ void free_plan(DevPlan& p) {
   cudaFree(p.d_kv);
   cudaFree(p.d_order);
   cudaFree(p.d_map);
+  cudaFree(p.d_pairs);
+  cudaFree(p.d_pkv);
+  cudaFree(p.d_porder);
+  p.d_pairs = nullptr;
+  p.d_pkv = nullptr;
+  p.d_porder = nullptr;
   p.d_q = nullptr;
   p.d_kv = nullptr;
   p.d_order = nullptr;
@@ -114,13 +124,14 @@ int upload(T** dst, const T* src, size_t n, cudaStream_t s) {
 
 // Find or build the device-resident plan for a mask.
 int get_plan(DevWs& ws, int mask_kind, const uint8_t* block_map, int Nq, int Nkv, bool need_map,
-             cudaStream_t s, DevPlan** out) {
+             int rows_mode, cudaStream_t s, DevPlan** out) {
   const size_t map_bytes =
       mask_kind == ATTN_MASK_BLOCK
           ? static_cast<size_t>((Nq + kGrain - 1) / kGrain) * ((Nkv + kGrain - 1) / kGrain)
           : 0;
   for (auto it = ws.plans.begin(); it != ws.plans.end(); ++it) {
-    if (it->mask_kind != mask_kind || it->Nq != Nq || it->Nkv != Nkv) continue;
+    if (it->mask_kind != mask_kind || it->Nq != Nq || it->Nkv != Nkv || it->rows_mode != rows_mode)
+      continue;
     if (map_bytes && (it->map.size() != map_bytes ||
                       std::memcmp(it->map.data(), block_map, map_bytes) != 0))
       continue;
@@ -135,13 +146,21 @@ int get_plan(DevWs& ws, int mask_kind, const uint8_t* block_map, int Nq, int Nkv
   dp.mask_kind = mask_kind;
   dp.Nq = Nq;
   dp.Nkv = Nkv;
+  dp.rows_mode = rows_mode;
   if (map_bytes) dp.map.assign(block_map, block_map + map_bytes);
   dp.n_q = static_cast<int>(p.q.size());
   dp.n_kv = static_cast<int>(p.kv.size());
+  PairPlan pp;
+  build_pairs(p, rows_mode != 0, &pp);
+  dp.n_pairs = static_cast<int>(pp.pairs.size());
+  static_assert(sizeof(PairTile) == 2 * sizeof(int4) && sizeof(PairKV) == sizeof(int4), "layout");
   int rc;
   if ((rc = upload(&dp.d_q, reinterpret_cast<const int4*>(p.q.data()), p.q.size(), s)) ||
       (rc = upload(&dp.d_kv, reinterpret_cast<const int4*>(p.kv.data()), p.kv.size(), s)) ||
       (rc = upload(&dp.d_order, p.order.data(), p.order.size(), s)) ||
+      (rc = upload(&dp.d_pairs, reinterpret_cast<const int4*>(pp.pairs.data()), 2 * pp.pairs.size(), s)) ||
+      (rc = upload(&dp.d_pkv, reinterpret_cast<const int4*>(pp.kv.data()), pp.kv.size(), s)) ||
+      (rc = upload(&dp.d_porder, pp.order.data(), pp.order.size(), s)) ||
       (map_bytes && need_map && (rc = upload(&dp.d_map, block_map, map_bytes, s)))) {
     free_plan(dp);
     return rc;
@@ -246,7 +265,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (dtype == ATTN_F32) {
     DevPlan* pl = nullptr;
     if (mask_kind == ATTN_MASK_BLOCK) {
-      if (int rc = get_plan(*ws, mask_kind, block_map, Nq, Nkv, true, s, &pl)) return rc;
+      if (int rc = get_plan(*ws, mask_kind, block_map, Nq, Nkv, true, 0, s, &pl)) return rc;
     }
     PrefillF32Args a{};
     a.q = static_cast<const float*>(q);
@@ -266,18 +285,21 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     return e == cudaSuccess ? ATTN_OK : cuda_err(e, "fp32 prefill launch");
   }
 
+  const int G = Hq / Hkv;
+  const int rows_mode = G == 1 ? 1 : 0;
   DevPlan* pl = nullptr;
-  if (int rc = get_plan(*ws, mask_kind, block_map, Nq, Nkv, false, s, &pl)) return rc;
-  if (static_cast<long long>(pl->n_q) * B * Hq >= (1ll << 31))
-    return set_err(ATTN_ERR_SHAPE, "too many work items (B*Hq*Q tiles)");
+  if (int rc = get_plan(*ws, mask_kind, block_map, Nq, Nkv, false, rows_mode, s, &pl)) return rc;
   CUtensorMap tq, tk, tv;
   if (int rc = make_map(&tq, q, B, Nq, Hq, d)) return rc;
   if (int rc = make_map(&tk, k, B, Nkv, Hkv, d)) return rc;
   if (int rc = make_map(&tv, v, B, Nkv, Hkv, d)) return rc;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   PrefillArgs a{};
-  a.qtiles = pl->d_q;
-  a.kvtiles = pl->d_kv;
-  a.order = pl->d_order;
+  a.pairs = pl->d_pairs;
+  a.kvtiles = pl->d_pkv;
+  a.order = pl->d_porder;
   a.o = o;
   a.lse = lse;
   a.err = ws->d_err;
@@ -286,7 +308,11 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.Hkv = Hkv;
   a.Nq = Nq;
   a.Nkv = Nkv;
-  a.n_qtiles = pl->n_q;
+  a.G = G;
+  a.HP = rows_mode ? 1 : (G + 1) / 2;
+  a.rows_mode = rows_mode;
+  a.n_items = static_cast<long long>(pl->n_pairs) * B * Hkv * a.HP;
+  a.num_ctas = sms > 0 ? sms : 148;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.causal = mask_kind == ATTN_MASK_CAUSAL;
   a.causal_off = Nkv - Nq;

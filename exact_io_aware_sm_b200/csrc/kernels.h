@@ -13,14 +13,19 @@ constexpr int kErrDeviceTimeout = 7;
 constexpr int kErrDeviceArg = 9;
 
 struct PrefillArgs {
-  const int4* qtiles;   // (row0, nrows, first_kv, n_kv)
-  const int4* kvtiles;  // (col0, ncols, partial, 0)
-  const int* order;     // Q-tile visit order
+  const int4* pairs;    // per pair: (rowA, nrowsA, rowB, nrowsB), (kv_first, nA, nB, 0)
+  const int4* kvtiles;  // (col0, ncols, flags, 0); flags bit 0 partial for A, bit 1 for B
+  const int* order;     // pairs, most KV tiles first
   void* o;              // [B, Nq, Hq, d] bf16
   float* lse;           // [B, Hq, Nq] or nullptr
   int* err;
-  int B, Hq, Hkv, Nq, Nkv, n_qtiles;
-  float scale_log2;  // scale * log2(e)
+  int B, Hq, Hkv, Nq, Nkv;
+  int G;                // query heads per KV head
+  int HP;               // head pairs per KV head (ceil(G/2)), 1 in rows mode
+  int rows_mode;        // 1: slots are two Q tiles of one head (G == 1)
+  long long n_items;    // pairs * B * Hkv * HP
+  int num_ctas;         // persistent grid size (SM count)
+  float scale_log2;     // scale * log2(e)
   int causal, causal_off;
 };
 

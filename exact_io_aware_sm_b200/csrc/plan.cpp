@@ -81,6 +81,65 @@ void build_plan(int mask_kind, const uint8_t* block_map, int Nq, int Nkv, Plan* 
   });
 }
 
+void build_pairs(const Plan& plan, bool rows_mode, PairPlan* out) {
+  out->rows_mode = rows_mode;
+  out->pairs.clear();
+  out->kv.clear();
+  out->order.clear();
+  auto push_pair = [&](const QTile* a, const QTile& b) {
+    PairTile pt{};
+    pt.rowB = b.row0;
+    pt.nrowsB = b.nrows;
+    pt.nB = b.n_kv;
+    pt.kv_first = static_cast<int32_t>(out->kv.size());
+    if (a) {
+      pt.rowA = a->row0;
+      pt.nrowsA = a->nrows;
+      pt.nA = a->n_kv;
+    }
+    for (int k = 0; k < b.n_kv; ++k) {
+      const KVTile& t = plan.kv[b.first_kv + k];
+      int flags = t.partial ? 2 : 0;
+      if (a && k < a->n_kv && plan.kv[a->first_kv + k].partial) flags |= 1;
+      out->kv.push_back(PairKV{t.col0, t.ncols, flags, 0});
+    }
+    out->pairs.push_back(pt);
+  };
+  // A's KV list is a prefix of B's (same tiles, same order).
+  auto nests = [&](const QTile& a, const QTile& b) {
+    if (a.n_kv > b.n_kv) return false;
+    for (int k = 0; k < a.n_kv; ++k) {
+      const KVTile& x = plan.kv[a.first_kv + k];
+      const KVTile& y = plan.kv[b.first_kv + k];
+      if (x.col0 != y.col0 || x.ncols != y.ncols) return false;
+    }
+    return true;
+  };
+  const size_t nq = plan.q.size();
+  if (!rows_mode) {
+    for (size_t i = 0; i < nq; ++i) push_pair(&plan.q[i], plan.q[i]);
+  } else {
+    size_t i = 0;
+    while (i < nq) {
+      if (i + 1 < nq && nests(plan.q[i], plan.q[i + 1])) {
+        push_pair(&plan.q[i], plan.q[i + 1]);
+        i += 2;
+      } else if (i + 1 < nq && nests(plan.q[i + 1], plan.q[i])) {
+        push_pair(&plan.q[i + 1], plan.q[i]);
+        i += 2;
+      } else {
+        push_pair(nullptr, plan.q[i]);
+        i += 1;
+      }
+    }
+  }
+  out->order.resize(out->pairs.size());
+  for (size_t i = 0; i < out->pairs.size(); ++i) out->order[i] = static_cast<int32_t>(i);
+  std::stable_sort(out->order.begin(), out->order.end(), [&](int32_t x, int32_t y) {
+    return out->pairs[x].nB > out->pairs[y].nB;
+  });
+}
+
 void classify_tiles(int mask_kind, const uint8_t* block_map, int Nq, int Nkv, int tq, int tk,
                     uint8_t* out) {
   const int nti = ceil_div(Nq, tq), ntj = ceil_div(Nkv, tk);

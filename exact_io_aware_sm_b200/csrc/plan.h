@@ -33,6 +33,28 @@ struct Plan {
 // Build the plan.  mask_kind: 0 none, 1 causal, 2 block (block_map required).
 void build_plan(int mask_kind, const uint8_t* block_map, int Nq, int Nkv, Plan* out);
 
+// Q tiles processed two at a time by one CTA ("slots" A and B) that share
+// every K/V tile: slot B visits the whole KV list, slot A a prefix of it.
+//   mode 'heads' (query heads per KV head G >= 2): A and B are the same Q tile
+//     for two query heads of one KV group (identical KV lists);
+//   mode 'rows' (G == 1): A and B are two Q tiles of one head whose KV lists
+//     nest (A's list is a prefix of B's), e.g. consecutive causal tiles.
+// A Q tile without a partner runs alone in slot B.
+struct PairTile {
+  int32_t rowA, nrowsA, rowB, nrowsB;  // nrowsA == 0: slot A unused
+  int32_t kv_first, nA, nB, pad;       // KV tiles [kv_first, kv_first + nB); A uses the first nA
+};
+struct PairKV {
+  int32_t col0, ncols, flags, pad;  // flags bit 0: partial for A, bit 1: partial for B
+};
+struct PairPlan {
+  bool rows_mode = false;
+  std::vector<PairTile> pairs;
+  std::vector<PairKV> kv;
+  std::vector<int32_t> order;  // pairs, most KV tiles first
+};
+void build_pairs(const Plan& plan, bool rows_mode, PairPlan* out);
+
 // Tile classes over an arbitrary grid: 0 empty, 1 full, 2 partial.
 void classify_tiles(int mask_kind, const uint8_t* block_map, int Nq, int Nkv, int tq, int tk,
                     uint8_t* out);

@@ -1,28 +1,39 @@
 // prefill_sm100.cu -- exact attention forward on sm_100a tensor cores.
 //
-// One CTA computes one 128-row Q tile of one (batch, query head): the fused,
-// tiled forward pass of "FlashAttention: memory-saving exact attention"
-// (section 3), in the Q-outer loop order, with block-sparse skipping
-// (section 6): the host plan lists only the live KV tiles of each Q tile.
+// The fused, tiled forward pass of "FlashAttention: memory-saving exact
+// attention" (section 3) in the Q-outer loop order, with block-sparse
+// skipping (section 6): the host plan lists only the live KV tiles of each Q
+// tile, and marks the few that need an element predicate.
 //
-// Roles (192 threads):
-//   warp 0      TMA producer: Q once, then K_j / V_j into a ring of stages.
-//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
-//               score buffers, and O += P_j V_j into a TMEM accumulator.
-//               Also owns the TMEM allocation.
-//   warps 2..5  softmax: one thread per query row.  Reads S_j from TMEM,
-//               applies the predicate on partial tiles only, updates the
-//               running max m and sum l (online softmax, FlashAttention page
-//               section 2; inference page "Online-Softmax"), writes P_j
-//               (bf16) to shared memory, rescales O in TMEM when m moved,
-//               and finally writes O / l and LSE.
+// Persistent CTAs (one per SM) walk a list of work items.  An item is two
+// 128-row Q tiles ("slots" A and B) that share every K/V tile loaded into
+// shared memory: two query heads of one GQA group on the same rows, or two Q
+// tiles of one head whose KV lists nest (slot A visits a prefix of slot B's
+// list).  While the softmax warps of one slot work, the tensor core runs the
+// other slot's GEMMs.
 //
-// The running max is only moved when the new row max exceeds it by more than
-// 2^8 in the exponent; otherwise the old base is kept and P may reach 256.
-// O and l are always scaled against the same base, so the result is exactly
-// softmax(S) V; the threshold only skips accumulator rescales.
+// Roles (384 threads, three warpgroups):
+//   warp 0        TMA producer: Q_A, Q_B once per item, then K_j, V_j into a
+//                 ring of shared-memory stages.
+//   warp 1        MMA issuer (one thread) and TMEM owner:
+//                   S_X = Q_X K_j^T      (A and B from shared memory)
+//                   O_X += P_X V_j       (P_X from TMEM, V_j from shared memory)
+//   warps 2, 3    idle.
+//   warps 4..7    softmax for slot A, one thread per query row.
+//   warps 8..11   softmax for slot B.
+// Each softmax thread reads its S row from TMEM in 32-column chunks, keeps the
+// running max m and sum l (online softmax: FlashAttention page section 2,
+// inference page "Online-Softmax"), packs P to bf16 in registers and writes it
+// back over the first 64 columns of its own S row, where the PV MMA reads it.
+// At the end of an item it writes O / l (bf16) and LSE.
 //
-// TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256, 256+d) O.
+// The exponent base moves only when a tile's row max exceeds it by more than
+// 8 (log2 units); P may then reach 2^8, with O and l scaled against the same
+// base, so the result is exactly softmax(S) V while most rescales vanish.
+//
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+d), O_B after O_A.
+// P_X is stored as bf16 pairs in S_X's first 64 columns; the MMA issuer
+// orders S_X(j+1) after PV_X(j) has completed, since they share columns.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -31,22 +42,21 @@
 namespace eio {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
 struct Cfg {
-  static constexpr int kStages = (D == 64) ? 4 : 2;
-  static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 64 bf16 (one swizzle span)
-  static constexpr int kTileBytes = 128 * D * 2;       // Q, K or V tile (128 rows)
-  static constexpr int kPBytes = 128 * 128 * 2;        // P tile (128 x 128 bf16)
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTileBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffP = kOffV + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffP + kPBytes;
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 1 + 1;
+  static constexpr int kRing = (D == 64) ? 10 : 4;       // K/V tiles in flight
+  static constexpr int kChunkBytes = 128 * 128;           // 128 rows x 64 bf16 (one swizzle span)
+  static constexpr int kTileBytes = 128 * D * 2;          // Q, K or V tile (128 rows)
+  static constexpr int kOffQ = 0;                         // Q_A, Q_B
+  static constexpr int kOffRing = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffRing + kRing * kTileBytes;
+  // q_full[2] q_empty[2] ring_full[R] ring_empty[R] s_full[2] p_full[2]
+  // pv_done[2] o_free[2] mma_idle
+  static constexpr int kNumBars = 4 + 2 * kRing + 8 + 1;
   static constexpr int kSmem = kOffBar + 8 * kNumBars + 16 + 1024;  // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -89,58 +99,88 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// One work item, decoded identically by every role.
+struct Item {
+  int b, hkv, headA, headB;
+  int rowA, nrowsA, rowB, nrowsB;
+  int kv_first, nA, nB;
+};
+
+__device__ __forceinline__ Item decode_item(const PrefillArgs& a, long long w) {
+  const long long per_rank = static_cast<long long>(a.B) * a.Hkv * a.HP;
+  const int rank = static_cast<int>(w / per_rank);
+  long long rem = w - rank * per_rank;
+  Item it;
+  it.b = static_cast<int>(rem / (static_cast<long long>(a.Hkv) * a.HP));
+  rem -= static_cast<long long>(it.b) * a.Hkv * a.HP;
+  it.hkv = static_cast<int>(rem / a.HP);
+  const int hp = static_cast<int>(rem - static_cast<long long>(it.hkv) * a.HP);
+  const int p = a.order[rank];
+  const int4 x0 = a.pairs[2 * p];
+  const int4 x1 = a.pairs[2 * p + 1];
+  it.rowA = x0.x;
+  it.nrowsA = x0.y;
+  it.rowB = x0.z;
+  it.nrowsB = x0.w;
+  it.kv_first = x1.x;
+  it.nA = x1.y;
+  it.nB = x1.z;
+  if (a.rows_mode) {
+    it.headA = it.headB = it.hkv;  // one query head per KV head
+  } else {
+    it.headA = it.hkv * a.G + 2 * hp;
+    if (2 * hp + 1 < a.G) {
+      it.headB = it.headA + 1;
+    } else {  // odd group: its last head runs alone in slot B
+      it.headB = it.headA;
+      it.nrowsA = 0;
+      it.nA = 0;
+    }
+  }
+  return it;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
   using C = Cfg<D>;
-  constexpr int S = C::kStages;
+  constexpr int R = C::kRing;
   constexpr int NCH = D / 64;  // 64-element swizzle chunks per row
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* v_full = k_full + S;
-  uint64_t* k_empty = v_full + S;
-  uint64_t* v_empty = k_empty + S;
-  uint64_t* s_full = v_empty + S;   // [2]
-  uint64_t* s_free = s_full + 2;    // [2]
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* mma_idle = pv_done + 1;
+  uint64_t* q_full = bars;            // [2]
+  uint64_t* q_empty = bars + 2;       // [2]
+  uint64_t* ring_full = bars + 4;     // [R]
+  uint64_t* ring_empty = ring_full + R;
+  uint64_t* s_full = ring_empty + R;  // [2]
+  uint64_t* p_full = s_full + 2;      // [2]
+  uint64_t* pv_done = p_full + 2;     // [2]
+  uint64_t* o_free = pv_done + 2;     // [2]
+  uint64_t* mma_idle = o_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int bh = a.B * a.Hq;
-  const int rank = blockIdx.x / bh;
-  const int rem = blockIdx.x - rank * bh;
-  const int b = rem / a.Hq;
-  const int hq = rem - b * a.Hq;
-  const int hkv = hq / (a.Hq / a.Hkv);
-  const int4 qt = a.qtiles[a.order[rank]];
-  const int q_row0 = qt.x, q_rows = qt.y, kv_first = qt.z, n_kv = qt.w;
-
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int i = 0; i < S; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-      mbar_init(&v_empty[i], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 4);
+      mbar_init(&pv_done[x], 1);
+      mbar_init(&o_free[x], 4);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+    for (int i = 0; i < R; ++i) {
+      mbar_init(&ring_full[i], 1);
+      mbar_init(&ring_empty[i], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     mbar_init(mma_idle, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -160,126 +200,163 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   const uint32_t sQ = smem_u32(smem + C::kOffQ);
-  const uint32_t sK = smem_u32(smem + C::kOffK);
-  const uint32_t sV = smem_u32(smem + C::kOffV);
-  const uint32_t sP = smem_u32(smem + C::kOffP);
+  const uint32_t sRing = smem_u32(smem + C::kOffRing);
+  const long long n_items = a.n_items;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_kv > 0) {
+    if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, C::kTileBytes);
+      uint32_t seq = 0;
+      uint32_t qcnt[2] = {0, 0};
+      bool ok = true;
+      for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+        const Item it = decode_item(a, w);
+        const int nX[2] = {it.nA, it.nB};
+        const int rowX[2] = {it.rowA, it.rowB};
+        const int headX[2] = {it.headA, it.headB};
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (nX[x] == 0) continue;
+          if (qcnt[x] > 0 && (*abort_flag || !mbar_wait(&q_empty[x], (qcnt[x] - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&q_full[x], C::kTileBytes);
 #pragma unroll
-      for (int ch = 0; ch < NCH; ++ch)
-        tma_load_4d(smem + C::kOffQ + ch * C::kChunkBytes, &tmQ, q_full, ch * 64, hq, q_row0, b);
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        if (*abort_flag) break;
-        const int4 kt = a.kvtiles[kv_first + j];
-        const int st = j % S;
-        const uint32_t ph_empty = ((j / S) + 1) & 1;
-        if (j >= S && !mbar_wait(&k_empty[st], ph_empty)) {
-          fail(kErrDeviceTimeout);
-          break;
+          for (int ch = 0; ch < NCH; ++ch)
+            tma_load_4d(smem + C::kOffQ + x * C::kTileBytes + ch * C::kChunkBytes, &tmQ, &q_full[x],
+                        ch * 64, headX[x], rowX[x], it.b);
+          qcnt[x]++;
         }
-        mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
+        for (int j = 0; ok && j < it.nB; ++j) {
+          const int4 kt = a.kvtiles[it.kv_first + j];
+          for (int t = 0; t < 2; ++t) {
+            const uint32_t slot = seq % R;
+            if (seq >= R && (*abort_flag || !mbar_wait(&ring_empty[slot], ((seq / R) + 1) & 1))) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&ring_full[slot], C::kTileBytes);
+            const CUtensorMap* map = t == 0 ? &tmK : &tmV;
 #pragma unroll
-        for (int ch = 0; ch < NCH; ++ch)
-          tma_load_4d(smem + C::kOffK + st * C::kTileBytes + ch * C::kChunkBytes, &tmK, &k_full[st],
-                      ch * 64, hkv, kt.x, b);
-        k_issued = j + 1;
-        if (j >= S && !mbar_wait(&v_empty[st], ph_empty)) {
-          fail(kErrDeviceTimeout);
-          break;
+            for (int ch = 0; ch < NCH; ++ch)
+              tma_load_4d(smem + C::kOffRing + slot * C::kTileBytes + ch * C::kChunkBytes, map,
+                          &ring_full[slot], ch * 64, it.hkv, kt.x, it.b);
+            ++seq;
+          }
         }
-        mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
-#pragma unroll
-        for (int ch = 0; ch < NCH; ++ch)
-          tma_load_4d(smem + C::kOffV + st * C::kTileBytes + ch * C::kChunkBytes, &tmV, &v_full[st],
-                      ch * 64, hkv, kt.x, b);
-        v_issued = j + 1;
       }
-      if (*abort_flag) {
+      if (!ok) {
+        fail(kErrDeviceTimeout);
         // Let every copy this thread started land before the CTA retires.
-        mbar_wait(q_full, 0);
-        for (int j = k_issued - S < 0 ? 0 : k_issued - S; j < k_issued; ++j)
-          mbar_wait(&k_full[j % S], (j / S) & 1);
-        for (int j = v_issued - S < 0 ? 0 : v_issued - S; j < v_issued; ++j)
-          mbar_wait(&v_full[j % S], (j / S) & 1);
+        for (int x = 0; x < 2; ++x)
+          if (qcnt[x] > 0) mbar_wait(&q_full[x], (qcnt[x] - 1) & 1);
+        for (uint32_t s = seq > R ? seq - R : 0; s < seq; ++s)
+          mbar_wait(&ring_full[s % R], (s / R) & 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_kv > 0) {
-      const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);  // A = P (K-major), B = V (MN-major)
-      bool ok = mbar_wait(q_full, 0);
-      if (!ok) fail(kErrDeviceTimeout);
-      tc_fence_after();
+    if (lane == 0) {
+      const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);  // A = P (TMEM), B = V (MN-major)
+      uint32_t seq = 0;
+      uint32_t qcnt[2] = {0, 0}, scnt[2] = {0, 0}, pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
+      bool ok = true;
 
-      auto issue_s = [&](int j) -> bool {
-        const int4 kt = a.kvtiles[kv_first + j];
-        const int st = j % S;
-        if (*abort_flag) return false;
-        if (!mbar_wait(&k_full[st], (j / S) & 1)) return false;
-        if (j >= 2 && !mbar_wait(&s_free[j & 1], ((j >> 1) - 1) & 1)) return false;
+      auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
+        if (!ok) return false;
+        if (*abort_flag || !mbar_wait(bar, parity)) ok = false;
+        return ok;
+      };
+      // S_X = Q_X K^T for the K tile in ring slot kslot.
+      auto issue_s = [&](int x, int ncols, uint32_t kslot) {
+        if (scnt[x] > 0 && !wait_bar(&pv_done[x], (pcnt[x] - 1) & 1)) return;  // P_X shares S_X
         tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>((j & 1) * 128);
-        const uint32_t id = idesc_bf16_f32(128, static_cast<uint32_t>(kt.y), 0, 0);
-        const uint32_t kbase = sK + st * C::kTileBytes;
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(x * 128);
+        const uint32_t id = idesc_bf16_f32(128, static_cast<uint32_t>(ncols), 0, 0);
+        const uint32_t qbase = sQ + x * C::kTileBytes;
+        const uint32_t kbase = sRing + kslot * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          mma_bf16_ss(d_tmem, sdesc_sw128(sQ + koff, 16, 1024), sdesc_sw128(kbase + koff, 16, 1024),
-                      id, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(d_tmem, sdesc_sw128(qbase + koff, 16, 1024),
+                      sdesc_sw128(kbase + koff, 16, 1024), id, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[j & 1]);
-        mma_commit(&k_empty[st]);
-        return true;
+        mma_commit(&s_full[x]);
+        scnt[x]++;
       };
-      auto issue_pv = [&](int j) -> bool {
-        const int4 kt = a.kvtiles[kv_first + j];
-        const int st = j % S;
-        if (*abort_flag) return false;
-        if (!mbar_wait(p_full, j & 1)) return false;
-        if (!mbar_wait(&v_full[st], (j / S) & 1)) return false;
+      // O_X (+)= P_X V for the V tile in ring slot vslot.
+      auto issue_pv = [&](int x, int j, int nX, int ncols, uint32_t vslot) {
+        if (!wait_bar(&p_full[x], pcnt[x] & 1)) return;
+        if (j == 0 && ocnt[x] > 0 && !wait_bar(&o_free[x], (ocnt[x] - 1) & 1)) return;
         tc_fence_after();
-        const uint32_t vbase = sV + st * C::kTileBytes;
-        const int ksteps = kt.y >> 4;
-        for (int kk = 0; kk < ksteps; ++kk) {
-          const uint32_t poff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          // V: 16 kv rows per step (2 groups of 8 rows at 1024 B); the two
-          // 64-wide d chunks are C::kChunkBytes apart (leading byte offset).
-          mma_bf16_ss(tmem + 256, sdesc_sw128(sP + poff, 16, 1024),
-                      sdesc_sw128(vbase + kk * 2048, C::kChunkBytes, 1024), idO,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(pv_done);
-        mma_commit(&v_empty[st]);
-        return true;
+        const uint32_t p_tmem = tmem + static_cast<uint32_t>(x * 128);
+        const uint32_t o_tmem = tmem + static_cast<uint32_t>(256 + x * D);
+        const uint32_t vbase = sRing + vslot * C::kTileBytes;
+        const int ksteps = ncols >> 4;
+        for (int kk = 0; kk < ksteps; ++kk)
+          mma_bf16_ts(o_tmem, p_tmem + kk * 8, sdesc_sw128(vbase + kk * 2048, C::kChunkBytes, 1024),
+                      idO, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&pv_done[x]);
+        pcnt[x]++;
+        if (j == nX - 1) ocnt[x]++;
       };
 
-      if (ok) ok = issue_s(0);
-      for (int j = 1; ok && j < n_kv; ++j) {
-        ok = issue_s(j);
-        if (ok) ok = issue_pv(j - 1);
+      for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+        const Item it = decode_item(a, w);
+        const int nA = it.nA, nB = it.nB;
+        if (nA > 0 && wait_bar(&q_full[0], qcnt[0] & 1)) qcnt[0]++;
+        if (nB > 0 && wait_bar(&q_full[1], qcnt[1] & 1)) qcnt[1]++;
+        if (!ok || nB == 0) continue;
+        const int4* kv = a.kvtiles + it.kv_first;
+        // tile 0: S_A, S_B
+        if (!wait_bar(&ring_full[seq % R], (seq / R) & 1)) break;
+        if (nA > 0) issue_s(0, kv[0].y, seq % R);
+        issue_s(1, kv[0].y, seq % R);
+        if (!ok) break;
+        mma_commit(&ring_empty[seq % R]);
+        for (int j = 0; ok && j < nB; ++j) {
+          const uint32_t vseq = seq + 2 * j + 1, kseq = vseq + 1;
+          const int ncj = kv[j].y;
+          if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
+          const bool next = j + 1 < nB;
+          const int ncn = next ? kv[j + 1].y : 0;
+          if (j < nA) {
+            issue_pv(0, j, nA, ncj, vseq % R);
+            if (j + 1 < nA && wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) issue_s(0, ncn, kseq % R);
+          }
+          issue_pv(1, j, nB, ncj, vseq % R);
+          if (!ok) break;
+          mma_commit(&ring_empty[vseq % R]);
+          if (next) {
+            if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
+            issue_s(1, ncn, kseq % R);
+            if (!ok) break;
+            mma_commit(&ring_empty[kseq % R]);
+          }
+        }
+        seq += 2 * nB;
+        if (!ok) break;
+        if (nA > 0) mma_commit(&q_empty[0]);
+        mma_commit(&q_empty[1]);
       }
-      if (ok) ok = issue_pv(n_kv - 1);
       if (!ok) fail(kErrDeviceTimeout);
       // Every MMA issued above has finished before TMEM is released.
       mma_commit(mma_idle);
       mbar_wait(mma_idle, 0);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
+    const int x = (warp - 4) >> 2;  // slot
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int grow = q_row0 + row;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_tmem = tmem + lane_off + static_cast<uint32_t>(x * 128);
+    const uint32_t o_tmem = tmem + lane_off + static_cast<uint32_t>(256 + x * D);
     const float sl2 = a.scale_log2;
-    float m_b = -INFINITY;  // exponent base, log2 units (scaled)
-    float l = 0.f;
+    uint32_t tcnt = 0;
     bool ok = true;
     // Waits and the abort decision are made warp-uniform, because the warp
     // then executes .sync.aligned tcgen05 instructions together.
@@ -288,174 +365,167 @@ __global__ void __launch_bounds__(kThreads, 1)
       return __all_sync(0xffffffffu, mine);
     };
 
-    for (int j = 0; j < n_kv; ++j) {
-      const int4 kt = a.kvtiles[kv_first + j];
-      const int nc = kt.y;
-      if (!warp_wait(&s_full[j & 1], (j >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sr[128];
-      const uint32_t sbase = tmem + lane_off + static_cast<uint32_t>((j & 1) * 128);
-      const bool full = nc == 128 && !kt.z;
-      if (full) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(sbase + c * 32, sr + c * 32);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          if (c * 16 < nc) tmem_ld16(sbase + c * 16, sr + c * 16);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[j & 1]);
+    for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+      const Item it = decode_item(a, w);
+      const int nX = x == 0 ? it.nA : it.nB;
+      const int nrows = x == 0 ? it.nrowsA : it.nrowsB;
+      const int row0 = x == 0 ? it.rowA : it.rowB;
+      const int head = x == 0 ? it.headA : it.headB;
+      if (nrows == 0) continue;  // slot unused in this item
+      const int grow = row0 + row;
+      const int4* kv = a.kvtiles + it.kv_first;
+      float m_b = -INFINITY;  // exponent base, log2 units
+      float l = 0.f;
 
-      // Predicate: only on partial tiles and on columns past a narrow tile.
-      if (!full) {
-        int lim = nc;  // allowed iff c < lim
-        if (kt.z) {
-          const int c0 = kt.x;
-          lim = min(lim, a.Nkv - c0);
-          if (a.causal) lim = min(lim, grow + a.causal_off + 1 - c0);
+      for (int t = 0; t < nX; ++t) {
+        const int4 kt = kv[t];
+        const int nc = kt.y;
+        if (!warp_wait(&s_full[x], tcnt & 1)) {
+          ok = false;
+          break;
         }
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
-      }
-      // Row max: four independent chains of 3-input max.
-      float mx4[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        float m = __uint_as_float(sr[t * 32]);
-#pragma unroll
-        for (int c = 1; c < 31; c += 2)
-          m = max3f(m, __uint_as_float(sr[t * 32 + c]), __uint_as_float(sr[t * 32 + c + 1]));
-        mx4[t] = fmaxf(m, __uint_as_float(sr[t * 32 + 31]));
-      }
-      const float mx = max3f(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
-      const float mx_s = mx * sl2;
-      const bool upd = mx_s > m_b + kRescaleThreshold;
-      const float m_new = upd ? mx_s : m_b;
-      const float alpha = upd ? ex2(m_b - m_new) : 1.0f;
-      const float base = (m_new == -INFINITY) ? 0.f : m_new;
+        tc_fence_after();
+        // Columns at or past `lim` are masked: past the tile width always,
+        // and on partial tiles past Nkv and past the causal diagonal.
+        int lim = nc;
+        if ((kt.z >> x) & 1) {
+          lim = min(lim, a.Nkv - kt.x);
+          if (a.causal) lim = min(lim, grow + a.causal_off + 1 - kt.x);
+        }
+        const bool need_mask = __any_sync(0xffffffffu, lim < 128);
 
-      // p = 2^(s * scale*log2e - base), packed two at a time; row sum in
-      // four independent pairs of accumulators.
-      float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-      uint32_t pk[64];
+        auto load_chunk = [&](int c, uint32_t* r) {
+          tmem_ld32(s_tmem + c * 32, r);
+          tmem_wait_ld();
+          if (need_mask) {
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float2 t = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
-                               make_float2(sl2, sl2), make_float2(-base, -base));
-        const float2 p = make_float2(ex2(t.x), ex2(t.y));
-        acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], p);
-        pk[c >> 1] = pack_bf16x2(p.x, p.y);
-      }
-      const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-      const float sum = s01.x + s01.y;
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i >= lim) r[i] = __float_as_uint(-INFINITY);
+          }
+        };
+        auto chunk_max = [&](const uint32_t* r) {
+          float m0 = max3f(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
+          float m1 = max3f(__uint_as_float(r[3]), __uint_as_float(r[4]), __uint_as_float(r[5]));
+#pragma unroll
+          for (int i = 6; i < 30; i += 4) {
+            m0 = max3f(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+            m1 = max3f(m1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+          }
+          return max3f(m0, m1, fmaxf(__uint_as_float(r[30]), __uint_as_float(r[31])));
+        };
+        uint32_t pk[64];
+        float2 acc[4];
+        float mx = -INFINITY;
+        // p = 2^(s * scale*log2e - base) packed into pk; row sum into acc.
+        auto exp_pass = [&](float base, bool track_max) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+          const float2 sl = make_float2(sl2, sl2), nb = make_float2(-base, -base);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            load_chunk(c, r);
+            if (track_max) mx = fmaxf(mx, chunk_max(r));
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float2 e = ffma2(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), sl, nb);
+              const float2 p = make_float2(ex2(e.x), ex2(e.y));
+              acc[(i >> 1) & 3] = fadd2(acc[(i >> 1) & 3], p);
+              pk[c * 16 + (i >> 1)] = pack_bf16x2(p.x, p.y);
+            }
+          }
+        };
 
-      // P buffer and O are free once PV_{j-1} has completed.
-      if (j > 0) {
-        if (!warp_wait(pv_done, (j - 1) & 1)) {
+        // A row with no base yet (first tile of the item, or all masked so
+        // far) takes this tile's max first; the warp does it together.
+        if (__any_sync(0xffffffffu, m_b == -INFINITY)) {
+          float m = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            load_chunk(c, r);
+            m = fmaxf(m, chunk_max(r));
+          }
+          if (m_b == -INFINITY) m_b = m * sl2;
+        }
+        exp_pass(m_b == -INFINITY ? 0.f : m_b, true);
+        const float mx_s = mx * sl2;
+        const bool upd = mx_s > m_b + kRescaleThreshold;
+        float alpha = 1.f;
+        if (__any_sync(0xffffffffu, upd)) {
+          // Rare: the max grew by more than 2^8; redo with the new base.
+          if (upd) {
+            alpha = ex2(m_b - mx_s);
+            m_b = mx_s;
+          }
+          exp_pass(m_b == -INFINITY ? 0.f : m_b, false);
+          if (t > 0) {  // O holds earlier tiles: rescale it (PV_{t-1} has completed)
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              uint32_t orr[32];
+              tmem_ld32(o_tmem + c, orr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+              tmem_st32(o_tmem + c, orr);
+            }
+          }
+        }
+        const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+        l = l * alpha + (s01.x + s01.y);
+        // P over the first 64 columns of this S row.
+        tmem_st32(s_tmem, pk);
+        tmem_st32(s_tmem + 32, pk + 32);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[x]);
+        tcnt++;
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue
+      if (nX > 0) {
+        if (!warp_wait(&pv_done[x], (tcnt - 1) & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
       }
-      uint8_t* prow = smem + C::kOffP + row * 128;
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (ch * 64 + u * 8 < nc)
-            *reinterpret_cast<uint4*>(prow + ch * C::kChunkBytes + ((u ^ (row & 7)) << 4)) =
-                make_uint4(pk[ch * 32 + u * 4 + 0], pk[ch * 32 + u * 4 + 1],
-                           pk[ch * 32 + u * 4 + 2], pk[ch * 32 + u * 4 + 3]);
-      fence_proxy_async_smem();
-
-      if (j > 0 && __any_sync(0xffffffffu, upd)) {
-        const uint32_t obase = tmem + lane_off + 256;
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t orr[32];
-          tmem_ld32(obase + c, orr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-          tmem_st32(obase + c, orr);
-        }
-        tmem_wait_st();
-      }
-      l = l * alpha + sum;
-      m_b = m_new;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-
-    if (!ok) {
-      fail(kErrDeviceTimeout);
-    } else {
-      if (n_kv > 0) {
-        if (!warp_wait(pv_done, (n_kv - 1) & 1)) {
-          fail(kErrDeviceTimeout);
-          ok = false;
-        }
-        tc_fence_after();
-      }
-    }
-    if (ok) {
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-      const float lse_val = l > 0.f ? (m_b + __log2f(l)) * kLn2 : -INFINITY;
-      // Stage the bf16 O row in the (now idle) P buffer, 16-byte units
-      // XOR-swizzled by row to keep the shared-memory banks apart.
-      constexpr int UPR = D / 8;  // 16-byte units per row
-      uint8_t* stg = smem + C::kOffP;
-      const uint32_t obase = tmem + lane_off + 256;
+      const bool valid = row < nrows;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(a.o) +
+                      2 * (((static_cast<size_t>(it.b) * a.Nq + grow) * a.Hq + head) * D);
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t orr[32];
-        if (n_kv > 0) {
-          tmem_ld32(obase + c, orr);
+        if (nX > 0) {
+          tmem_ld32(o_tmem + c, orr);
           tmem_wait_ld();
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) orr[i] = 0u;
         }
+        if (valid) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = c / 8 + u;
-          const int sw = (unit & ~7) | ((unit & 7) ^ (row & 7));
-          *reinterpret_cast<uint4*>(stg + row * (D * 2) + sw * 16) = make_uint4(
-              pack_bf16x2(__uint_as_float(orr[u * 8 + 0]) * inv_l,
-                          __uint_as_float(orr[u * 8 + 1]) * inv_l),
-              pack_bf16x2(__uint_as_float(orr[u * 8 + 2]) * inv_l,
-                          __uint_as_float(orr[u * 8 + 3]) * inv_l),
-              pack_bf16x2(__uint_as_float(orr[u * 8 + 4]) * inv_l,
-                          __uint_as_float(orr[u * 8 + 5]) * inv_l),
-              pack_bf16x2(__uint_as_float(orr[u * 8 + 6]) * inv_l,
-                          __uint_as_float(orr[u * 8 + 7]) * inv_l));
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(orow + 2 * (c + u * 8)) = make_uint4(
+                pack_bf16x2(__uint_as_float(orr[u * 8 + 0]) * inv_l, __uint_as_float(orr[u * 8 + 1]) * inv_l),
+                pack_bf16x2(__uint_as_float(orr[u * 8 + 2]) * inv_l, __uint_as_float(orr[u * 8 + 3]) * inv_l),
+                pack_bf16x2(__uint_as_float(orr[u * 8 + 4]) * inv_l, __uint_as_float(orr[u * 8 + 5]) * inv_l),
+                pack_bf16x2(__uint_as_float(orr[u * 8 + 6]) * inv_l, __uint_as_float(orr[u * 8 + 7]) * inv_l));
         }
       }
-      __syncwarp();
-      constexpr int RPI = 32 / UPR;  // rows per warp-wide store
-      uint8_t* obytes = reinterpret_cast<uint8_t*>(a.o);
-#pragma unroll 4
-      for (int it = 0; it < 32 / RPI; ++it) {
-        const int r = quarter * 32 + it * RPI + lane / UPR;
-        const int unit = lane % UPR;
-        if (r < q_rows) {
-          const int sw = (unit & ~7) | ((unit & 7) ^ (r & 7));
-          const uint4 val = *reinterpret_cast<const uint4*>(stg + r * (D * 2) + sw * 16);
-          const size_t off = ((static_cast<size_t>(b) * a.Nq + q_row0 + r) * a.Hq + hq) * D + unit * 8;
-          *reinterpret_cast<uint4*>(obytes + off * 2) = val;
-        }
+      if (nX > 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[x]);
       }
-      if (a.lse != nullptr && row < q_rows)
-        a.lse[(static_cast<size_t>(b) * a.Hq + hq) * a.Nq + grow] = lse_val;
+      if (a.lse != nullptr && valid)
+        a.lse[(static_cast<size_t>(it.b) * a.Hq + head) * a.Nq + grow] =
+            l > 0.f ? (m_b + __log2f(l)) * kLn2 : -INFINITY;
     }
+    if (!ok) fail(kErrDeviceTimeout);
   }
 
   tc_fence_before();
@@ -467,15 +537,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const PrefillArgs& a, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  static int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
     cudaError_t e = cudaFuncSetAttribute(prefill_bf16_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_dev = dev;
   }
-  const long long grid = static_cast<long long>(a.n_qtiles) * a.B * a.Hq;
-  if (grid == 0) return cudaSuccess;
+  if (a.n_items == 0) return cudaSuccess;
+  const long long grid = a.n_items < a.num_ctas ? a.n_items : a.num_ctas;
   prefill_bf16_kernel<D><<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmem, s>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
