@@ -12,20 +12,22 @@
 // list).  While the softmax warps of one slot work, the tensor core runs the
 // other slot's GEMMs.
 //
-// Roles (384 threads, three warpgroups):
-//   warp 0        TMA producer: Q_A, Q_B once per item, then K_j, V_j into a
-//                 ring of shared-memory stages.
+// Roles (384 threads, three warpgroups; the first gives registers to the
+// two softmax warpgroups with setmaxnreg: 128 x 72 + 256 x 216 = 384 x 168):
+//   warp 0        TMA producer: Q_A, Q_B once per item (double-buffered for
+//                 d = 64, whose items are short), then K_j, V_j into a ring of
+//                 shared-memory stages.
 //   warp 1        MMA issuer (one thread) and TMEM owner:
 //                   S_X = Q_X K_j^T      (A and B from shared memory)
 //                   O_X += P_X V_j       (P_X from TMEM, V_j from shared memory)
 //   warps 2, 3    idle.
 //   warps 4..7    softmax for slot A, one thread per query row.
 //   warps 8..11   softmax for slot B.
-// Each softmax thread reads its S row from TMEM in 32-column chunks, keeps the
-// running max m and sum l (online softmax: FlashAttention page section 2,
-// inference page "Online-Softmax"), packs P to bf16 in registers and writes it
-// back over the first 64 columns of its own S row, where the PV MMA reads it.
-// At the end of an item it writes O / l (bf16) and LSE.
+// Each softmax thread loads its whole S row from TMEM (one wait), takes the
+// row max, keeps the running max m and sum l (online softmax: FlashAttention
+// page section 2, inference page "Online-Softmax"), packs P to bf16 in place
+// and writes it back over the first 64 columns of its own S row, where the PV
+// MMA reads it.  At the end of an item it writes O / l (bf16) and LSE.
 //
 // The exponent base moves only when a tile's row max exceeds it by more than
 // 8 (log2 units); P may then reach 2^8, with O and l scaled against the same
@@ -43,20 +45,29 @@ namespace eio {
 namespace {
 
 constexpr int kThreads = 384;
+// Register split between the warpgroups.  The kernel must be compiled to
+// exactly kLaunchRegs registers per thread: the host refuses to launch it
+// otherwise, since an increase that the pool cannot cover never returns.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsControl = 72;   // warpgroup 0: producer, MMA issuer
+constexpr int kRegsSoftmax = 216;  // warpgroups 1 and 2
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
+              "register split must fit in the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
 struct Cfg {
-  static constexpr int kRing = (D == 64) ? 10 : 4;       // K/V tiles in flight
+  static constexpr int kQBuf = (D == 64) ? 2 : 1;         // Q buffers per slot
+  static constexpr int kRing = (D == 64) ? 8 : 4;         // K/V tiles in flight
   static constexpr int kChunkBytes = 128 * 128;           // 128 rows x 64 bf16 (one swizzle span)
   static constexpr int kTileBytes = 128 * D * 2;          // Q, K or V tile (128 rows)
-  static constexpr int kOffQ = 0;                         // Q_A, Q_B
-  static constexpr int kOffRing = 2 * kTileBytes;
+  static constexpr int kOffQ = 0;                         // Q[slot][buffer]
+  static constexpr int kOffRing = 2 * kQBuf * kTileBytes;
   static constexpr int kOffBar = kOffRing + kRing * kTileBytes;
-  // q_full[2] q_empty[2] ring_full[R] ring_empty[R] s_full[2] p_full[2]
+  // q_full[2*QB] q_empty[2*QB] ring_full[R] ring_empty[R] s_full[2] p_full[2]
   // pv_done[2] o_free[2] mma_idle
-  static constexpr int kNumBars = 4 + 2 * kRing + 8 + 1;
+  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 1;
   static constexpr int kSmem = kOffBar + 8 * kNumBars + 16 + 1024;  // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -153,9 +164,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* q_full = bars;            // [2]
-  uint64_t* q_empty = bars + 2;       // [2]
-  uint64_t* ring_full = bars + 4;     // [R]
+  constexpr int QB = C::kQBuf;
+  uint64_t* q_full = bars;            // [2][QB]
+  uint64_t* q_empty = bars + 2 * QB;  // [2][QB]
+  uint64_t* ring_full = bars + 4 * QB;  // [R]
   uint64_t* ring_empty = ring_full + R;
   uint64_t* s_full = ring_empty + R;  // [2]
   uint64_t* p_full = s_full + 2;      // [2]
@@ -169,9 +181,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * QB; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&q_full[x], 1);
-      mbar_init(&q_empty[x], 1);
       mbar_init(&s_full[x], 1);
       mbar_init(&p_full[x], 4);
       mbar_init(&pv_done[x], 1);
@@ -203,6 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sRing = smem_u32(smem + C::kOffRing);
   const long long n_items = a.n_items;
 
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -219,15 +235,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int headX[2] = {it.headA, it.headB};
         for (int x = 0; x < 2 && ok; ++x) {
           if (nX[x] == 0) continue;
-          if (qcnt[x] > 0 && (*abort_flag || !mbar_wait(&q_empty[x], (qcnt[x] - 1) & 1))) {
+          const uint32_t qb = qcnt[x] % QB, use = qcnt[x] / QB;
+          if (use > 0 && (*abort_flag || !mbar_wait(&q_empty[x * QB + qb], (use - 1) & 1))) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&q_full[x], C::kTileBytes);
+          mbar_arrive_expect_tx(&q_full[x * QB + qb], C::kTileBytes);
 #pragma unroll
           for (int ch = 0; ch < NCH; ++ch)
-            tma_load_4d(smem + C::kOffQ + x * C::kTileBytes + ch * C::kChunkBytes, &tmQ, &q_full[x],
-                        ch * 64, headX[x], rowX[x], it.b);
+            tma_load_4d(smem + C::kOffQ + (x * QB + qb) * C::kTileBytes + ch * C::kChunkBytes, &tmQ,
+                        &q_full[x * QB + qb], ch * 64, headX[x], rowX[x], it.b);
           qcnt[x]++;
         }
         for (int j = 0; ok && j < it.nB; ++j) {
@@ -252,7 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         fail(kErrDeviceTimeout);
         // Let every copy this thread started land before the CTA retires.
         for (int x = 0; x < 2; ++x)
-          if (qcnt[x] > 0) mbar_wait(&q_full[x], (qcnt[x] - 1) & 1);
+          for (uint32_t c = qcnt[x] > QB ? qcnt[x] - QB : 0; c < qcnt[x]; ++c)
+            mbar_wait(&q_full[x * QB + c % QB], (c / QB) & 1);
         for (uint32_t s = seq > R ? seq - R : 0; s < seq; ++s)
           mbar_wait(&ring_full[s % R], (s / R) & 1);
       }
@@ -271,12 +289,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         return ok;
       };
       // S_X = Q_X K^T for the K tile in ring slot kslot.
+      uint32_t qbuf[2] = {0, 0};
       auto issue_s = [&](int x, int ncols, uint32_t kslot) {
         if (scnt[x] > 0 && !wait_bar(&pv_done[x], (pcnt[x] - 1) & 1)) return;  // P_X shares S_X
         tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(x * 128);
         const uint32_t id = idesc_bf16_f32(128, static_cast<uint32_t>(ncols), 0, 0);
-        const uint32_t qbase = sQ + x * C::kTileBytes;
+        const uint32_t qbase = sQ + (x * QB + qbuf[x]) * C::kTileBytes;
         const uint32_t kbase = sRing + kslot * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -307,8 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
         const Item it = decode_item(a, w);
         const int nA = it.nA, nB = it.nB;
-        if (nA > 0 && wait_bar(&q_full[0], qcnt[0] & 1)) qcnt[0]++;
-        if (nB > 0 && wait_bar(&q_full[1], qcnt[1] & 1)) qcnt[1]++;
+        for (int x = 0; x < 2; ++x) {
+          if ((x == 0 ? nA : nB) == 0) continue;
+          qbuf[x] = qcnt[x] % QB;
+          if (wait_bar(&q_full[x * QB + qbuf[x]], (qcnt[x] / QB) & 1)) qcnt[x]++;
+        }
         if (!ok || nB == 0) continue;
         const int4* kv = a.kvtiles + it.kv_first;
         // tile 0: S_A, S_B
@@ -339,15 +361,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         seq += 2 * nB;
         if (!ok) break;
-        if (nA > 0) mma_commit(&q_empty[0]);
-        mma_commit(&q_empty[1]);
+        if (nA > 0) mma_commit(&q_empty[qbuf[0]]);
+        mma_commit(&q_empty[QB + qbuf[1]]);
       }
       if (!ok) fail(kErrDeviceTimeout);
       // Every MMA issued above has finished before TMEM is released.
       mma_commit(mma_idle);
       mbar_wait(mma_idle, 0);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax
     const int x = (warp - 4) >> 2;  // slot
     const int quarter = warp & 3;
@@ -392,90 +416,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           lim = min(lim, a.Nkv - kt.x);
           if (a.causal) lim = min(lim, grow + a.causal_off + 1 - kt.x);
         }
-        const bool need_mask = __any_sync(0xffffffffu, lim < 128);
-
-        auto load_chunk = [&](int c, uint32_t* r) {
-          tmem_ld32(s_tmem + c * 32, r);
-          tmem_wait_ld();
-          if (need_mask) {
+        uint32_t sr[128];
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c * 32 + i >= lim) r[i] = __float_as_uint(-INFINITY);
-          }
-        };
-        auto chunk_max = [&](const uint32_t* r) {
-          float m0 = max3f(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
-          float m1 = max3f(__uint_as_float(r[3]), __uint_as_float(r[4]), __uint_as_float(r[5]));
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_tmem + c * 32, sr + c * 32);
+        tmem_wait_ld();
+        if (__any_sync(0xffffffffu, lim < 128)) {
 #pragma unroll
-          for (int i = 6; i < 30; i += 4) {
-            m0 = max3f(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-            m1 = max3f(m1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-          }
-          return max3f(m0, m1, fmaxf(__uint_as_float(r[30]), __uint_as_float(r[31])));
-        };
-        uint32_t pk[64];
-        float2 acc[4];
-        float mx = -INFINITY;
-        // p = 2^(s * scale*log2e - base) packed into pk; row sum into acc.
-        auto exp_pass = [&](float base, bool track_max) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
-          const float2 sl = make_float2(sl2, sl2), nb = make_float2(-base, -base);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            load_chunk(c, r);
-            if (track_max) mx = fmaxf(mx, chunk_max(r));
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              const float2 e = ffma2(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), sl, nb);
-              const float2 p = make_float2(ex2(e.x), ex2(e.y));
-              acc[(i >> 1) & 3] = fadd2(acc[(i >> 1) & 3], p);
-              pk[c * 16 + (i >> 1)] = pack_bf16x2(p.x, p.y);
-            }
-          }
-        };
-
-        // A row with no base yet (first tile of the item, or all masked so
-        // far) takes this tile's max first; the warp does it together.
-        if (__any_sync(0xffffffffu, m_b == -INFINITY)) {
-          float m = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            load_chunk(c, r);
-            m = fmaxf(m, chunk_max(r));
-          }
-          if (m_b == -INFINITY) m_b = m * sl2;
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
         }
-        exp_pass(m_b == -INFINITY ? 0.f : m_b, true);
-        const float mx_s = mx * sl2;
+        // Row max: four independent chains of 3-input max.
+        float mx4[4];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float m = __uint_as_float(sr[q4 * 32]);
+#pragma unroll
+          for (int c = 1; c < 31; c += 2)
+            m = max3f(m, __uint_as_float(sr[q4 * 32 + c]), __uint_as_float(sr[q4 * 32 + c + 1]));
+          mx4[q4] = fmaxf(m, __uint_as_float(sr[q4 * 32 + 31]));
+        }
+        const float mx_s = max3f(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * sl2;
         const bool upd = mx_s > m_b + kRescaleThreshold;
-        float alpha = 1.f;
-        if (__any_sync(0xffffffffu, upd)) {
-          // Rare: the max grew by more than 2^8; redo with the new base.
-          if (upd) {
-            alpha = ex2(m_b - mx_s);
-            m_b = mx_s;
-          }
-          exp_pass(m_b == -INFINITY ? 0.f : m_b, false);
-          if (t > 0) {  // O holds earlier tiles: rescale it (PV_{t-1} has completed)
+        const float alpha = upd ? ex2(m_b - mx_s) : 1.f;  // 0 when m_b was -inf
+        if (upd) m_b = mx_s;
+        const float base = m_b == -INFINITY ? 0.f : m_b;
+        // p = 2^(s * scale*log2e - base); packed bf16 pairs overwrite sr[0..63].
+        float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        const float2 sl = make_float2(sl2, sl2), nb = make_float2(-base, -base);
 #pragma unroll
-            for (int c = 0; c < D; c += 32) {
-              uint32_t orr[32];
-              tmem_ld32(o_tmem + c, orr);
-              tmem_wait_ld();
+        for (int c = 0; c < 128; c += 2) {
+          const float2 e = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl, nb);
+          const float2 p = make_float2(ex2(e.x), ex2(e.y));
+          acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], p);
+          sr[c >> 1] = pack_bf16x2(p.x, p.y);
+        }
+        if (t > 0 && __any_sync(0xffffffffu, upd)) {
+          // O holds earlier tiles (PV_{t-1} has completed): rescale it.
 #pragma unroll
-              for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-              tmem_st32(o_tmem + c, orr);
-            }
+          for (int c = 0; c < D; c += 32) {
+            uint32_t orr[32];
+            tmem_ld32(o_tmem + c, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+            tmem_st32(o_tmem + c, orr);
           }
         }
         const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
         l = l * alpha + (s01.x + s01.y);
         // P over the first 64 columns of this S row.
-        tmem_st32(s_tmem, pk);
-        tmem_st32(s_tmem + 32, pk + 32);
+        tmem_st32(s_tmem, sr);
+        tmem_st32(s_tmem + 32, sr + 32);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -541,8 +532,14 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_bf16_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmem);
+    // The warpgroup register split is only safe when every thread starts with
+    // exactly kLaunchRegs registers.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, prefill_bf16_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs || fa.maxThreadsPerBlock < kThreads) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(prefill_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg<D>::kSmem);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
