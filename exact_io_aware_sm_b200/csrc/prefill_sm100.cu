@@ -58,6 +58,10 @@ constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
 struct Cfg {
+  // Of every 8 column pairs of a full tile, this many take the polynomial
+  // exp2 instead of the MUFU unit.  Measured slower on both head dims so far
+  // (the softmax is latency-bound, not MUFU-bound), hence 0.
+  static constexpr int kPolyPairs = 0;
   static constexpr int kQBuf = (D == 64) ? 2 : 1;         // Q buffers per slot
   static constexpr int kRing = (D == 64) ? 8 : 4;         // K/V tiles in flight
   static constexpr int kChunkBytes = 128 * 128;           // 128 rows x 64 bf16 (one swizzle span)
@@ -103,6 +107,27 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
+}
+
+// 2^x on the FMA pipe, two lanes at a time, for x finite: x = j + f with
+// j = rint(x) (added to 1.5 * 2^23, whose low mantissa bits then hold j) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (relative error
+// 7.5e-5, Remez exchange, coefficients from gen_exp2_poly.py); j is added to
+// the exponent field.  x is clamped at -126 so the result stays a normal
+// number (2^-126 instead of a smaller value).  Full tiles may route part of
+// their exponentials here instead of the MUFU unit (Cfg::kPolyPairs).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = fadd2(x, magic);
+  const float2 jf = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = ffma2(jf, make_float2(-1.0f, -1.0f), x);
+  float2 p = ffma2(make_float2(0.055171669f, 0.055171669f), f, make_float2(0.24261112f, 0.24261112f));
+  p = ffma2(p, f, make_float2(0.69326099f, 0.69326099f));
+  p = ffma2(p, f, make_float2(0.99992807f, 0.99992807f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -219,156 +244,160 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+  // The producer and MMA warps run converged; elect.sync picks the lane that
+  // issues each TMA copy, MMA and commit.
+  auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    const bool mine = !*abort_flag && mbar_wait(bar, parity);
+    return __all_sync(0xffffffffu, mine);
+  };
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      uint32_t seq = 0;
-      uint32_t qcnt[2] = {0, 0};
-      bool ok = true;
-      for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
-        const Item it = decode_item(a, w);
-        const int nX[2] = {it.nA, it.nB};
-        const int rowX[2] = {it.rowA, it.rowB};
-        const int headX[2] = {it.headA, it.headB};
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (nX[x] == 0) continue;
-          const uint32_t qb = qcnt[x] % QB, use = qcnt[x] / QB;
-          if (use > 0 && (*abort_flag || !mbar_wait(&q_empty[x * QB + qb], (use - 1) & 1))) {
+    }
+    uint32_t seq = 0;
+    uint32_t qcnt[2] = {0, 0};
+    bool ok = true;
+    for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+      const Item it = decode_item(a, w);
+      const int nX[2] = {it.nA, it.nB};
+      const int rowX[2] = {it.rowA, it.rowB};
+      const int headX[2] = {it.headA, it.headB};
+      for (int x = 0; x < 2 && ok; ++x) {
+        if (nX[x] == 0) continue;
+        const uint32_t qb = qcnt[x] % QB, use = qcnt[x] / QB;
+        if (use > 0 && !wwait(&q_empty[x * QB + qb], (use - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx_elect(&q_full[x * QB + qb], C::kTileBytes);
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch)
+          tma_load_4d_elect(smem + C::kOffQ + (x * QB + qb) * C::kTileBytes + ch * C::kChunkBytes, &tmQ,
+                            &q_full[x * QB + qb], ch * 64, headX[x], rowX[x], it.b);
+        qcnt[x]++;
+      }
+      for (int j = 0; ok && j < it.nB; ++j) {
+        const int4 kt = a.kvtiles[it.kv_first + j];
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t slot = seq % R;
+          if (seq >= R && !wwait(&ring_empty[slot], ((seq / R) + 1) & 1)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&q_full[x * QB + qb], C::kTileBytes);
+          mbar_arrive_expect_tx_elect(&ring_full[slot], C::kTileBytes);
+          const CUtensorMap* map = t == 0 ? &tmK : &tmV;
 #pragma unroll
           for (int ch = 0; ch < NCH; ++ch)
-            tma_load_4d(smem + C::kOffQ + (x * QB + qb) * C::kTileBytes + ch * C::kChunkBytes, &tmQ,
-                        &q_full[x * QB + qb], ch * 64, headX[x], rowX[x], it.b);
-          qcnt[x]++;
-        }
-        for (int j = 0; ok && j < it.nB; ++j) {
-          const int4 kt = a.kvtiles[it.kv_first + j];
-          for (int t = 0; t < 2; ++t) {
-            const uint32_t slot = seq % R;
-            if (seq >= R && (*abort_flag || !mbar_wait(&ring_empty[slot], ((seq / R) + 1) & 1))) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&ring_full[slot], C::kTileBytes);
-            const CUtensorMap* map = t == 0 ? &tmK : &tmV;
-#pragma unroll
-            for (int ch = 0; ch < NCH; ++ch)
-              tma_load_4d(smem + C::kOffRing + slot * C::kTileBytes + ch * C::kChunkBytes, map,
-                          &ring_full[slot], ch * 64, it.hkv, kt.x, it.b);
-            ++seq;
-          }
+            tma_load_4d_elect(smem + C::kOffRing + slot * C::kTileBytes + ch * C::kChunkBytes, map,
+                              &ring_full[slot], ch * 64, it.hkv, kt.x, it.b);
+          ++seq;
         }
       }
-      if (!ok) {
-        fail(kErrDeviceTimeout);
-        // Let every copy this thread started land before the CTA retires.
-        for (int x = 0; x < 2; ++x)
-          for (uint32_t c = qcnt[x] > QB ? qcnt[x] - QB : 0; c < qcnt[x]; ++c)
-            mbar_wait(&q_full[x * QB + c % QB], (c / QB) & 1);
-        for (uint32_t s = seq > R ? seq - R : 0; s < seq; ++s)
-          mbar_wait(&ring_full[s % R], (s / R) & 1);
-      }
+    }
+    if (!ok) {
+      if (lane == 0) fail(kErrDeviceTimeout);
+      // Let every copy this warp started land before the CTA retires.
+      for (int x = 0; x < 2; ++x)
+        for (uint32_t c = qcnt[x] > QB ? qcnt[x] - QB : 0; c < qcnt[x]; ++c)
+          mbar_wait(&q_full[x * QB + c % QB], (c / QB) & 1);
+      for (uint32_t s = seq > R ? seq - R : 0; s < seq; ++s)
+        mbar_wait(&ring_full[s % R], (s / R) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);  // A = P (TMEM), B = V (MN-major)
-      uint32_t seq = 0;
-      uint32_t qcnt[2] = {0, 0}, scnt[2] = {0, 0}, pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
-      bool ok = true;
+    const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);  // A = P (TMEM), B = V (MN-major)
+    uint32_t seq = 0;
+    uint32_t qcnt[2] = {0, 0}, scnt[2] = {0, 0}, pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
+    bool ok = true;
 
-      auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
-        if (!ok) return false;
-        if (*abort_flag || !mbar_wait(bar, parity)) ok = false;
-        return ok;
-      };
-      // S_X = Q_X K^T for the K tile in ring slot kslot.
-      uint32_t qbuf[2] = {0, 0};
-      auto issue_s = [&](int x, int ncols, uint32_t kslot) {
-        if (scnt[x] > 0 && !wait_bar(&pv_done[x], (pcnt[x] - 1) & 1)) return;  // P_X shares S_X
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(x * 128);
-        const uint32_t id = idesc_bf16_f32(128, static_cast<uint32_t>(ncols), 0, 0);
-        const uint32_t qbase = sQ + (x * QB + qbuf[x]) * C::kTileBytes;
-        const uint32_t kbase = sRing + kslot * C::kTileBytes;
+    auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
+      if (!ok) return false;
+      ok = wwait(bar, parity);
+      return ok;
+    };
+    uint32_t qbuf[2] = {0, 0};
+    // S_X = Q_X K^T for the K tile in ring slot kslot.
+    auto issue_s = [&](int x, int ncols, uint32_t kslot) {
+      if (scnt[x] > 0 && !wait_bar(&pv_done[x], (pcnt[x] - 1) & 1)) return;  // P_X shares S_X
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(x * 128);
+      const uint32_t id = idesc_bf16_f32(128, static_cast<uint32_t>(ncols), 0, 0);
+      const uint32_t qbase = sQ + (x * QB + qbuf[x]) * C::kTileBytes;
+      const uint32_t kbase = sRing + kslot * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          mma_bf16_ss(d_tmem, sdesc_sw128(qbase + koff, 16, 1024),
-                      sdesc_sw128(kbase + koff, 16, 1024), id, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&s_full[x]);
-        scnt[x]++;
-      };
-      // O_X (+)= P_X V for the V tile in ring slot vslot.
-      auto issue_pv = [&](int x, int j, int nX, int ncols, uint32_t vslot) {
-        if (!wait_bar(&p_full[x], pcnt[x] & 1)) return;
-        if (j == 0 && ocnt[x] > 0 && !wait_bar(&o_free[x], (ocnt[x] - 1) & 1)) return;
-        tc_fence_after();
-        const uint32_t p_tmem = tmem + static_cast<uint32_t>(x * 128);
-        const uint32_t o_tmem = tmem + static_cast<uint32_t>(256 + x * D);
-        const uint32_t vbase = sRing + vslot * C::kTileBytes;
-        const int ksteps = ncols >> 4;
-        for (int kk = 0; kk < ksteps; ++kk)
-          mma_bf16_ts(o_tmem, p_tmem + kk * 8, sdesc_sw128(vbase + kk * 2048, C::kChunkBytes, 1024),
-                      idO, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&pv_done[x]);
-        pcnt[x]++;
-        if (j == nX - 1) ocnt[x]++;
-      };
-
-      for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
-        const Item it = decode_item(a, w);
-        const int nA = it.nA, nB = it.nB;
-        for (int x = 0; x < 2; ++x) {
-          if ((x == 0 ? nA : nB) == 0) continue;
-          qbuf[x] = qcnt[x] % QB;
-          if (wait_bar(&q_full[x * QB + qbuf[x]], (qcnt[x] / QB) & 1)) qcnt[x]++;
-        }
-        if (!ok || nB == 0) continue;
-        const int4* kv = a.kvtiles + it.kv_first;
-        // tile 0: S_A, S_B
-        if (!wait_bar(&ring_full[seq % R], (seq / R) & 1)) break;
-        if (nA > 0) issue_s(0, kv[0].y, seq % R);
-        issue_s(1, kv[0].y, seq % R);
-        if (!ok) break;
-        mma_commit(&ring_empty[seq % R]);
-        for (int j = 0; ok && j < nB; ++j) {
-          const uint32_t vseq = seq + 2 * j + 1, kseq = vseq + 1;
-          const int ncj = kv[j].y;
-          if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
-          const bool next = j + 1 < nB;
-          const int ncn = next ? kv[j + 1].y : 0;
-          if (j < nA) {
-            issue_pv(0, j, nA, ncj, vseq % R);
-            if (j + 1 < nA && wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) issue_s(0, ncn, kseq % R);
-          }
-          issue_pv(1, j, nB, ncj, vseq % R);
-          if (!ok) break;
-          mma_commit(&ring_empty[vseq % R]);
-          if (next) {
-            if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
-            issue_s(1, ncn, kseq % R);
-            if (!ok) break;
-            mma_commit(&ring_empty[kseq % R]);
-          }
-        }
-        seq += 2 * nB;
-        if (!ok) break;
-        if (nA > 0) mma_commit(&q_empty[qbuf[0]]);
-        mma_commit(&q_empty[QB + qbuf[1]]);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+        mma_bf16_ss_elect(d_tmem, sdesc_sw128(qbase + koff, 16, 1024),
+                          sdesc_sw128(kbase + koff, 16, 1024), id, kk > 0 ? 1u : 0u);
       }
-      if (!ok) fail(kErrDeviceTimeout);
-      // Every MMA issued above has finished before TMEM is released.
-      mma_commit(mma_idle);
-      mbar_wait(mma_idle, 0);
+      mma_commit_elect(&s_full[x]);
+      scnt[x]++;
+    };
+    // O_X (+)= P_X V for the V tile in ring slot vslot.
+    auto issue_pv = [&](int x, int j, int nX, int ncols, uint32_t vslot) {
+      if (!wait_bar(&p_full[x], pcnt[x] & 1)) return;
+      if (j == 0 && ocnt[x] > 0 && !wait_bar(&o_free[x], (ocnt[x] - 1) & 1)) return;
+      tc_fence_after();
+      const uint32_t p_tmem = tmem + static_cast<uint32_t>(x * 128);
+      const uint32_t o_tmem = tmem + static_cast<uint32_t>(256 + x * D);
+      const uint32_t vbase = sRing + vslot * C::kTileBytes;
+      const int ksteps = ncols >> 4;
+      for (int kk = 0; kk < ksteps; ++kk)
+        mma_bf16_ts_elect(o_tmem, p_tmem + kk * 8, sdesc_sw128(vbase + kk * 2048, C::kChunkBytes, 1024),
+                          idO, (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit_elect(&pv_done[x]);
+      pcnt[x]++;
+      if (j == nX - 1) ocnt[x]++;
+    };
+
+    for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+      const Item it = decode_item(a, w);
+      const int nA = it.nA, nB = it.nB;
+      for (int x = 0; x < 2; ++x) {
+        if ((x == 0 ? nA : nB) == 0) continue;
+        qbuf[x] = qcnt[x] % QB;
+        if (wait_bar(&q_full[x * QB + qbuf[x]], (qcnt[x] / QB) & 1)) qcnt[x]++;
+      }
+      if (!ok || nB == 0) continue;
+      const int4* kv = a.kvtiles + it.kv_first;
+      // tile 0: S_A, S_B
+      if (!wait_bar(&ring_full[seq % R], (seq / R) & 1)) break;
+      if (nA > 0) issue_s(0, kv[0].y, seq % R);
+      issue_s(1, kv[0].y, seq % R);
+      if (!ok) break;
+      mma_commit_elect(&ring_empty[seq % R]);
+      for (int j = 0; ok && j < nB; ++j) {
+        const uint32_t vseq = seq + 2 * j + 1, kseq = vseq + 1;
+        const int ncj = kv[j].y;
+        if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
+        const bool next = j + 1 < nB;
+        const int ncn = next ? kv[j + 1].y : 0;
+        if (j < nA) {
+          issue_pv(0, j, nA, ncj, vseq % R);
+          if (j + 1 < nA && wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) issue_s(0, ncn, kseq % R);
+        }
+        issue_pv(1, j, nB, ncj, vseq % R);
+        if (!ok) break;
+        mma_commit_elect(&ring_empty[vseq % R]);
+        if (next) {
+          if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
+          issue_s(1, ncn, kseq % R);
+          if (!ok) break;
+          mma_commit_elect(&ring_empty[kseq % R]);
+        }
+      }
+      seq += 2 * nB;
+      if (!ok) break;
+      if (nA > 0) mma_commit_elect(&q_empty[qbuf[0]]);
+      mma_commit_elect(&q_empty[QB + qbuf[1]]);
     }
+    if (!ok && lane == 0) fail(kErrDeviceTimeout);
+    // Every MMA issued above has finished before TMEM is released.
+    mma_commit_elect(mma_idle);
+    mbar_wait(mma_idle, 0);
   }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
@@ -443,10 +472,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // p = 2^(s * scale*log2e - base); packed bf16 pairs overwrite sr[0..63].
         float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
         const float2 sl = make_float2(sl2, sl2), nb = make_float2(-base, -base);
+        const bool poly_ok = !__any_sync(0xffffffffu, lim < 128);  // every score finite
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
           const float2 e = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl, nb);
-          const float2 p = make_float2(ex2(e.x), ex2(e.y));
+          const float2 p = (((c >> 1) & 7) < C::kPolyPairs && poly_ok) ? exp2_poly2(e)
+                                                                       : make_float2(ex2(e.x), ex2(e.y));
           acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], p);
           sr[c >> 1] = pack_bf16x2(p.x, p.y);
         }
