@@ -271,6 +271,17 @@ def time_steps(step, K, W, world, flush=None):
     return sum(ms) / K, wall
 
 
+def capture_graph(step):
+    """Capture one call of `step` (library call, warm: plan and workspace
+    cached) into a CUDA graph; replaying it removes the per-call host work."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    torch.cuda.synchronize()
+    return g
+
+
 def make_flush():
     import torch
     buf = torch.empty(256 * MIB, dtype=torch.uint8, device="cuda")
@@ -296,9 +307,15 @@ def bench_prefill(w, args, world, rank, peaks, with_e2e=True):
         eio.attn_fwd(tq, tk, tv, o=o, lse=lse, scale=scale, mask_kind=mk, block_map=bm)
 
     flush = make_flush()
-    ms, wall = time_steps(step, args.steps, args.warmup, world, flush)
+    # Eager calls first (warms the plan cache), then the same call replayed
+    # from a CUDA graph: the graph time is the kernel's, the eager time adds
+    # the host-side call overhead when the GPU would otherwise idle.
+    eager_ms, _ = time_steps(step, args.steps, args.warmup, world, flush)
+    graph = capture_graph(step)
+    ms, wall = time_steps(graph.replay, args.steps, args.warmup, world, flush)
     eio.sync_status()
     ms = max_over_ranks(ms, world)
+    eager_ms = max_over_ranks(eager_ms, world)
     flops = prefill_flops(w)
     tflops = world * flops / (ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
@@ -311,6 +328,8 @@ def bench_prefill(w, args, world, rank, peaks, with_e2e=True):
                      "traffic": recorded_traffic(f"prefill_{args_key(w)}")},
         "gpu_launches": args.steps,
         "wall_s": wall,
+        "eager_ms_per_step": eager_ms,
+        "timing": "CUDA graph replay of one attn_fwd call per step; eager_ms_per_step is the plain call",
     }
     # attainable at this arithmetic intensity: min(peak, AI * HBM)
     alg_bytes = q.nbytes + k.nbytes + v.nbytes + q.nbytes + lse.numel() * 4  # Q, K, V in; O, LSE out
@@ -367,9 +386,12 @@ def bench_decode(w, args, world, rank, peaks, with_e2e=True):
         eio.attn_decode(tq, tk, tv, tl, o=o, lse=lse, scale=scale)
 
     steps = max(args.steps, 20)
-    ms, wall = time_steps(step, steps, args.warmup, world)
+    eager_ms, _ = time_steps(step, steps, args.warmup, world)
+    graph = capture_graph(step)
+    ms, wall = time_steps(graph.replay, steps, args.warmup, world)
     eio.sync_status()
     ms = max_over_ranks(ms, world)
+    eager_ms = max_over_ranks(eager_ms, world)
     kvb = decode_kv_bytes(lens, Hkv, d)
     alg = kvb + q.nbytes * 2 + B * Hq * 4
     gbs = world * alg / (ms * 1e-3) / 1e9
@@ -383,6 +405,8 @@ def bench_decode(w, args, world, rank, peaks, with_e2e=True):
                      "kernel": "decode_split_kernel + decode_combine_kernel (one call)",
                      "traffic": recorded_traffic("decode")},
         "gpu_launches": 2 * steps, "steps": steps, "wall_s": wall,
+        "eager_ms_per_step": eager_ms,
+        "timing": "CUDA graph replay of one attn_decode call (split + combine) per step",
     }
     if with_e2e:
         # A decode step's input is the new query; the cache stays resident.
@@ -519,7 +543,8 @@ def main():
                 r = bench_prefill(wx, argparse.Namespace(steps=max(5, args.steps // 5), warmup=3),
                                   world, rank, peaks, with_e2e=False)
                 extra[name] = {"metric": "prefill attn TFLOP/s", "value": r["tflops"], "unit": "TFLOP/s",
-                               "ms_per_step": r["ms_per_step"], "config": {"workload": wx["desc"]},
+                               "ms_per_step": r["ms_per_step"], "eager_ms_per_step": r["eager_ms_per_step"],
+                               "config": {"workload": wx["desc"]},
                                "roofline": r["roofline"], "gpu_launches": r["gpu_launches"]}
 
     cpu = None
@@ -540,6 +565,7 @@ def main():
                        "l2": "flushed before every step (256 MiB write)",
                        "flops_per_step_per_gpu": head["flops_per_step"]},
             "roofline": head["roofline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+            "eager_ms_per_step": head["eager_ms_per_step"], "timing": head["timing"],
             "clocks": sampler.summary(), "cpu_baseline": cpu,
         }
         line.update(extra)

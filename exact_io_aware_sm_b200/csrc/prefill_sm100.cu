@@ -63,6 +63,9 @@ struct Cfg {
   // (the softmax is latency-bound, not MUFU-bound), hence 0.
   static constexpr int kPolyPairs = 0;
   static constexpr int kQBuf = (D == 64) ? 2 : 1;         // Q buffers per slot
+  // d = 64 leaves 128 TMEM columns free: P gets its own columns, so the next
+  // S of a slot can be computed while the softmax of the current tile runs.
+  static constexpr bool kSepP = D == 64;
   static constexpr int kRing = (D == 64) ? 8 : 4;         // K/V tiles in flight
   static constexpr int kChunkBytes = 128 * 128;           // 128 rows x 64 bf16 (one swizzle span)
   static constexpr int kTileBytes = 128 * D * 2;          // Q, K or V tile (128 rows)
@@ -71,7 +74,7 @@ struct Cfg {
   static constexpr int kOffBar = kOffRing + kRing * kTileBytes;
   // q_full[2*QB] q_empty[2*QB] ring_full[R] ring_empty[R] s_full[2] p_full[2]
   // pv_done[2] o_free[2] mma_idle
-  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 1;
+  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 1 + 2;  // + s_free[2]
   static constexpr int kSmem = kOffBar + 8 * kNumBars + 16 + 1024;  // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -199,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pv_done = p_full + 2;     // [2]
   uint64_t* o_free = pv_done + 2;     // [2]
   uint64_t* mma_idle = o_free + 2;
+  uint64_t* s_free = mma_idle + 1;    // [2] (separate-P layout): S loaded by the softmax
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -215,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[x], 4);
       mbar_init(&pv_done[x], 1);
       mbar_init(&o_free[x], 4);
+      mbar_init(&s_free[x], 4);
     }
     for (int i = 0; i < R; ++i) {
       mbar_init(&ring_full[i], 1);
@@ -321,7 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t qbuf[2] = {0, 0};
     // S_X = Q_X K^T for the K tile in ring slot kslot.
     auto issue_s = [&](int x, int ncols, uint32_t kslot) {
-      if (scnt[x] > 0 && !wait_bar(&pv_done[x], (pcnt[x] - 1) & 1)) return;  // P_X shares S_X
+      if (scnt[x] > 0) {
+        // S_X is rewritten: the softmax must have loaded it (separate P) or
+        // the PV that read P from its columns must have completed.
+        if (C::kSepP ? !wait_bar(&s_free[x], (scnt[x] - 1) & 1)
+                     : !wait_bar(&pv_done[x], (pcnt[x] - 1) & 1))
+          return;
+      }
       tc_fence_after();
       const uint32_t d_tmem = tmem + static_cast<uint32_t>(x * 128);
       const uint32_t id = idesc_bf16_f32(128, static_cast<uint32_t>(ncols), 0, 0);
@@ -341,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!wait_bar(&p_full[x], pcnt[x] & 1)) return;
       if (j == 0 && ocnt[x] > 0 && !wait_bar(&o_free[x], (ocnt[x] - 1) & 1)) return;
       tc_fence_after();
-      const uint32_t p_tmem = tmem + static_cast<uint32_t>(x * 128);
+      const uint32_t p_tmem = tmem + static_cast<uint32_t>(C::kSepP ? 256 + 2 * D + x * 64 : x * 128);
       const uint32_t o_tmem = tmem + static_cast<uint32_t>(256 + x * D);
       const uint32_t vbase = sRing + vslot * C::kTileBytes;
       const int ksteps = ncols >> 4;
@@ -372,21 +383,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < nB; ++j) {
         const uint32_t vseq = seq + 2 * j + 1, kseq = vseq + 1;
         const int ncj = kv[j].y;
-        if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
         const bool next = j + 1 < nB;
         const int ncn = next ? kv[j + 1].y : 0;
-        if (j < nA) {
-          issue_pv(0, j, nA, ncj, vseq % R);
-          if (j + 1 < nA && wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) issue_s(0, ncn, kseq % R);
-        }
-        issue_pv(1, j, nB, ncj, vseq % R);
-        if (!ok) break;
-        mma_commit_elect(&ring_empty[vseq % R]);
-        if (next) {
-          if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
-          issue_s(1, ncn, kseq % R);
+        if constexpr (C::kSepP) {
+          // S for tile j+1 first (the softmax frees S as soon as it has
+          // loaded it), then the PVs of tile j.
+          if (next) {
+            if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
+            if (j + 1 < nA) issue_s(0, ncn, kseq % R);
+            issue_s(1, ncn, kseq % R);
+            if (!ok) break;
+            mma_commit_elect(&ring_empty[kseq % R]);
+          }
+          if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
+          if (j < nA) issue_pv(0, j, nA, ncj, vseq % R);
+          issue_pv(1, j, nB, ncj, vseq % R);
           if (!ok) break;
-          mma_commit_elect(&ring_empty[kseq % R]);
+          mma_commit_elect(&ring_empty[vseq % R]);
+        } else {
+          if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
+          if (j < nA) {
+            issue_pv(0, j, nA, ncj, vseq % R);
+            if (j + 1 < nA && wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) issue_s(0, ncn, kseq % R);
+          }
+          issue_pv(1, j, nB, ncj, vseq % R);
+          if (!ok) break;
+          mma_commit_elect(&ring_empty[vseq % R]);
+          if (next) {
+            if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
+            issue_s(1, ncn, kseq % R);
+            if (!ok) break;
+            mma_commit_elect(&ring_empty[kseq % R]);
+          }
         }
       }
       seq += 2 * nB;
@@ -408,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_tmem = tmem + lane_off + static_cast<uint32_t>(x * 128);
     const uint32_t o_tmem = tmem + lane_off + static_cast<uint32_t>(256 + x * D);
+    const uint32_t p_tmem = C::kSepP ? tmem + lane_off + static_cast<uint32_t>(256 + 2 * D + x * 64) : s_tmem;
     const float sl2 = a.scale_log2;
     uint32_t tcnt = 0;
     bool ok = true;
@@ -449,6 +478,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(s_tmem + c * 32, sr + c * 32);
         tmem_wait_ld();
+        if constexpr (C::kSepP) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[x]);
+        }
         if (__any_sync(0xffffffffu, lim < 128)) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -481,6 +515,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], p);
           sr[c >> 1] = pack_bf16x2(p.x, p.y);
         }
+        if (C::kSepP && t > 0) {
+          // P_X and O_X are free once PV_{t-1} has completed.
+          if (!warp_wait(&pv_done[x], (tcnt - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
         if (t > 0 && __any_sync(0xffffffffu, upd)) {
           // O holds earlier tiles (PV_{t-1} has completed): rescale it.
 #pragma unroll
@@ -496,8 +538,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
         l = l * alpha + (s01.x + s01.y);
         // P over the first 64 columns of this S row.
-        tmem_st32(s_tmem, sr);
-        tmem_st32(s_tmem + 32, sr + 32);
+        tmem_st32(p_tmem, sr);
+        tmem_st32(p_tmem + 32, sr + 32);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
