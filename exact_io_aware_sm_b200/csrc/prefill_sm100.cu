@@ -17,10 +17,11 @@
 //   warp 0        TMA producer: Q_A, Q_B once per item (double-buffered for
 //                 d = 64, whose items are short), then K_j, V_j into a ring of
 //                 shared-memory stages.
-//   warp 1        MMA issuer (one thread) and TMEM owner:
+//   warps 1, 2    MMA issuers for slot A and slot B (warp 1 also owns TMEM):
 //                   S_X = Q_X K_j^T      (A and B from shared memory)
 //                   O_X += P_X V_j       (P_X from TMEM, V_j from shared memory)
-//   warps 2, 3    idle.
+//                 issued from the converged warp by an elect.sync-chosen lane.
+//   warp 3        idle.
 //   warps 4..7    softmax for slot A, one thread per query row.
 //   warps 8..11   softmax for slot B.
 // Each softmax thread loads its whole S row from TMEM (one wait), takes the
@@ -71,10 +72,14 @@ struct Cfg {
   static constexpr int kTileBytes = 128 * D * 2;          // Q, K or V tile (128 rows)
   static constexpr int kOffQ = 0;                         // Q[slot][buffer]
   static constexpr int kOffRing = 2 * kQBuf * kTileBytes;
-  static constexpr int kOffBar = kOffRing + kRing * kTileBytes;
+  // d = 64: the epilogue stages each slot's bf16 O tile (128 rows x 128 B) in
+  // shared memory so that rows are stored to HBM as whole 128-byte lines.
+  static constexpr bool kStageO = D == 64;
+  static constexpr int kOffStage = kOffRing + kRing * kTileBytes;
+  static constexpr int kOffBar = kOffStage + (kStageO ? 2 * 128 * D * 2 : 0);
   // q_full[2*QB] q_empty[2*QB] ring_full[R] ring_empty[R] s_full[2] p_full[2]
   // pv_done[2] o_free[2] mma_idle
-  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 1 + 2;  // + s_free[2]
+  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 2 + 2;  // + mma_idle[2], s_free[2]
   static constexpr int kSmem = kOffBar + 8 * kNumBars + 16 + 1024;  // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -179,6 +184,16 @@ __device__ __forceinline__ Item decode_item(const PrefillArgs& a, long long w) {
   return it;
 }
 
+// The k-th work item of this CTA, or -1 when there is none.  Items are sorted
+// by size (largest first); rounds of gridDim.x items are dealt to the CTAs in
+// alternating directions, which evens out the total work per CTA.
+__device__ __forceinline__ long long item_index(long long k, long long n_items) {
+  const long long g = gridDim.x, base = k * g;
+  if (base >= n_items) return -1;
+  const long long idx = (k & 1) ? base + (g - 1 - blockIdx.x) : base + blockIdx.x;
+  return idx < n_items ? idx : -1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -201,8 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + 2;      // [2]
   uint64_t* pv_done = p_full + 2;     // [2]
   uint64_t* o_free = pv_done + 2;     // [2]
-  uint64_t* mma_idle = o_free + 2;
-  uint64_t* s_free = mma_idle + 1;    // [2] (separate-P layout): S loaded by the softmax
+  uint64_t* mma_idle = o_free + 2;    // [2]
+  uint64_t* s_free = mma_idle + 2;    // [2] (separate-P layout): S loaded by the softmax
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -223,9 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < R; ++i) {
       mbar_init(&ring_full[i], 1);
-      mbar_init(&ring_empty[i], 1);
+      mbar_init(&ring_empty[i], 2);  // released by both slot issuers
     }
-    mbar_init(mma_idle, 1);
+    mbar_init(&mma_idle[0], 1);
+    mbar_init(&mma_idle[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -265,8 +281,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t seq = 0;
     uint32_t qcnt[2] = {0, 0};
     bool ok = true;
-    for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
-      const Item it = decode_item(a, w);
+    long long wk = 0, w = item_index(0, n_items);
+    Item it_next = w >= 0 ? decode_item(a, w) : Item{};
+    for (; ok && w >= 0;) {
+      const Item it = it_next;  // decoded one item ahead
+      w = item_index(++wk, n_items);
+      if (w >= 0) it_next = decode_item(a, w);
       const int nX[2] = {it.nA, it.nB};
       const int rowX[2] = {it.rowA, it.rowB};
       const int headX[2] = {it.headA, it.headB};
@@ -311,121 +331,106 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t s = seq > R ? seq - R : 0; s < seq; ++s)
         mbar_wait(&ring_full[s % R], (s / R) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 1 issues slot A's GEMMs, warp 2 slot B's, so each slot's chain
+    // (S -> softmax -> PV) advances on its own.
+    const int x = warp - 1;
     const uint32_t idO = idesc_bf16_f32(128, D, 0, 1);  // A = P (TMEM), B = V (MN-major)
-    uint32_t seq = 0;
-    uint32_t qcnt[2] = {0, 0}, scnt[2] = {0, 0}, pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
+    const uint32_t s_col = tmem + static_cast<uint32_t>(x * 128);
+    const uint32_t o_col = tmem + static_cast<uint32_t>(256 + x * D);
+    const uint32_t p_col = C::kSepP ? tmem + static_cast<uint32_t>(256 + 2 * D + x * 64) : s_col;
+    uint32_t seq = 0, qcnt = 0, scnt = 0, pcnt = 0, ocnt = 0;
     bool ok = true;
-
     auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
       if (!ok) return false;
       ok = wwait(bar, parity);
       return ok;
     };
-    uint32_t qbuf[2] = {0, 0};
-    // S_X = Q_X K^T for the K tile in ring slot kslot.
-    auto issue_s = [&](int x, int ncols, uint32_t kslot) {
-      if (scnt[x] > 0) {
+    // S_X = Q_X K^T for the K tile in ring slot kslot; releases the stage.
+    auto issue_s = [&](uint32_t qbase, int ncols, uint32_t kslot) {
+      if (scnt > 0) {
         // S_X is rewritten: the softmax must have loaded it (separate P) or
         // the PV that read P from its columns must have completed.
-        if (C::kSepP ? !wait_bar(&s_free[x], (scnt[x] - 1) & 1)
-                     : !wait_bar(&pv_done[x], (pcnt[x] - 1) & 1))
+        if (C::kSepP ? !wait_bar(&s_free[x], (scnt - 1) & 1) : !wait_bar(&pv_done[x], (pcnt - 1) & 1))
           return;
       }
       tc_fence_after();
-      const uint32_t d_tmem = tmem + static_cast<uint32_t>(x * 128);
       const uint32_t id = idesc_bf16_f32(128, static_cast<uint32_t>(ncols), 0, 0);
-      const uint32_t qbase = sQ + (x * QB + qbuf[x]) * C::kTileBytes;
       const uint32_t kbase = sRing + kslot * C::kTileBytes;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-        mma_bf16_ss_elect(d_tmem, sdesc_sw128(qbase + koff, 16, 1024),
-                          sdesc_sw128(kbase + koff, 16, 1024), id, kk > 0 ? 1u : 0u);
+        mma_bf16_ss_elect(s_col, sdesc_sw128(qbase + koff, 16, 1024), sdesc_sw128(kbase + koff, 16, 1024),
+                          id, kk > 0 ? 1u : 0u);
       }
       mma_commit_elect(&s_full[x]);
-      scnt[x]++;
+      mma_commit_elect(&ring_empty[kslot]);
+      scnt++;
     };
-    // O_X (+)= P_X V for the V tile in ring slot vslot.
-    auto issue_pv = [&](int x, int j, int nX, int ncols, uint32_t vslot) {
-      if (!wait_bar(&p_full[x], pcnt[x] & 1)) return;
-      if (j == 0 && ocnt[x] > 0 && !wait_bar(&o_free[x], (ocnt[x] - 1) & 1)) return;
+    // O_X (+)= P_X V for the V tile in ring slot vslot; releases the stage.
+    auto issue_pv = [&](int j, int ncols, uint32_t vslot) {
+      if (!wait_bar(&p_full[x], pcnt & 1)) return;
+      if (j == 0 && ocnt > 0 && !wait_bar(&o_free[x], (ocnt - 1) & 1)) return;
       tc_fence_after();
-      const uint32_t p_tmem = tmem + static_cast<uint32_t>(C::kSepP ? 256 + 2 * D + x * 64 : x * 128);
-      const uint32_t o_tmem = tmem + static_cast<uint32_t>(256 + x * D);
       const uint32_t vbase = sRing + vslot * C::kTileBytes;
-      const int ksteps = ncols >> 4;
-      for (int kk = 0; kk < ksteps; ++kk)
-        mma_bf16_ts_elect(o_tmem, p_tmem + kk * 8, sdesc_sw128(vbase + kk * 2048, C::kChunkBytes, 1024),
+      for (int kk = 0; kk < (ncols >> 4); ++kk)
+        mma_bf16_ts_elect(o_col, p_col + kk * 8, sdesc_sw128(vbase + kk * 2048, C::kChunkBytes, 1024),
                           idO, (j > 0 || kk > 0) ? 1u : 0u);
       mma_commit_elect(&pv_done[x]);
-      pcnt[x]++;
-      if (j == nX - 1) ocnt[x]++;
+      mma_commit_elect(&ring_empty[vslot]);
+      pcnt++;
     };
 
-    for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
-      const Item it = decode_item(a, w);
-      const int nA = it.nA, nB = it.nB;
-      for (int x = 0; x < 2; ++x) {
-        if ((x == 0 ? nA : nB) == 0) continue;
-        qbuf[x] = qcnt[x] % QB;
-        if (wait_bar(&q_full[x * QB + qbuf[x]], (qcnt[x] / QB) & 1)) qcnt[x]++;
-      }
-      if (!ok || nB == 0) continue;
+    long long wk = 0, w = item_index(0, n_items);
+    Item it_next = w >= 0 ? decode_item(a, w) : Item{};
+    for (; ok && w >= 0;) {
+      const Item it = it_next;  // decoded one item ahead
+      w = item_index(++wk, n_items);
+      if (w >= 0) it_next = decode_item(a, w);
+      const int nX = x == 0 ? it.nA : it.nB;
+      const int nB = it.nB;
       const int4* kv = a.kvtiles + it.kv_first;
-      // tile 0: S_A, S_B
-      if (!wait_bar(&ring_full[seq % R], (seq / R) & 1)) break;
-      if (nA > 0) issue_s(0, kv[0].y, seq % R);
-      issue_s(1, kv[0].y, seq % R);
-      if (!ok) break;
-      mma_commit_elect(&ring_empty[seq % R]);
-      for (int j = 0; ok && j < nB; ++j) {
-        const uint32_t vseq = seq + 2 * j + 1, kseq = vseq + 1;
-        const int ncj = kv[j].y;
-        const bool next = j + 1 < nB;
-        const int ncn = next ? kv[j + 1].y : 0;
-        if constexpr (C::kSepP) {
-          // S for tile j+1 first (the softmax frees S as soon as it has
-          // loaded it), then the PVs of tile j.
-          if (next) {
+      uint32_t qbuf = 0;
+      if (nX > 0) {
+        qbuf = qcnt % QB;
+        if (!wait_bar(&q_full[x * QB + qbuf], (qcnt / QB) & 1)) break;
+        qcnt++;
+        const uint32_t qbase = sQ + (x * QB + qbuf) * C::kTileBytes;
+        if (!wait_bar(&ring_full[seq % R], (seq / R) & 1)) break;
+        issue_s(qbase, kv[0].y, seq % R);
+        for (int j = 0; ok && j < nX; ++j) {
+          const uint32_t vseq = seq + 2 * j + 1, kseq = vseq + 1;
+          const bool next = j + 1 < nX;
+          if (C::kSepP && next) {  // next S as soon as the softmax has loaded this one
             if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
-            if (j + 1 < nA) issue_s(0, ncn, kseq % R);
-            issue_s(1, ncn, kseq % R);
-            if (!ok) break;
-            mma_commit_elect(&ring_empty[kseq % R]);
+            issue_s(qbase, kv[j + 1].y, kseq % R);
           }
           if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
-          if (j < nA) issue_pv(0, j, nA, ncj, vseq % R);
-          issue_pv(1, j, nB, ncj, vseq % R);
-          if (!ok) break;
-          mma_commit_elect(&ring_empty[vseq % R]);
-        } else {
-          if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
-          if (j < nA) {
-            issue_pv(0, j, nA, ncj, vseq % R);
-            if (j + 1 < nA && wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) issue_s(0, ncn, kseq % R);
-          }
-          issue_pv(1, j, nB, ncj, vseq % R);
-          if (!ok) break;
-          mma_commit_elect(&ring_empty[vseq % R]);
-          if (next) {
+          issue_pv(j, kv[j].y, vseq % R);
+          if (!C::kSepP && next) {  // P shares S's columns: after this PV
             if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
-            issue_s(1, ncn, kseq % R);
-            if (!ok) break;
-            mma_commit_elect(&ring_empty[kseq % R]);
+            issue_s(qbase, kv[j + 1].y, kseq % R);
           }
         }
+        ocnt++;
+      }
+      // Stages of tiles this slot does not visit: release once filled.
+      for (int j = nX; ok && j < nB; ++j) {
+        const uint32_t kseq = seq + 2 * j, vseq = kseq + 1;
+        if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
+        mbar_arrive_elect(&ring_empty[kseq % R]);
+        if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
+        mbar_arrive_elect(&ring_empty[vseq % R]);
       }
       seq += 2 * nB;
       if (!ok) break;
-      if (nA > 0) mma_commit_elect(&q_empty[qbuf[0]]);
-      mma_commit_elect(&q_empty[QB + qbuf[1]]);
+      if (nX > 0) mma_commit_elect(&q_empty[x * QB + qbuf]);
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
     // Every MMA issued above has finished before TMEM is released.
-    mma_commit_elect(mma_idle);
-    mbar_wait(mma_idle, 0);
+    mma_commit_elect(&mma_idle[x]);
+    mbar_wait(&mma_idle[x], 0);
   }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
@@ -447,8 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       return __all_sync(0xffffffffu, mine);
     };
 
-    for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
-      const Item it = decode_item(a, w);
+    long long wk = 0, w = item_index(0, n_items);
+    Item it_next = w >= 0 ? decode_item(a, w) : Item{};
+    for (; ok && w >= 0;) {
+      const Item it = it_next;  // decoded one item ahead
+      w = item_index(++wk, n_items);
+      if (w >= 0) it_next = decode_item(a, w);
       const int nX = x == 0 ? it.nA : it.nB;
       const int nrows = x == 0 ? it.nrowsA : it.nrowsB;
       const int row0 = x == 0 ? it.rowA : it.rowB;
@@ -558,6 +567,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
       const bool valid = row < nrows;
+      if constexpr (C::kStageO) {
+        // Row -> shared staging (16-byte units XOR-swizzled by row), then
+        // each warp stores its 32 rows as whole lines: 8 lanes per row.
+        constexpr int UPR = D / 8;  // 16-byte units per row
+        uint8_t* stg = smem + C::kOffStage + x * (128 * D * 2);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t orr[32];
+          if (nX > 0) {
+            tmem_ld32(o_tmem + c, orr);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) orr[i] = 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int unit = c / 8 + u;
+            *reinterpret_cast<uint4*>(stg + row * (D * 2) + ((unit ^ (row & 7)) << 4)) = make_uint4(
+                pack_bf16x2(__uint_as_float(orr[u * 8 + 0]) * inv_l, __uint_as_float(orr[u * 8 + 1]) * inv_l),
+                pack_bf16x2(__uint_as_float(orr[u * 8 + 2]) * inv_l, __uint_as_float(orr[u * 8 + 3]) * inv_l),
+                pack_bf16x2(__uint_as_float(orr[u * 8 + 4]) * inv_l, __uint_as_float(orr[u * 8 + 5]) * inv_l),
+                pack_bf16x2(__uint_as_float(orr[u * 8 + 6]) * inv_l, __uint_as_float(orr[u * 8 + 7]) * inv_l));
+          }
+        }
+        __syncwarp();
+        constexpr int RPI = 32 / UPR;  // rows per warp-wide store
+#pragma unroll
+        for (int i = 0; i < 32 / RPI; ++i) {
+          const int r = quarter * 32 + i * RPI + lane / UPR;
+          const int unit = lane % UPR;
+          if (r < nrows) {
+            const uint4 val = *reinterpret_cast<const uint4*>(stg + r * (D * 2) + ((unit ^ (r & 7)) << 4));
+            uint8_t* dst = reinterpret_cast<uint8_t*>(a.o) +
+                           2 * (((static_cast<size_t>(it.b) * a.Nq + row0 + r) * a.Hq + head) * D) + unit * 16;
+            *reinterpret_cast<uint4*>(dst) = val;
+          }
+        }
+        __syncwarp();
+      } else {
       uint8_t* orow = reinterpret_cast<uint8_t*>(a.o) +
                       2 * (((static_cast<size_t>(it.b) * a.Nq + grow) * a.Hq + head) * D);
 #pragma unroll
@@ -579,6 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pack_bf16x2(__uint_as_float(orr[u * 8 + 4]) * inv_l, __uint_as_float(orr[u * 8 + 5]) * inv_l),
                 pack_bf16x2(__uint_as_float(orr[u * 8 + 6]) * inv_l, __uint_as_float(orr[u * 8 + 7]) * inv_l));
         }
+      }
       }
       if (nX > 0) {
         tc_fence_before();
