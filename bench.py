@@ -212,6 +212,12 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def whole_job_rate(units_per_rank: float, ms_max: float, world: int) -> float:
+    """Units per second for the whole job: every rank processes
+    `units_per_rank` in a step and the step takes the slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 def rank_seed(seed: int, rank: int) -> int:
     """Each rank works on its own batch (weak scaling): distinct seeds."""
     return seed + 100000 * rank
@@ -317,7 +323,7 @@ def bench_prefill(w, args, world, rank, peaks, with_e2e=True):
     ms = max_over_ranks(ms, world)
     eager_ms = max_over_ranks(eager_ms, world)
     flops = prefill_flops(w)
-    tflops = world * flops / (ms * 1e-3) / 1e12
+    tflops = whole_job_rate(flops, ms, world) / 1e12
     peak = peaks["bf16_tflops"]
     out = {
         "ms_per_step": ms, "tflops": tflops, "flops_per_step": flops,
@@ -352,7 +358,7 @@ def bench_prefill(w, args, world, rank, peaks, with_e2e=True):
         ems, _ = time_steps(e2e_step, max(3, args.steps // 4), 2, world, flush)
         torch.cuda.synchronize()
         ems = max_over_ranks(ems, world)
-        out["e2e"] = {"value": world * flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+        out["e2e"] = {"value": whole_job_rate(flops, ems, world) / 1e12, "unit": "TFLOP/s",
                       "ms_per_step": ems,
                       "h2d_bytes_per_step": int(q.nbytes + k.nbytes + v.nbytes),
                       "d2h_bytes_per_step": int(ho.numel() * ho.element_size() + hl.numel() * 4)}
@@ -394,7 +400,7 @@ def bench_decode(w, args, world, rank, peaks, with_e2e=True):
     eager_ms = max_over_ranks(eager_ms, world)
     kvb = decode_kv_bytes(lens, Hkv, d)
     alg = kvb + q.nbytes * 2 + B * Hq * 4
-    gbs = world * alg / (ms * 1e-3) / 1e9
+    gbs = whole_job_rate(alg, ms, world) / 1e9
     peak = peaks["hbm_gbs"]
     out = {
         "metric": "decode KV GB/s", "value": gbs, "unit": "GB/s", "ms_per_step": ms,
@@ -422,7 +428,7 @@ def bench_decode(w, args, world, rank, peaks, with_e2e=True):
 
         ems, _ = time_steps(e2e_step, steps, 3, world)
         ems = max_over_ranks(ems, world)
-        out["e2e"] = {"value": world * alg / (ems * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ems,
+        out["e2e"] = {"value": whole_job_rate(alg, ems, world) / 1e9, "unit": "GB/s", "ms_per_step": ems,
                       "h2d_bytes_per_step": int(q.nbytes), "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4)}
     del tq, tk, tv
     torch.cuda.empty_cache()
@@ -437,9 +443,9 @@ def oracle_prefill_sample(w, seed, batch_elems):
     B = w["B"]
     w1 = dict(w, B=1)
     q, k, v = host_prefill_inputs(w, seed)
-    mk, bm = mask_of(w)
     kinds = {"none": oracle.MASK_NONE, "causal": oracle.MASK_CAUSAL}
     ok = kinds.get(w["mask"], oracle.MASK_BLOCK)
+    bm = oracle.frame_block_map(w["frames"], w["frame_len"]) if ok == oracle.MASK_BLOCK else None
     t0 = time.perf_counter()
     for b in range(min(batch_elems, B)):
         oracle.attn_fwd(q[b:b + 1], k[b:b + 1], v[b:b + 1], 1.0 / math.sqrt(w["d"]), ok, bm)

@@ -59,9 +59,10 @@ def lib() -> ctypes.CDLL:
         L.attn_sync_status.argtypes = [P]
         L.attn_last_error_detail.argtypes = [ctypes.c_char_p, I]
         L.attn_shutdown.argtypes = []
+        L.attn_debug_fault.argtypes = [I]
         L.attn_version.restype = ctypes.c_char_p
         for fn in (L.attn_fwd, L.attn_decode, L.attn_frame_block_map, L.attn_classify, L.attn_plan,
-                   L.attn_sync_status, L.attn_last_error_detail, L.attn_shutdown):
+                   L.attn_sync_status, L.attn_last_error_detail, L.attn_shutdown, L.attn_debug_fault):
             fn.restype = I
         _lib = L
     return _lib
@@ -172,6 +173,12 @@ def plan(mask_kind, block_map, Nq, Nkv):
 def sync_status(stream=None) -> None:
     """Synchronise the stream and raise if a kernel latched a device error."""
     _check(lib().attn_sync_status(_stream_ptr(stream)))
+
+
+def debug_fault(kind: int) -> None:
+    """Test hook: kind 1 makes the next bf16 attn_fwd on this thread run one
+    bounded wait out, so that its sync_status raises ATTN_ERR_DEVICE_TIMEOUT."""
+    _check(lib().attn_debug_fault(kind))
 
 
 def shutdown() -> None:

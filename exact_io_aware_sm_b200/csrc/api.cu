@@ -26,6 +26,7 @@ namespace {
 using namespace eio;
 
 thread_local char g_err[512] = "";
+thread_local int g_fault_next = 0;  // test hook for the next attn_fwd on this thread
 
 int set_err(int code, const char* fmt, ...) {
   va_list ap;
@@ -316,6 +317,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.scale_log2 = scale * 1.4426950408889634f;
   a.causal = mask_kind == ATTN_MASK_CAUSAL;
   a.causal_off = Nkv - Nq;
+  a.fault = g_fault_next;
+  g_fault_next = 0;
   cudaError_t e = launch_prefill_bf16(d, tq, tk, tv, a, s);
   return e == cudaSuccess ? ATTN_OK : cuda_err(e, "prefill launch");
 }
@@ -455,6 +458,12 @@ int attn_shutdown(void) {
   }
   g_ws.clear();
   cudaSetDevice(cur);
+  return ATTN_OK;
+}
+
+int attn_debug_fault(int kind) {
+  if (kind < 0 || kind > 1) return set_err(ATTN_ERR_SHAPE, "unknown fault kind %d", kind);
+  g_fault_next = kind;
   return ATTN_OK;
 }
 

@@ -27,6 +27,7 @@ struct PrefillArgs {
   int num_ctas;         // persistent grid size (SM count)
   float scale_log2;     // scale * log2(e)
   int causal, causal_off;
+  int fault;            // test hook: 1 = CTA 0 skips its first K load (a wait then runs out)
 };
 
 // bf16 tensor-core prefill (tcgen05 / TMA).  d in {64, 128}.

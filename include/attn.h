@@ -213,6 +213,17 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                         const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
                         int Lmax, int d, float scale, void* stream);
 
+/*
+ * attn_debug_fault -- test hook for the device time-out path.
+ *
+ * kind 1: the next bf16 attn_fwd call on this thread makes CTA 0 skip its
+ * first K tile load, so a bounded wait in that CTA runs out (about 2 s);
+ * the kernel then stops cleanly, the context stays usable, and the next
+ * attn_sync_status() returns ATTN_ERR_DEVICE_TIMEOUT.  The outputs of that
+ * call are undefined.  kind 0 clears a pending fault.  Nothing else uses it.
+ */
+int attn_debug_fault(int kind);
+
 /* Library version string, e.g. "exact_io_aware_sm_b200 0.1". */
 const char* attn_version(void);
 

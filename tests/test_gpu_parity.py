@@ -100,14 +100,17 @@ SMALL = [
 
 
 def mask_args(kind, Nq, Nkv, seed):
+    """(mask kind, block map for the library, block map for the oracle): a
+    frame map is built by each side on its own."""
     if kind == "none":
-        return eio.MASK_NONE, None
+        return eio.MASK_NONE, None, None
     if kind == "causal":
-        return eio.MASK_CAUSAL, None
+        return eio.MASK_CAUSAL, None, None
     if kind == "block":
-        return eio.MASK_BLOCK, random_block_map(seed, Nq, Nkv, 0.45)
+        bm = random_block_map(seed, Nq, Nkv, 0.45)
+        return eio.MASK_BLOCK, bm, bm
     L = int(kind[len("frame"):])
-    return eio.MASK_BLOCK, eio.frame_block_map(Nq // L, L)
+    return eio.MASK_BLOCK, eio.frame_block_map(Nq // L, L), oracle.frame_block_map(Nq // L, L)
 
 
 @pytest.mark.parametrize("case", SMALL, ids=[f"{c[-1]}-{c[3]}x{c[4]}-d{c[5]}-g{c[1]//c[2]}" for c in SMALL])
@@ -115,10 +118,10 @@ def test_prefill_small_all_elements(case):
     B, Hq, Hkv, Nq, Nkv, d, kind = case
     seed = 7000 + SMALL.index(case)
     q, k, v = make_inputs(seed, B, Hq, Hkv, Nq, Nkv, d)
-    mk, bm = mask_args(kind, Nq, Nkv, seed)
+    mk, bm, bm_ref = mask_args(kind, Nq, Nkv, seed)
     scale = 1 / math.sqrt(d)
     o, lse = run_fwd(q, k, v, scale, mk, bm)
-    ro, rl = oracle.attn_fwd(q, k, v, scale, mk, bm)
+    ro, rl = oracle.attn_fwd(q, k, v, scale, mk, bm_ref)
     check(o, lse, ro, rl, str(case))
 
 
@@ -184,7 +187,7 @@ def test_config4_frame_block_sparse_full_size():
     o, lse = run_fwd(q, k, v, 1 / math.sqrt(128), eio.MASK_BLOCK, bm)
     special = [0, 1023, 1024, 1039, 1040, 2079, 2080, 3119, 3120, 12345, N - 17, N - 16, N - 1]
     rows = sampled_rows(np.random.default_rng(4), 1, H, N, special, 120)
-    ro, rl = oracle.attn_rows(q, k, v, 1 / math.sqrt(128), rows, oracle.MASK_BLOCK, bm)
+    ro, rl = oracle.attn_rows(q, k, v, 1 / math.sqrt(128), rows, oracle.MASK_BLOCK, oracle.frame_block_map(F, L))
     check_rows(o, lse, ro, rl, rows, "config4")
 
 
@@ -236,6 +239,24 @@ def test_decode_zero_length_and_bad_length():
     assert ei.value.code == 9
     assert torch.all(o2[1].float() == 0) and torch.isneginf(l2[1]).all()
     eio.sync_status()  # cleared
+
+
+def test_device_timeout_is_latched_and_context_recovers():
+    # The hook makes CTA 0 skip one K tile copy, so the MMA issuer's bounded
+    # wait on that stage runs out; the kernel must stop by itself, latch
+    # ATTN_ERR_DEVICE_TIMEOUT and leave the context usable.
+    B, Hq, Hkv, N, d = 1, 4, 2, 300, 128
+    q, k, v = make_inputs(77, B, Hq, Hkv, N, N, d)
+    tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    eio.debug_fault(1)
+    eio.attn_fwd(tq, tk, tv, scale=0.088, mask_kind=eio.MASK_CAUSAL)
+    with pytest.raises(eio.AttnError) as ei:
+        eio.sync_status()
+    assert ei.value.code == 7
+    eio.sync_status()  # the error word was cleared
+    o, lse = run_fwd(q, k, v, 0.088, eio.MASK_CAUSAL, None)
+    ro, rl = oracle.attn_fwd(q, k, v, 0.088, eio.MASK_CAUSAL, None)
+    check(o, lse, ro, rl, "after time-out")
 
 
 def test_config5_gqa_decode_full_size():
