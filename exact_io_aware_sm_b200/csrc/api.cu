@@ -202,21 +202,27 @@ int get_encoder(EncodeTiledFn* fn) {
   return ATTN_OK;
 }
 
-// [B, N, H, d] bf16 viewed as 4-D {d, H, N, B}; box {64, 1, 128, 1}, 128-byte swizzle.
-int make_map(CUtensorMap* m, const void* base, int B, int N, int H, int d) {
+// [B, N, H, d] bf16 viewed as 4-D {d, H, N, B}; box {64, 1, box_rows, 1}, 128-byte swizzle;
+// rows past N read as zeros.
+CUresult encode_map(CUtensorMap* m, const void* base, int B, int N, int H, int d, int box_rows) {
   EncodeTiledFn enc;
-  int rc = get_encoder(&enc);
-  if (rc) return rc;
+  if (get_encoder(&enc)) return CUDA_ERROR_NOT_SUPPORTED;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
                                  static_cast<cuuint64_t>(H) * d * 2,
                                  static_cast<cuuint64_t>(N) * H * d * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+int make_map(CUtensorMap* m, const void* base, int B, int N, int H, int d) {
+  EncodeTiledFn enc;
+  if (int rc = get_encoder(&enc)) return rc;
+  CUresult r = encode_map(m, base, B, N, H, d, 128);
   if (r != CUDA_SUCCESS) return set_err(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return ATTN_OK;
 }
@@ -232,6 +238,15 @@ int check_mask_args(int mask_kind, const uint8_t* block_map) {
 }  // namespace
 
 void eio::set_error_detail(const char* msg) { std::snprintf(g_err, sizeof g_err, "%s", msg); }
+
+bool eio::encode_bf16_map(CUtensorMap* m, const void* base, int B, int N, int H, int d, int box_rows) {
+  const CUresult r = encode_map(m, base, B, N, H, d, box_rows);
+  if (r != CUDA_SUCCESS) {
+    set_err(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return false;
+  }
+  return true;
+}
 
 extern "C" {
 

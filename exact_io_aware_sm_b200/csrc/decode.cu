@@ -1,18 +1,23 @@
 // decode.cu -- single-token GQA decode over a KV cache, split along the keys.
 //
 // Decode reads the whole cache once per step and does about 2 FLOPs per byte
-// (inference page, "Why Decode is Memory-bound"), so this path is built for
-// HBM streaming on the CUDA cores rather than for the tensor cores:
+// (inference page, "Why Decode is Memory-bound"), so this path is built to
+// keep HBM streaming and to spend as few instructions per byte as possible:
 //
-//   decode_split_kernel   one CTA per (split of 512 keys, KV head, sequence).
-//     Each half-warp owns one key row at a time; each lane holds d/16
-//     consecutive elements (16-byte loads for d = 128), so a warp-wide load
-//     moves two full 256-byte rows.  The G query heads of the group share
-//     every K/V row that is loaded.  Scores are reduced with xor-shuffles
-//     inside the half-warp; each half-warp keeps its own online-softmax state
-//     (m, l, acc) over its keys; the halves and the four warps are merged at
-//     the end.  Output: a normalised partial O and its log2-sum-exp per
-//     (sequence, query head, split).
+//   decode_split_kernel   persistent, one CTA per SM, four warps.  A work
+//     item is (sequence b, KV head, split of 512 keys); only splits below the
+//     sequence's length exist.  Every CTA counts the live splits from seqlens
+//     (prefix sums in shared memory), takes an equal share of the items, and
+//     its warps draw items from that share through a shared-memory counter.
+//     Each warp is its own pipeline: a ring of 32-key stages (K and V tiles
+//     brought in by TMA, 128-byte swizzle) that it refills as it consumes, so
+//     every warp keeps up to 48 KB of loads in flight.  The G query heads of
+//     the item share every K/V tile:
+//       S^T (16 keys x 8 heads) = K (16 x d) q^T      mma.m16n8k16, K by ldmatrix
+//       online softmax on the fragment (max over the 16 keys by 3 shuffles)
+//       O^T (d x 8 heads) += V^T (d x 16) P^T        V by ldmatrix.trans, P^T by movmatrix
+//     Heads past G are zero columns.  The output is a normalised partial O
+//     and its log2-sum-exp per (sequence, query head, split).
 //   decode_combine_kernel  one CTA per (sequence, query head): merges the
 //     splits with the block rule of the FlashAttention page, section 2
 //     (rescale each part by 2^(lse_s - lse)), writes O (bf16) and LSE
@@ -20,13 +25,32 @@
 #include <cuda_bf16.h>
 
 #include "kernels.h"
+#include "ptx_sm100.cuh"
 
 namespace eio {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kPairsPerIter = 4;  // key pairs in flight per lane per iteration
+constexpr int kWarps = 4;            // independent pipelines per CTA
+constexpr int kStageKeys = 32;       // keys per pipeline stage
+constexpr int kBoxRows = 16;         // rows per TMA box
+constexpr int kWarpRingBytes = 48 * 1024;
+constexpr int kMaxB = 2048;          // sequences per launch (prefix sums in shared memory)
 constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kRebase = 8.f;       // move the exponent base only when the max grows by more
+
+template <int D>
+struct DCfg {
+  static constexpr int KB = D / 64;                        // 128-byte column blocks per row
+  static constexpr int kBlockBytes = kStageKeys * 128;     // one column block of a tile
+  static constexpr int kTileBytes = KB * kBlockBytes;      // K (or V) of one stage
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int R = kWarpRingBytes / kStageBytes;   // stages per warp: 3 (d=128), 6 (d=64)
+  static constexpr int kOffBars = kWarps * R * kStageBytes;
+  static constexpr int kOffMeta = kOffBars + kWarps * R * 8;
+  static constexpr int kOffPre = kOffMeta + kWarps * R * 16;  // int[kMaxB + 1] prefix, int[kMaxB] lengths
+  static constexpr int kOffCtr = kOffPre + (2 * kMaxB + 1) * 4;
+  static constexpr int kSmem = kOffCtr + 16 + 1024;          // + slack to align the base to 1 KB
+};
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -34,32 +58,36 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-template <int VEC>
-struct Vec;  // VEC bf16 values in one load
-template <>
-struct Vec<8> {
-  using T = uint4;
-};
-template <>
-struct Vec<4> {
-  using T = uint2;
-};
-
-__device__ __forceinline__ void unpack(const uint4& r, float* f) {
-  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ void unpack(const uint2& r, float* f) {
-  const uint32_t w[2] = {r.x, r.y};
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// D (16x8 f32) += A (16x16 bf16, row) * B (16x8 bf16, col).
+__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ int checked_len(const DecodeArgs& a, int b) {
@@ -71,159 +99,268 @@ __device__ __forceinline__ int checked_len(const DecodeArgs& a, int b) {
   return len;
 }
 
+// Producer cursor of one warp (warp-uniform).
+struct Cursor {
+  int b, hkv, split, k, kend;
+};
+
 template <int D, int G>
-__global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeArgs a) {
-  constexpr int VEC = D / 16;  // elements per lane
-  using LoadT = typename Vec<VEC>::T;
-  const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
-  const int len = checked_len(a, b);
-  const int k0 = split * kDecodeChunk;
-  if (k0 >= len) return;
-  const int k1 = min(k0 + kDecodeChunk, len);
+__global__ void __launch_bounds__(kWarps * 32, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const DecodeArgs a) {
+  using C = DCfg<D>;
+  constexpr int R = C::R, KB = C::KB;
+  constexpr int NK = D / 16;  // k-steps of S, m-tiles of O
+  extern __shared__ uint8_t dsmem[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = lane >> 4, sl = lane & 15;
+  const int g = lane >> 2, t = lane & 3;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars) + warp * R;
+  int4* meta = reinterpret_cast<int4*>(smem + C::kOffMeta) + warp * R;
+  int* pre = reinterpret_cast<int*>(smem + C::kOffPre);  // [B + 1] live splits before sequence b
+  int* lens = pre + kMaxB + 1;                             // [B]
+  int* ctr = reinterpret_cast<int*>(smem + C::kOffCtr);
+  uint8_t* ring = smem + warp * R * C::kStageBytes;
+  const uint32_t ring_u32 = smem_u32(ring);
 
-  // q for the G heads of this KV head, this lane's VEC dims, in fp32.
-  float qf[G][VEC];
-  const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(a.q);
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const LoadT r = *reinterpret_cast<const LoadT*>(
-        qb + (static_cast<size_t>(b) * a.Hq + hkv * G + g) * D + sl * VEC);
-    unpack(r, qf[g]);
+  if (threadIdx.x == 0) *ctr = 0;
+  if (lane == 0) {
+    for (int r = 0; r < R; ++r) mbar_init(&bars[r], 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
   }
-
-  float m[G], l[G], acc[G][VEC];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[g][e] = 0.f;
-  }
-
-  const size_t row_stride = static_cast<size_t>(a.Hkv) * D;  // elements between cache rows
-  const __nv_bfloat16* kb =
-      reinterpret_cast<const __nv_bfloat16*>(a.kc) + (static_cast<size_t>(b) * a.Lmax * a.Hkv + hkv) * D + sl * VEC;
-  const __nv_bfloat16* vb =
-      reinterpret_cast<const __nv_bfloat16*>(a.vc) + (static_cast<size_t>(b) * a.Lmax * a.Hkv + hkv) * D + sl * VEC;
-
-  // This warp's contiguous share of the split.
-  const int per_warp = (kDecodeChunk / kWarps);
-  const int w0 = k0 + warp * per_warp;
-  const int w1 = min(w0 + per_warp, k1);
-
-  for (int kb0 = w0; kb0 < w1; kb0 += 2 * kPairsPerIter) {
-    LoadT kr[kPairsPerIter], vr[kPairsPerIter];
-#pragma unroll
-    for (int u = 0; u < kPairsPerIter; ++u) {
-      const int key = kb0 + 2 * u + half;
-      if (key < w1) {
-        kr[u] = __ldcs(reinterpret_cast<const LoadT*>(kb + key * row_stride));
-        vr[u] = __ldcs(reinterpret_cast<const LoadT*>(vb + key * row_stride));
-      } else {
-        kr[u] = LoadT{};
-        vr[u] = LoadT{};
+  if (warp == 0) {
+    int carry = 0;
+    if (lane == 0) pre[0] = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      const int b = b0 + lane;
+      int n = 0;
+      if (b < a.B) {
+        const int len = checked_len(a, b);
+        lens[b] = len;
+        n = (len + kDecodeChunk - 1) / kDecodeChunk;
       }
-    }
-    float s[G][kPairsPerIter];
 #pragma unroll
-    for (int u = 0; u < kPairsPerIter; ++u) {
-      float kf[VEC];
-      unpack(kr[u], kf);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float dot = 0.f;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) dot = fmaf(qf[g][e], kf[e], dot);
-        s[g][u] = dot;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, n, off);
+        if (lane >= off) n += v;
       }
-    }
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1)
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int u = 0; u < kPairsPerIter; ++u) s[g][u] += __shfl_xor_sync(0xffffffffu, s[g][u], off);
-
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int u = 0; u < kPairsPerIter; ++u) {
-        const int key = kb0 + 2 * u + half;
-        s[g][u] = key < w1 ? s[g][u] * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[g][u]);
-      }
-      const float m_new = fmaxf(m[g], mx);
-      // alpha is 0 when m was -inf (and 1 while nothing has been seen yet)
-      const float alpha = m_new == -INFINITY ? 1.f : ex2(m[g] - m_new);
-      const float base = m_new == -INFINITY ? 0.f : m_new;
-      l[g] *= alpha;
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[g][e] *= alpha;
-      m[g] = m_new;
-#pragma unroll
-      for (int u = 0; u < kPairsPerIter; ++u) {
-        const float p = ex2(s[g][u] - base);
-        l[g] += p;
-        float vf[VEC];
-        unpack(vr[u], vf);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[g][e] = fmaf(p, vf[e], acc[g][e]);
-      }
-    }
-  }
-
-  // Merge the two half-warps (same dims, different keys).
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float mo = __shfl_xor_sync(0xffffffffu, m[g], 16);
-    const float lo = __shfl_xor_sync(0xffffffffu, l[g], 16);
-    const float mn = fmaxf(m[g], mo);
-    const float fa = mn == -INFINITY ? 0.f : ex2(m[g] - mn);
-    const float fb = mn == -INFINITY ? 0.f : ex2(mo - mn);
-    l[g] = l[g] * fa + lo * fb;
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const float ao = __shfl_xor_sync(0xffffffffu, acc[g][e], 16);
-      acc[g][e] = acc[g][e] * fa + ao * fb;
-    }
-    m[g] = mn;
-  }
-
-  // Merge the warps through shared memory.
-  __shared__ float s_acc[kWarps][G][D];
-  __shared__ float s_m[kWarps][G], s_l[kWarps][G];
-  if (half == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) s_acc[warp][g][sl * VEC + e] = acc[g][e];
-      if (sl == 0) {
-        s_m[warp][g] = m[g];
-        s_l[warp][g] = l[g];
-      }
+      if (b < a.B) pre[b + 1] = carry + n;
+      carry += __shfl_sync(0xffffffffu, n, 31);
     }
   }
   __syncthreads();
-  const size_t part_base = static_cast<size_t>(b) * a.Hq + hkv * G;
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-    const int g = idx / D, t = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, s_m[w][g]);
-    float L = 0.f, O = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float f = s_m[w][g] == -INFINITY ? 0.f : ex2(s_m[w][g] - M);
-      L += s_l[w][g] * f;
-      O += s_acc[w][g][t] * f;
+
+  const long long total = static_cast<long long>(pre[a.B]) * a.Hkv;
+  const long long i0 = total * blockIdx.x / gridDim.x;
+  const long long i1 = total * (blockIdx.x + 1) / gridDim.x;
+
+  // Next item of this CTA's share into the cursor; false when none is left.
+  auto fetch = [&](Cursor& c) -> bool {
+    int it = 0;
+    if (lane == 0) it = atomicAdd(ctr, 1);
+    it = __shfl_sync(0xffffffffu, it, 0);
+    const long long i = i0 + it;
+    if (i >= i1) return false;
+    const int j = static_cast<int>(i / a.Hkv);
+    c.hkv = static_cast<int>(i % a.Hkv);
+    int lo = 0, hi = a.B;  // largest b with pre[b] <= j
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= j) lo = mid;
+      else hi = mid;
     }
-    const size_t p = (part_base + g) * a.nsplit + split;
-    a.opart[p * D + t] = O / L;
-    if (t == 0) a.lpart[p] = M + __log2f(L);
+    c.b = lo;
+    c.split = j - pre[lo];
+    c.k = c.split * kDecodeChunk;
+    c.kend = min(c.k + kDecodeChunk, lens[lo]);
+    return true;
+  };
+
+  Cursor cur{0, 0, 0, 0, 0};
+  bool more = true;
+  // Issue the next stage of this warp's stream into ring slot `slot`.
+  auto produce = [&](int slot) -> bool {
+    if (cur.k >= cur.kend && !fetch(cur)) return false;
+    const int nvalid = min(kStageKeys, cur.kend - cur.k);
+    const int flags = (cur.k == cur.split * kDecodeChunk ? 1 : 0) | (cur.k + kStageKeys >= cur.kend ? 2 : 0);
+    if (lane == 0) meta[slot] = make_int4(cur.b, cur.hkv, cur.split, nvalid | (flags << 16));
+    const int nbox = nvalid > kBoxRows ? 2 : 1;
+    uint8_t* st = ring + slot * C::kStageBytes;
+    fence_proxy_async_smem();  // earlier generic writes to this slot come first
+    mbar_arrive_expect_tx_elect(&bars[slot], static_cast<uint32_t>(nbox * 2 * KB * kBoxRows * 128));
+    for (int rh = 0; rh < nbox; ++rh) {
+#pragma unroll
+      for (int h = 0; h < KB; ++h) {
+        const int off = h * C::kBlockBytes + rh * kBoxRows * 128;
+        tma_load_4d_elect(st + off, &tmK, &bars[slot], 64 * h, cur.hkv, cur.k + rh * kBoxRows, cur.b);
+        tma_load_4d_elect(st + C::kTileBytes + off, &tmV, &bars[slot], 64 * h, cur.hkv, cur.k + rh * kBoxRows,
+                          cur.b);
+      }
+    }
+    cur.k += kStageKeys;
+    return true;
+  };
+
+  uint32_t produced = 0, consumed = 0;
+  for (int r = 0; r < R && more; ++r) {
+    more = produce(r);
+    if (more) ++produced;
+  }
+  __syncwarp();
+
+  const float sl2 = a.scale_log2;
+  uint32_t qf[NK][2];
+  float acc[NK][4];
+  float m[2], l[2];
+  bool ok = true;
+
+  while (consumed < produced) {
+    const int slot = static_cast<int>(consumed % R);
+    const bool mine = mbar_wait(&bars[slot], (consumed / R) & 1);
+    if (!__all_sync(0xffffffffu, mine)) {
+      ok = false;
+      break;
+    }
+    const int4 md = meta[slot];
+    const int b = md.x, hkv = md.y, split = md.z;
+    const int nvalid = md.w & 0xffff, flags = md.w >> 16;
+    const uint32_t kt = ring_u32 + slot * C::kStageBytes;
+    const uint32_t vt = kt + C::kTileBytes;
+
+    if (flags & 1) {  // first stage of an item: this item's queries, fresh state
+      const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
+                                  (static_cast<size_t>(b) * a.Hq + hkv * G + (g < G ? g : 0)) * D + 2 * t;
+#pragma unroll
+      for (int ks = 0; ks < NK; ++ks) {
+        qf[ks][0] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks) : 0u;
+        qf[ks][1] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8) : 0u;
+      }
+#pragma unroll
+      for (int mt = 0; mt < NK; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
+      m[0] = m[1] = -INFINITY;
+      l[0] = l[1] = 0.f;
+    }
+    if (nvalid < kStageKeys) {
+      // V rows past the sequence (read by the last box, or stale) must be
+      // finite: zero them so that P = 0 there gives exactly 0.
+      uint8_t* vrow = ring + slot * C::kStageBytes + C::kTileBytes;
+      for (int idx = lane; idx < (kStageKeys - nvalid) * KB * 8; idx += 32) {
+        const int r = nvalid + idx / (KB * 8), h = (idx / 8) % KB, c = idx % 8;
+        *reinterpret_cast<uint4*>(vrow + h * C::kBlockBytes + r * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncwarp();
+    }
+
+    const int nch = nvalid > 16 ? 2 : 1;
+    float s[2][4];
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[ch][i] = 0.f;
+      if (ch < nch) {
+        const int r = ch * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int ks = 0; ks < NK; ++ks) {
+          const int cc = (ks & 3) * 2 + (lane >> 4);
+          uint32_t af[4];
+          ldsm_x4(kt + (ks >> 2) * C::kBlockBytes + r * 128 + ((cc ^ (r & 7)) << 4), af);
+          mma_16816(s[ch], af, qf[ks][0], qf[ks][1]);
+        }
+      }
+      // keys past the valid ones carry no weight
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int key = ch * 16 + g + (i >> 1) * 8;
+        if (key >= nvalid) s[ch][i] = -INFINITY;
+      }
+    }
+
+    // Running max per head (2t and 2t+1), over the 32 keys of the stage.
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float v = fmaxf(fmaxf(s[0][j], s[0][j + 2]), fmaxf(s[1][j], s[1][j + 2]));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+      v *= sl2;
+      if (v > m[j] + kRebase) {  // move the base (always on the first stage)
+        const float alpha = ex2(m[j] - v);
+        l[j] *= alpha;
+#pragma unroll
+        for (int mt = 0; mt < NK; ++mt) {
+          acc[mt][j] *= alpha;
+          acc[mt][j + 2] *= alpha;
+        }
+        m[j] = v;
+      }
+    }
+
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+      if (ch < nch) {
+        float p[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          p[i] = ex2(fmaf(s[ch][i], sl2, -m[i & 1]));
+          l[i & 1] += p[i];
+        }
+        const uint32_t b0 = movmatrix_trans(pack_bf16x2(p[0], p[1]));
+        const uint32_t b1 = movmatrix_trans(pack_bf16x2(p[2], p[3]));
+        const int r = ch * 16 + (lane >> 4) * 8 + (lane & 7);
+#pragma unroll
+        for (int mt = 0; mt < NK; ++mt) {
+          const int cc = (mt & 3) * 2 + ((lane >> 3) & 1);
+          uint32_t af[4];
+          ldsm_x4_trans(vt + (mt >> 2) * C::kBlockBytes + r * 128 + ((cc ^ (r & 7)) << 4), af);
+          mma_16816(acc[mt], af, b0, b1);
+        }
+      }
+    }
+
+    if (flags & 2) {  // last stage of the item: normalise and write the partial
+      float lt[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float v = l[j];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        lt[j] = v;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int head = 2 * t + j;
+        if (head < G) {
+          const size_t p = (static_cast<size_t>(b) * a.Hq + hkv * G + head) * a.nsplit + split;
+          const float inv = 1.f / lt[j];
+          float* op = a.opart + p * D;
+#pragma unroll
+          for (int mt = 0; mt < NK; ++mt) {
+            op[16 * mt + g] = acc[mt][j] * inv;
+            op[16 * mt + g + 8] = acc[mt][j + 2] * inv;
+          }
+          if (g == 0) a.lpart[p] = m[j] + __log2f(lt[j]);
+        }
+      }
+    }
+
+    __syncwarp();
+    ++consumed;
+    if (more) {
+      more = produce(static_cast<int>(produced % R));
+      if (more) ++produced;
+    }
+  }
+
+  if (!ok) {
+    if (lane == 0) atomicCAS(a.err, 0, kErrDeviceTimeout);
+    // Let every copy this warp started land before the CTA retires.
+    for (uint32_t c = consumed; c < produced; ++c) mbar_wait(&bars[c % R], (c / R) & 1);
   }
 }
 
@@ -256,10 +393,41 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
 
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
-  dim3 grid(a.nsplit, a.Hkv, a.B);
-  decode_split_kernel<D, G><<<grid, kWarps * 32, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  static int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         DCfg<D>::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_dev = dev;
+  }
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Sequences go in groups of at most kMaxB per launch (the prefix sums live
+  // in shared memory); every array is sequence-major, so a group is a pointer
+  // offset.
+  for (int b0 = 0; b0 < a.B; b0 += kMaxB) {
+    DecodeArgs c = a;
+    c.B = min(kMaxB, a.B - b0);
+    const size_t cache_off = static_cast<size_t>(b0) * a.Lmax * a.Hkv * D * 2;
+    c.q = static_cast<const uint8_t*>(a.q) + static_cast<size_t>(b0) * a.Hq * D * 2;
+    c.kc = static_cast<const uint8_t*>(a.kc) + cache_off;
+    c.vc = static_cast<const uint8_t*>(a.vc) + cache_off;
+    c.seqlens = a.seqlens + b0;
+    c.opart = a.opart + static_cast<size_t>(b0) * a.Hq * a.nsplit * D;
+    c.lpart = a.lpart + static_cast<size_t>(b0) * a.Hq * a.nsplit;
+    CUtensorMap tk, tv;
+    if (!encode_bf16_map(&tk, c.kc, c.B, a.Lmax, a.Hkv, D, kBoxRows) ||
+        !encode_bf16_map(&tv, c.vc, c.B, a.Lmax, a.Hkv, D, kBoxRows))
+      return cudaErrorInvalidValue;
+    const long long items = static_cast<long long>(c.B) * a.nsplit * a.Hkv;
+    const long long want = (items + kWarps - 1) / kWarps;
+    const int grid = static_cast<int>(want < sms ? want : sms);
+    decode_split_kernel<D, G><<<grid, kWarps * 32, DCfg<D>::kSmem, s>>>(tk, tv, c);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, s>>>(a);
   return cudaGetLastError();
 }

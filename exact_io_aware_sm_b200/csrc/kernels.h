@@ -65,6 +65,11 @@ struct DecodeArgs {
 cudaError_t launch_decode(int d, int G, const DecodeArgs& a, cudaStream_t s);
 size_t decode_partial_floats(int B, int Hq, int Lmax, int d);
 
+// TMA map of a [B, N, H, d] bf16 array as {d, H, N, B} with a {64, 1, box_rows, 1}
+// box and 128-byte swizzle; rows past N read as zeros.  False (with the error
+// detail set) if the driver refuses it.
+bool encode_bf16_map(CUtensorMap* m, const void* base, int B, int N, int H, int d, int box_rows);
+
 // Sets the text returned by attn_last_error_detail() on this thread.
 void set_error_detail(const char* msg);
 

@@ -112,7 +112,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
  *   k_cache   device, [B, Lmax, Hkv, d] bf16
  *   v_cache   device, [B, Lmax, Hkv, d] bf16
  *   seqlens   device, int32 [B]; sequence b attends to cache rows
- *             0 .. seqlens[b]-1.  Rows at or above seqlens[b] are never read.
+ *             0 .. seqlens[b]-1.  Rows at or above seqlens[b] never affect
+ *             the result, whatever they hold (NaN included); the kernel may
+ *             read up to 15 of them, never at or beyond Lmax.
  *             A value outside [0, Lmax] latches ATTN_ERR_DEVICE_ARG and that
  *             sequence gets O = 0, LSE = -inf; 0 gives O = 0, LSE = -inf.
  *   o         device, [B, Hq, d] bf16 (written)

@@ -206,6 +206,8 @@ DECODE_SMALL = [
     (2, 16, 2, 2000, 128, [1025, 2000]),
     (2, 8, 1, 700, 64, [700, 3]),
     (5, 4, 2, 64, 64, [64, 1, 33, 2, 63]),
+    (3, 8, 2, 1037, 128, [1037, 1000, 45]),
+    (2, 4, 1, 37, 64, [37, 20]),
 ]
 
 
@@ -220,6 +222,18 @@ def test_decode_small(case):
     o, lse = run_decode(q, kc, vc, lens, 1 / math.sqrt(d))
     ro, rl = oracle.decode(q, kc, vc, lens, 1 / math.sqrt(d))
     check(o, lse, ro, rl, str(case))
+
+
+def test_decode_more_sequences_than_one_launch_holds():
+    # more than 2048 sequences: the split kernel runs in sequence groups
+    B, Hq, Hkv, Lmax, d = 2100, 4, 2, 40, 64
+    lens = (np.arange(B, dtype=np.int64) * 7919 % 41).astype(np.int32)  # 0..40, zeros included
+    q = synthetic.tensor(2200, synthetic.TID_Q, (B, Hq, d))
+    kc = synthetic.kv_cache(2200, synthetic.TID_K, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
+    vc = synthetic.kv_cache(2200, synthetic.TID_V, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
+    o, lse = run_decode(q, kc, vc, lens, 0.125)
+    ro, rl = oracle.decode(q, kc, vc, lens, 0.125)
+    check(o, lse, ro, rl, "B=2100")
 
 
 def test_decode_zero_length_and_bad_length():
