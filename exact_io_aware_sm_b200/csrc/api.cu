@@ -52,9 +52,9 @@ struct DevPlan {
   int* d_order = nullptr;
   uint8_t* d_map = nullptr;  // device copy of the block map (fp32 path)
   int n_pairs = 0;
-  int4* d_pairs = nullptr;   // tensor-core path: Q-tile pairs, their KV lists, visit order
+  int equal_pairs = 0;  // every used slot A visits as many KV tiles as its slot B
+  int4* d_pairs = nullptr;   // tensor-core path: Q-tile pairs in visit order, their KV lists
   int4* d_pkv = nullptr;
-  int* d_porder = nullptr;
 };
 
 struct DevWs {
@@ -75,10 +75,8 @@ void free_plan(DevPlan& p) {
   cudaFree(p.d_map);
   cudaFree(p.d_pairs);
   cudaFree(p.d_pkv);
-  cudaFree(p.d_porder);
   p.d_pairs = nullptr;
   p.d_pkv = nullptr;
-  p.d_porder = nullptr;
   p.d_q = nullptr;
   p.d_kv = nullptr;
   p.d_order = nullptr;
@@ -154,14 +152,19 @@ int get_plan(DevWs& ws, int mask_kind, const uint8_t* block_map, int Nq, int Nkv
   PairPlan pp;
   build_pairs(p, rows_mode != 0, &pp);
   dp.n_pairs = static_cast<int>(pp.pairs.size());
+  dp.equal_pairs = 1;
+  for (const PairTile& t : pp.pairs)
+    if (t.nrowsA > 0 && t.nA != t.nB) dp.equal_pairs = 0;
   static_assert(sizeof(PairTile) == 2 * sizeof(int4) && sizeof(PairKV) == sizeof(int4), "layout");
+  // The kernel visits pairs in this order (most KV tiles first).
+  std::vector<PairTile> sorted(pp.pairs.size());
+  for (size_t i = 0; i < sorted.size(); ++i) sorted[i] = pp.pairs[pp.order[i]];
   int rc;
   if ((rc = upload(&dp.d_q, reinterpret_cast<const int4*>(p.q.data()), p.q.size(), s)) ||
       (rc = upload(&dp.d_kv, reinterpret_cast<const int4*>(p.kv.data()), p.kv.size(), s)) ||
       (rc = upload(&dp.d_order, p.order.data(), p.order.size(), s)) ||
-      (rc = upload(&dp.d_pairs, reinterpret_cast<const int4*>(pp.pairs.data()), 2 * pp.pairs.size(), s)) ||
+      (rc = upload(&dp.d_pairs, reinterpret_cast<const int4*>(sorted.data()), 2 * sorted.size(), s)) ||
       (rc = upload(&dp.d_pkv, reinterpret_cast<const int4*>(pp.kv.data()), pp.kv.size(), s)) ||
-      (rc = upload(&dp.d_porder, pp.order.data(), pp.order.size(), s)) ||
       (map_bytes && need_map && (rc = upload(&dp.d_map, block_map, map_bytes, s)))) {
     free_plan(dp);
     return rc;
@@ -309,13 +312,14 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (int rc = make_map(&tq, q, B, Nq, Hq, d)) return rc;
   if (int rc = make_map(&tk, k, B, Nkv, Hkv, d)) return rc;
   if (int rc = make_map(&tv, v, B, Nkv, Hkv, d)) return rc;
+  CUtensorMap to;
+  if (!encode_bf16_map(&to, o, B, Nq, Hq, d, 16)) return ATTN_ERR_CUDA;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   PrefillArgs a{};
   a.pairs = pl->d_pairs;
   a.kvtiles = pl->d_pkv;
-  a.order = pl->d_porder;
   a.o = o;
   a.lse = lse;
   a.err = ws->d_err;
@@ -332,9 +336,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.scale_log2 = scale * 1.4426950408889634f;
   a.causal = mask_kind == ATTN_MASK_CAUSAL;
   a.causal_off = Nkv - Nq;
+  a.stagger = pl->equal_pairs;
   a.fault = g_fault_next;
   g_fault_next = 0;
-  cudaError_t e = launch_prefill_bf16(d, tq, tk, tv, a, s);
+  cudaError_t e = launch_prefill_bf16(d, tq, tk, tv, to, a, s);
   return e == cudaSuccess ? ATTN_OK : cuda_err(e, "prefill launch");
 }
 

@@ -13,9 +13,8 @@ constexpr int kErrDeviceTimeout = 7;
 constexpr int kErrDeviceArg = 9;
 
 struct PrefillArgs {
-  const int4* pairs;    // per pair: (rowA, nrowsA, rowB, nrowsB), (kv_first, nA, nB, 0)
+  const int4* pairs;    // per pair, most KV tiles first: (rowA, nrowsA, rowB, nrowsB), (kv_first, nA, nB, 0)
   const int4* kvtiles;  // (col0, ncols, flags, 0); flags bit 0 partial for A, bit 1 for B
-  const int* order;     // pairs, most KV tiles first
   void* o;              // [B, Nq, Hq, d] bf16
   float* lse;           // [B, Hq, Nq] or nullptr
   int* err;
@@ -27,12 +26,15 @@ struct PrefillArgs {
   int num_ctas;         // persistent grid size (SM count)
   float scale_log2;     // scale * log2(e)
   int causal, causal_off;
+  int stagger;          // 1: both slots of every pair visit the same number of KV tiles
   int fault;            // test hook: 1 = CTA 0 skips its first K load (a wait then runs out)
 };
 
 // bf16 tensor-core prefill (tcgen05 / TMA).  d in {64, 128}.
+// to: O as {d, Hq, Nq, B} with a {64, 1, 16, 1} box (used by the d = 64 epilogue).
 cudaError_t launch_prefill_bf16(int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                                const CUtensorMap& tv, const PrefillArgs& a, cudaStream_t s);
+                                const CUtensorMap& tv, const CUtensorMap& to, const PrefillArgs& a,
+                                cudaStream_t s);
 int prefill_bf16_smem_bytes(int d);
 
 struct PrefillF32Args {

@@ -79,7 +79,7 @@ struct Cfg {
   static constexpr int kOffBar = kOffStage + (kStageO ? 2 * 128 * D * 2 : 0);
   // q_full[2*QB] q_empty[2*QB] ring_full[R] ring_empty[R] s_full[2] p_full[2]
   // pv_done[2] o_free[2] mma_idle
-  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 2 + 2;  // + mma_idle[2], s_free[2]
+  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 2 + 2 + 1;  // + mma_idle[2], s_free[2], b_first
   static constexpr int kSmem = kOffBar + 8 * kNumBars + 16 + 1024;  // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -159,9 +159,8 @@ __device__ __forceinline__ Item decode_item(const PrefillArgs& a, long long w) {
   rem -= static_cast<long long>(it.b) * a.Hkv * a.HP;
   it.hkv = static_cast<int>(rem / a.HP);
   const int hp = static_cast<int>(rem - static_cast<long long>(it.hkv) * a.HP);
-  const int p = a.order[rank];
-  const int4 x0 = a.pairs[2 * p];
-  const int4 x1 = a.pairs[2 * p + 1];
+  const int4 x0 = a.pairs[2 * rank];
+  const int4 x1 = a.pairs[2 * rank + 1];
   it.rowA = x0.x;
   it.nrowsA = x0.y;
   it.rowB = x0.z;
@@ -194,11 +193,16 @@ __device__ __forceinline__ long long item_index(long long k, long long n_items) 
   return idx < n_items ? idx : -1;
 }
 
-template <int D>
+constexpr bool kFirstLoadsFirst = true;
+
+// STAGGER: both slots of every pair visit the same number of KV tiles, and
+// slot A starts each item after slot B's first exponentials (see below).
+template <int D, bool STAGGER>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmO, const PrefillArgs a) {
   using C = Cfg<D>;
   constexpr int R = C::kRing;
   constexpr int NCH = D / 64;  // 64-element swizzle chunks per row
@@ -218,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_free = pv_done + 2;     // [2]
   uint64_t* mma_idle = o_free + 2;    // [2]
   uint64_t* s_free = mma_idle + 2;    // [2] (separate-P layout): S loaded by the softmax
+  uint64_t* b_first = s_free + 2;     // slot B finished the exponentials of an item's first tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -240,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ring_full[i], 1);
       mbar_init(&ring_empty[i], 2);  // released by both slot issuers
     }
+    mbar_init(b_first, 4);
     mbar_init(&mma_idle[0], 1);
     mbar_init(&mma_idle[1], 1);
     *abort_flag = 0;
@@ -323,6 +329,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d_elect(smem + C::kOffRing + slot * C::kTileBytes + ch * C::kChunkBytes, map,
                               &ring_full[slot], ch * 64, it.hkv, kt.x, it.b);
           ++seq;
+          // At start-up every CTA fills its whole ring at once; let the first
+          // K tile (and the Q tiles issued before it) land before queueing the
+          // rest, so that the first S does not wait behind the whole burst.
+          if (kFirstLoadsFirst && seq == 2 && !wwait(&ring_full[0], 0)) {
+            ok = false;
+            break;
+          }
         }
       }
     }
@@ -447,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_tmem = tmem + lane_off + static_cast<uint32_t>(256 + x * D);
     const uint32_t p_tmem = C::kSepP ? tmem + lane_off + static_cast<uint32_t>(256 + 2 * D + x * 64) : s_tmem;
     const float sl2 = a.scale_log2;
-    uint32_t tcnt = 0;
+    uint32_t tcnt = 0, bcnt = 0;
     bool ok = true;
     // Waits and the abort decision are made warp-uniform, because the warp
     // then executes .sync.aligned tcgen05 instructions together.
@@ -467,6 +480,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = x == 0 ? it.rowA : it.rowB;
       const int head = x == 0 ? it.headA : it.headB;
       if (nrows == 0) continue;  // slot unused in this item
+      // Offset the two slots, so that one slot's exponentials overlap the
+      // other's loads, stores and waits instead of both contending for the
+      // MUFU at once: slot A starts an item when slot B has finished the
+      // exponentials of its first tile.  Done when both slots of every pair
+      // visit the same number of KV tiles (GQA head pairs, Q tiles inside one
+      // frame); the offset then persists through the item.
+      const bool stagger = STAGGER && it.nA > 0;
+      if (stagger && x == 0) {
+        if (!warp_wait(b_first, bcnt & 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (stagger) bcnt++;
       const int grow = row0 + row;
       const int4* kv = a.kvtiles + it.kv_first;
       float m_b = -INFINITY;  // exponent base, log2 units
@@ -528,6 +555,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], p);
           sr[c >> 1] = pack_bf16x2(p.x, p.y);
         }
+        if (stagger && x == 1 && t == 0) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_first);
+        }
         if (C::kSepP && t > 0) {
           // P_X and O_X are free once PV_{t-1} has completed.
           if (!warp_wait(&pv_done[x], (tcnt - 1) & 1)) {
@@ -576,6 +607,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // each warp stores its 32 rows as whole lines: 8 lanes per row.
         constexpr int UPR = D / 8;  // 16-byte units per row
         uint8_t* stg = smem + C::kOffStage + x * (128 * D * 2);
+        // The previous item's stores from this buffer must have read it.
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t orr[32];
@@ -596,20 +630,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pack_bf16x2(__uint_as_float(orr[u * 8 + 6]) * inv_l, __uint_as_float(orr[u * 8 + 7]) * inv_l));
           }
         }
+        // The staging rows are in the 128-byte-swizzled layout of the O map:
+        // one TMA store per 16 rows of the tile (a tile's row count is a
+        // multiple of 16 unless it ends at Nq, where the map clips).
+        fence_proxy_async_smem();
         __syncwarp();
-        constexpr int RPI = 32 / UPR;  // rows per warp-wide store
+        if (lane == 0) {
 #pragma unroll
-        for (int i = 0; i < 32 / RPI; ++i) {
-          const int r = quarter * 32 + i * RPI + lane / UPR;
-          const int unit = lane % UPR;
-          if (r < nrows) {
-            const uint4 val = *reinterpret_cast<const uint4*>(stg + r * (D * 2) + ((unit ^ (r & 7)) << 4));
-            uint8_t* dst = reinterpret_cast<uint8_t*>(a.o) +
-                           2 * (((static_cast<size_t>(it.b) * a.Nq + row0 + r) * a.Hq + head) * D) + unit * 16;
-            *reinterpret_cast<uint4*>(dst) = val;
-          }
+          for (int h = 0; h < 2; ++h)
+            if (quarter * 32 + 16 * h < nrows)
+              tma_store_4d(&tmO, stg + (quarter * 32 + 16 * h) * (D * 2), 0, head, row0 + quarter * 32 + 16 * h,
+                           it.b);
+          bulk_commit();
         }
-        __syncwarp();
       } else {
       uint8_t* orow = reinterpret_cast<uint8_t*>(a.o) +
                       2 * (((static_cast<size_t>(it.b) * a.Nq + grow) * a.Hq + head) * D);
@@ -644,6 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             l > 0.f ? (m_b + __log2f(l)) * kLn2 : -INFINITY;
     }
     if (!ok) fail(kErrDeviceTimeout);
+    if constexpr (C::kStageO) {
+      if (lane == 0) bulk_wait_all();  // O stores complete before the CTA retires
+    }
   }
 
   tc_fence_before();
@@ -652,9 +688,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D>
-cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                     const PrefillArgs& a, cudaStream_t s) {
+template <int D, bool STAGGER>
+cudaError_t launch_ds(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const CUtensorMap& to, const PrefillArgs& a, cudaStream_t s) {
   static int attr_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -662,18 +698,25 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
     // The warpgroup register split is only safe when every thread starts with
     // exactly kLaunchRegs registers.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, prefill_bf16_kernel<D>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, prefill_bf16_kernel<D, STAGGER>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kLaunchRegs || fa.maxThreadsPerBlock < kThreads) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(prefill_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(prefill_bf16_kernel<D, STAGGER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg<D>::kSmem);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
   if (a.n_items == 0) return cudaSuccess;
   const long long grid = a.n_items < a.num_ctas ? a.n_items : a.num_ctas;
-  prefill_bf16_kernel<D><<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmem, s>>>(tq, tk, tv, a);
+  prefill_bf16_kernel<D, STAGGER>
+      <<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmem, s>>>(tq, tk, tv, to, a);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const CUtensorMap& to, const PrefillArgs& a, cudaStream_t s) {
+  return a.stagger ? launch_ds<D, true>(tq, tk, tv, to, a, s) : launch_ds<D, false>(tq, tk, tv, to, a, s);
 }
 
 }  // namespace
@@ -681,9 +724,10 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 int prefill_bf16_smem_bytes(int d) { return d == 64 ? Cfg<64>::kSmem : Cfg<128>::kSmem; }
 
 cudaError_t launch_prefill_bf16(int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                                const CUtensorMap& tv, const PrefillArgs& a, cudaStream_t s) {
-  if (d == 64) return launch_d<64>(tq, tk, tv, a, s);
-  return launch_d<128>(tq, tk, tv, a, s);
+                                const CUtensorMap& tv, const CUtensorMap& to, const PrefillArgs& a,
+                                cudaStream_t s) {
+  if (d == 64) return launch_d<64>(tq, tk, tv, to, a, s);
+  return launch_d<128>(tq, tk, tv, to, a, s);
 }
 
 }  // namespace eio

@@ -122,6 +122,10 @@ def test_plan_block_maps_valid_and_predicate_free(seed):
     # only a tile running past Nkv may need a predicate
     for c0, nc, part in kt:
         assert part == (1 if c0 + nc > Nkv else 0)
+    # Q tiles start on 16-row boundaries and span a multiple of 16 rows unless
+    # they end at Nq (the d=64 epilogue stores O in 16-row boxes)
+    for r0, nr, _, _ in qt:
+        assert r0 % 16 == 0 and (nr % 16 == 0 or r0 + nr == Nq)
 
 
 def test_plan_frame_config_has_no_partial_tiles():
@@ -133,6 +137,15 @@ def test_plan_frame_config_has_no_partial_tiles():
     # live (query row, key) pairs visited == allowed pairs: nothing padded on the key side
     visited = sum(int(r[1]) * int(kt[r[2]:r[2] + r[3], 1].sum()) for r in qt)
     assert visited == 69 * 1040 * 1040
+
+
+@pytest.mark.parametrize("Nq,Nkv", [(1, 1), (300, 300), (1000, 77), (77, 1000), (4097, 4097)])
+def test_plan_q_tiles_on_16_row_boundaries(Nq, Nkv):
+    for kind in (oracle.MASK_NONE, oracle.MASK_CAUSAL):
+        qt, kt = eio.plan(kind, None, Nq, Nkv)
+        assert oracle.check_schedule(kind, None, Nq, Nkv, qt, kt) == 0
+        for r0, nr, _, _ in qt:
+            assert r0 % 16 == 0 and (nr % 16 == 0 or r0 + nr == Nq)
 
 
 def test_plan_causal_counts():
