@@ -96,6 +96,8 @@ SMALL = [
     (1, 2, 2, 240, 240, 128, "frame48"),
     (1, 2, 2, 3120, 3120, 128, "frame1040"),
     (1, 2, 2, 3120, 3120, 64, "frame1040"),
+    (2, 5, 5, 300, 300, 64, "causal"),   # d=64 head pairs, odd head count
+    (1, 3, 3, 517, 700, 64, "causal"),
 ]
 
 
