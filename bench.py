@@ -337,6 +337,15 @@ def bench_prefill(w, args, world, rank, peaks, with_e2e=True):
         "eager_ms_per_step": eager_ms,
         "timing": "CUDA graph replay of one attn_fwd call per step; eager_ms_per_step is the plain call",
     }
+    # The exponentials: one per allowed (query, key) pair, on the MUFU unit
+    # (16 per clock per SM on B200, measured; 148 SMs at the 1965 MHz boost
+    # clock).  At d = 64 this bound is lower than the tensor-core one.
+    n_exp = allowed_pairs(w) * w["B"] * w["Hq"]
+    exp_peak = 16 * 148 * 1.965e9
+    out["roofline_exp"] = {"bound": "alu", "unit": "Gexp/s", "achieved": n_exp / (ms * 1e-3) / 1e9,
+                           "peak": exp_peak / 1e9, "frac": n_exp / (ms * 1e-3) / exp_peak,
+                           "peak_source": "MUFU ex2 16/clk/SM x 148 SMs x 1965 MHz",
+                           "attainable_tflops": flops / (n_exp / exp_peak) / 1e12}
     # attainable at this arithmetic intensity: min(peak, AI * HBM)
     alg_bytes = q.nbytes + k.nbytes + v.nbytes + q.nbytes + lse.numel() * 4  # Q, K, V in; O, LSE out
     ai = flops / alg_bytes
@@ -436,21 +445,60 @@ def bench_decode(w, args, world, rank, peaks, with_e2e=True):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def oracle_prefill_sample(w, seed, batch_elems):
-    """Run the fp64 oracle on `batch_elems` batch elements of the workload;
-    returns (seconds, flops)."""
+def row_allowed(w, i) -> int:
+    """Allowed keys of query row i (per head) of a prefill workload."""
+    N = w["N"]
+    if w["mask"] == "none":
+        return N
+    if w["mask"] == "causal":
+        return i + 1
+    L = w["frame_len"]
+    f = i // L
+    return len({0, max(f - 1, 0), f}) * L
+
+
+def oracle_prefill_call(w, seed, row_budget_flops=2e10):
+    """One bounded pass of the fp64 oracle over the workload: the whole
+    workload when it holds at most `row_budget_flops` algorithmic FLOPs, else
+    a seeded uniform sample of (batch, head, query row) triples of about that
+    size.  Returns a callable that runs the pass and returns its FLOPs, and a
+    description of the sample."""
     import oracle
-    B = w["B"]
-    w1 = dict(w, B=1)
     q, k, v = host_prefill_inputs(w, seed)
     kinds = {"none": oracle.MASK_NONE, "causal": oracle.MASK_CAUSAL}
     ok = kinds.get(w["mask"], oracle.MASK_BLOCK)
     bm = oracle.frame_block_map(w["frames"], w["frame_len"]) if ok == oracle.MASK_BLOCK else None
-    t0 = time.perf_counter()
-    for b in range(min(batch_elems, B)):
-        oracle.attn_fwd(q[b:b + 1], k[b:b + 1], v[b:b + 1], 1.0 / math.sqrt(w["d"]), ok, bm)
-    dt = time.perf_counter() - t0
-    return dt, prefill_flops(w1) * min(batch_elems, B)
+    scale = 1.0 / math.sqrt(w["d"])
+    total = prefill_flops(w)
+    if total <= row_budget_flops:
+        def run():
+            oracle.attn_fwd(q, k, v, scale, ok, bm)
+            return total
+        return run, f"the whole workload ({w['B']} batch elements)"
+    rng = np.random.default_rng(seed)
+    per_row = 4 * w["d"] * allowed_pairs(w) / w["N"]  # mean FLOPs of one (b, h, i) row
+    n = max(1, int(row_budget_flops / per_row))
+    rows = np.stack([rng.integers(0, w["B"], n), rng.integers(0, w["Hq"], n), rng.integers(0, w["N"], n)],
+                    axis=1).astype(np.int32)
+    flops = sum(4 * w["d"] * row_allowed(w, int(i)) for i in rows[:, 2])
+
+    def run():
+        oracle.attn_rows(q, k, v, scale, rows, ok, bm)
+        return flops
+    return run, f"{n} sampled (batch, head, query) rows of the workload"
+
+
+def oracle_prefill_sample(w, seed, min_seconds=10.0, max_passes=200):
+    """Repeat bounded oracle passes until `min_seconds` of CPU work; returns
+    (seconds, flops, description)."""
+    run, desc = oracle_prefill_call(w, seed)
+    dt, fl, n = 0.0, 0, 0
+    while n < max_passes and (n == 0 or dt < min_seconds):
+        t0 = time.perf_counter()
+        fl += run()
+        dt += time.perf_counter() - t0
+        n += 1
+    return dt, fl, f"{desc}, {n} passes, fp64, {dt:.1f} s"
 
 
 def cpu_cores():
@@ -461,29 +509,31 @@ def cpu_cores():
 
 
 def run_reference(args, world, rank):
-    """The oracle as the reference arm, on the same metric and workload."""
+    """The oracle as the reference arm, on the same metric and workload: each
+    step is one bounded pass over the workload (see oracle_prefill_call)."""
     w = WORKLOADS[args.workload]
     if rank != 0:
         return
     import oracle
     oracle.build()
-    seed = w["seed"]
-    steps = []
-    for _ in range(args.warmup if args.warmup < 1 else 1):
-        oracle_prefill_sample(w, seed, 1)
+    run, desc = oracle_prefill_call(w, w["seed"])
+    for _ in range(min(args.warmup, 1)):
+        run()
+    dt, fl = 0.0, 0
     for _ in range(args.steps):
-        dt, fl = oracle_prefill_sample(w, seed, 1)
-        steps.append((dt, fl))
-    ms = 1e3 * sum(s[0] for s in steps) / len(steps)
-    tflops = steps[0][1] / (ms * 1e-3) / 1e12
+        t0 = time.perf_counter()
+        fl += run()
+        dt += time.perf_counter() - t0
+    ms = 1e3 * dt / args.steps
+    tflops = fl / dt / 1e12
     line = {
         "impl": "reference", "metric": "prefill attn TFLOP/s", "value": tflops, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w["desc"], "sample": "one batch element (1 of 8) per step"},
+        "config": {"workload": w["desc"], "sample": f"{desc} per step"},
         "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-                         "sample": "one batch element of the GPT-2 causal workload per step"},
+                         "sample": f"{desc} per step, {args.steps} steps, fp64"},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -551,15 +601,16 @@ def main():
                 extra[name] = {"metric": "prefill attn TFLOP/s", "value": r["tflops"], "unit": "TFLOP/s",
                                "ms_per_step": r["ms_per_step"], "eager_ms_per_step": r["eager_ms_per_step"],
                                "config": {"workload": wx["desc"]},
-                               "roofline": r["roofline"], "gpu_launches": r["gpu_launches"]}
+                               "roofline": r["roofline"], "roofline_exp": r["roofline_exp"],
+                               "gpu_launches": r["gpu_launches"]}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        dt, fl = oracle_prefill_sample(w, rank_seed(w["seed"], 0), w["B"])
+        dt, fl, desc = oracle_prefill_sample(w, rank_seed(w["seed"], 0))
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"the whole workload ({w['B']} batch elements), fp64, {dt:.2f} s"}
+               "sample": desc}
 
     if rank == 0:
         line = {
@@ -570,7 +621,8 @@ def main():
             "config": {"workload": w["desc"], "parallelism": f"replicas x{world} (independent batches)",
                        "l2": "flushed before every step (256 MiB write)",
                        "flops_per_step_per_gpu": head["flops_per_step"]},
-            "roofline": head["roofline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+            "roofline": head["roofline"], "roofline_exp": head["roofline_exp"],
+            "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
             "eager_ms_per_step": head["eager_ms_per_step"], "timing": head["timing"],
             "clocks": sampler.summary(), "cpu_baseline": cpu,
         }
