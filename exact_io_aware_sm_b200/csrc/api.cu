@@ -89,9 +89,10 @@ int get_ws(DevWs** out) {
   if (e != cudaSuccess) return cuda_err(e, "cudaGetDevice");
   DevWs& ws = g_ws[dev];
   if (!ws.d_err) {
-    e = cudaMalloc(&ws.d_err, sizeof(int));
+    // [0] the error word, [1..] decode work-item counters
+    e = cudaMalloc(&ws.d_err, (1 + kDecodeMaxCounters) * sizeof(int));
     if (e != cudaSuccess) return set_err(ATTN_ERR_WORKSPACE, "error word: %s", cudaGetErrorString(e));
-    e = cudaMemset(ws.d_err, 0, sizeof(int));
+    e = cudaMemset(ws.d_err, 0, (1 + kDecodeMaxCounters) * sizeof(int));
     if (e != cudaSuccess) return cuda_err(e, "cudaMemset");
   }
   *out = &ws;
@@ -387,6 +388,7 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   a.opart = ws->d_part;
   a.lpart = ws->d_part + static_cast<size_t>(B) * Hq * a.nsplit * d;
   a.err = ws->d_err;
+  a.counter = ws->d_err + 1;
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;

@@ -7,8 +7,9 @@
 //   decode_split_kernel   persistent, one CTA per SM, four warps.  A work
 //     item is (sequence b, KV head, split of 512 keys); only splits below the
 //     sequence's length exist.  Every CTA counts the live splits from seqlens
-//     (prefix sums in shared memory), takes an equal share of the items, and
-//     its warps draw items from that share through a shared-memory counter.
+//     (prefix sums in shared memory); warps draw items one at a time from a
+//     global counter, so the work evens out to within one item per warp
+//     (the combine kernel resets the counter for the next call).
 //     Each warp is its own pipeline: a ring of 32-key stages (K and V tiles
 //     brought in by TMA, 128-byte swizzle) that it refills as it consumes, so
 //     every warp keeps up to 48 KB of loads in flight.  The G query heads of
@@ -48,8 +49,7 @@ struct DCfg {
   static constexpr int kOffBars = kWarps * R * kStageBytes;
   static constexpr int kOffMeta = kOffBars + kWarps * R * 8;
   static constexpr int kOffPre = kOffMeta + kWarps * R * 16;  // int[kMaxB + 1] prefix, int[kMaxB] lengths
-  static constexpr int kOffCtr = kOffPre + (2 * kMaxB + 1) * 4;
-  static constexpr int kSmem = kOffCtr + 16 + 1024;          // + slack to align the base to 1 KB
+  static constexpr int kSmem = kOffPre + (2 * kMaxB + 1) * 4 + 1024;  // + slack to align the base to 1 KB
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -120,11 +120,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   int4* meta = reinterpret_cast<int4*>(smem + C::kOffMeta) + warp * R;
   int* pre = reinterpret_cast<int*>(smem + C::kOffPre);  // [B + 1] live splits before sequence b
   int* lens = pre + kMaxB + 1;                             // [B]
-  int* ctr = reinterpret_cast<int*>(smem + C::kOffCtr);
   uint8_t* ring = smem + warp * R * C::kStageBytes;
   const uint32_t ring_u32 = smem_u32(ring);
 
-  if (threadIdx.x == 0) *ctr = 0;
   if (lane == 0) {
     for (int r = 0; r < R; ++r) mbar_init(&bars[r], 1);
     fence_mbar_init();
@@ -154,16 +152,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   __syncthreads();
 
   const long long total = static_cast<long long>(pre[a.B]) * a.Hkv;
-  const long long i0 = total * blockIdx.x / gridDim.x;
-  const long long i1 = total * (blockIdx.x + 1) / gridDim.x;
 
-  // Next item of this CTA's share into the cursor; false when none is left.
+  // Next item into the cursor; false when none is left.
   auto fetch = [&](Cursor& c) -> bool {
     int it = 0;
-    if (lane == 0) it = atomicAdd(ctr, 1);
+    if (lane == 0) it = atomicAdd(a.counter, 1);
     it = __shfl_sync(0xffffffffu, it, 0);
-    const long long i = i0 + it;
-    if (i >= i1) return false;
+    const long long i = it;
+    if (i >= total) return false;
     const int j = static_cast<int>(i / a.Hkv);
     c.hkv = static_cast<int>(i % a.Hkv);
     int lo = 0, hi = a.B;  // largest b with pre[b] <= j
@@ -391,6 +387,11 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
   if (t == 0 && a.lse != nullptr) a.lse[bh] = (M + __log2f(W)) * kLn2;
 }
 
+// The split kernels of this call have finished: zero their item counters.
+__global__ void decode_reset_kernel(int* counters, int n) {
+  if (threadIdx.x < n) counters[threadIdx.x] = 0;
+}
+
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
   static int attr_dev = -1;
@@ -415,6 +416,7 @@ cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
     c.kc = static_cast<const uint8_t*>(a.kc) + cache_off;
     c.vc = static_cast<const uint8_t*>(a.vc) + cache_off;
     c.seqlens = a.seqlens + b0;
+    c.counter = a.counter + b0 / kMaxB;
     c.opart = a.opart + static_cast<size_t>(b0) * a.Hq * a.nsplit * D;
     c.lpart = a.lpart + static_cast<size_t>(b0) * a.Hq * a.nsplit;
     CUtensorMap tk, tv;
@@ -429,6 +431,7 @@ cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, s>>>(a);
+  decode_reset_kernel<<<1, 32, 0, s>>>(a.counter, (a.B + kMaxB - 1) / kMaxB);
   return cudaGetLastError();
 }
 

@@ -23,7 +23,8 @@
 namespace {
 
 constexpr size_t kScratchBytes = ATTN_NOALLOC_SCRATCH_BYTES;
-constexpr size_t kErrSlotBytes = 256;  // error word, padded to keep the partials aligned
+constexpr size_t kErrSlotBytes = 256;  // error word and decode item counters, padded to keep the partials aligned
+static_assert((1 + eio::kDecodeMaxCounters) * sizeof(int) <= kErrSlotBytes, "error slot layout");
 
 // The scratch: [error word (256 B)] [O partials] [log2-sum-exp partials].
 // Host code must not use this name as an address (it is a host-side stand-in);
@@ -106,6 +107,7 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
   a.opart = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + kErrSlotBytes);
   a.lpart = a.opart + static_cast<size_t>(B) * Hq * a.nsplit * d;
   a.err = err;
+  a.counter = err + 1;  // zero at load, and zeroed again at the end of every call
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;

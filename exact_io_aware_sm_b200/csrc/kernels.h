@@ -61,9 +61,11 @@ struct DecodeArgs {
   float* opart;     // [B, Hq, nsplit, d]
   float* lpart;     // [B, Hq, nsplit]  (log2 domain)
   int* err;
+  int* counter;     // work-item counters, one per group of 2048 sequences; zero before the call, zeroed after
   int B, Hq, Hkv, Lmax, nsplit;
   float scale_log2;
 };
+constexpr int kDecodeMaxCounters = 63;  // sequence groups one call may need (B <= 65535)
 cudaError_t launch_decode(int d, int G, const DecodeArgs& a, cudaStream_t s);
 size_t decode_partial_floats(int B, int Hq, int Lmax, int d);
 
