@@ -9,7 +9,7 @@
 //     sequence's length exist.  Every CTA counts the live splits from seqlens
 //     (prefix sums in shared memory); warps draw items one at a time from a
 //     global counter, so the work evens out to within one item per warp
-//     (the combine kernel resets the counter for the next call).
+//     (the combine kernel zeroes the counter for the next call).
 //     Each warp is its own pipeline: a ring of 32-key stages (K and V tiles
 //     brought in by TMA, 128-byte swizzle) that it refills as it consumes, so
 //     every warp keeps up to 48 KB of loads in flight.  The G query heads of
@@ -365,6 +365,9 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
   const int bh = blockIdx.x;
   const int b = bh / a.Hq;
   const int t = threadIdx.x;
+  // The split kernels of this call have finished: zero their item counters
+  // for the next call.
+  if (bh == 0 && t < (a.B + kMaxB - 1) / kMaxB) a.counter[t] = 0;
   const int len = checked_len(a, b);
   const int ns = (len + kDecodeChunk - 1) / kDecodeChunk;
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.o) + static_cast<size_t>(bh) * D;
@@ -387,10 +390,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
   if (t == 0 && a.lse != nullptr) a.lse[bh] = (M + __log2f(W)) * kLn2;
 }
 
-// The split kernels of this call have finished: zero their item counters.
-__global__ void decode_reset_kernel(int* counters, int n) {
-  if (threadIdx.x < n) counters[threadIdx.x] = 0;
-}
+
 
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
@@ -431,7 +431,6 @@ cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, s>>>(a);
-  decode_reset_kernel<<<1, 32, 0, s>>>(a.counter, (a.B + kMaxB - 1) / kMaxB);
   return cudaGetLastError();
 }
 
