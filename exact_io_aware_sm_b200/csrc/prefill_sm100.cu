@@ -59,10 +59,11 @@ constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
 struct Cfg {
-  // Of every 8 column pairs of a full tile, this many take the polynomial
-  // exp2 instead of the MUFU unit.  Measured slower on both head dims so far
-  // (the softmax is latency-bound, not MUFU-bound), hence 0.
-  static constexpr int kPolyPairs = 0;
+  // Of every 8 column pairs of a tile, this many take the polynomial exp2
+  // on the FMA pipe instead of the MUFU unit.  At d = 64, where the MUFU is
+  // the bound, one in eight measured about 1 % faster; two in eight, and any
+  // share at d = 128, measured slower.
+  static constexpr int kPolyPairs = D == 64 ? 1 : 0;
   static constexpr int kQBuf = (D == 64) ? 2 : 1;         // Q buffers per slot
   // d = 64 leaves 128 TMEM columns free: P gets its own columns, so the next
   // S of a slot can be computed while the softmax of the current tile runs.
@@ -117,25 +118,26 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
-// 2^x on the FMA pipe, two lanes at a time, for x finite: x = j + f with
-// j = rint(x) (added to 1.5 * 2^23, whose low mantissa bits then hold j) and
-// f in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (relative error
-// 7.5e-5, Remez exchange, coefficients from gen_exp2_poly.py); j is added to
-// the exponent field.  x is clamped at -126 so the result stays a normal
-// number (2^-126 instead of a smaller value).  Full tiles may route part of
-// their exponentials here instead of the MUFU unit (Cfg::kPolyPairs).
+// 2^x on the FMA pipe, two lanes at a time: x = j + f with j = rint(x)
+// (added to 1.5 * 2^23, whose low mantissa bits then hold j) and f in
+// [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (relative error 7.5e-5,
+// Remez exchange, coefficients from gen_exp2_poly.py); j is added to the
+// exponent field.  Results below 2^-126 (and -inf inputs) give 0.  A fixed
+// share of each tile's exponentials may go here instead of the MUFU unit
+// (Cfg::kPolyPairs).
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 magic = make_float2(12582912.0f, 12582912.0f);
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 t = fadd2(x, magic);
+  const float2 xc = make_float2(fmaxf(x.x, -126.0f), fmaxf(x.y, -126.0f));
+  const float2 t = fadd2(xc, magic);
   const float2 jf = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = ffma2(jf, make_float2(-1.0f, -1.0f), x);
+  const float2 f = ffma2(jf, make_float2(-1.0f, -1.0f), xc);
   float2 p = ffma2(make_float2(0.055171669f, 0.055171669f), f, make_float2(0.24261112f, 0.24261112f));
   p = ffma2(p, f, make_float2(0.69326099f, 0.69326099f));
   p = ffma2(p, f, make_float2(0.99992807f, 0.99992807f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+  // Below 2^-126 the result is flushed to zero, as ex2.approx.ftz does; a
+  // masked score (-inf) gives exactly 0.
+  return make_float2(x.x < -126.0f ? 0.f : __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     x.y < -126.0f ? 0.f : __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -546,12 +548,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // p = 2^(s * scale*log2e - base); packed bf16 pairs overwrite sr[0..63].
         float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
         const float2 sl = make_float2(sl2, sl2), nb = make_float2(-base, -base);
-        const bool poly_ok = !__any_sync(0xffffffffu, lim < 128);  // every score finite
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
           const float2 e = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl, nb);
-          const float2 p = (((c >> 1) & 7) < C::kPolyPairs && poly_ok) ? exp2_poly2(e)
-                                                                       : make_float2(ex2(e.x), ex2(e.y));
+          const float2 p = ((c >> 1) & 7) < C::kPolyPairs ? exp2_poly2(e) : make_float2(ex2(e.x), ex2(e.y));
           acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], p);
           sr[c >> 1] = pack_bf16x2(p.x, p.y);
         }
