@@ -423,6 +423,26 @@ def bench_decode(w, args, world, rank, peaks, with_e2e=True):
         "eager_ms_per_step": eager_ms,
         "timing": "CUDA graph replay of one attn_decode call (split + combine) per step",
     }
+    # Two new tokens per sequence (multi-token decode): the same cache bytes
+    # serve both, so tokens per byte double if the time stays.
+    q2 = to_torch(synthetic.tensor(seed + 7, synthetic.TID_Q, (B, 2, Hq, d)), "cuda")
+    o2 = torch.empty_like(q2)
+    l2 = torch.empty((B, Hq, 2), dtype=torch.float32, device="cuda")
+
+    def step2():
+        eio.attn_decode_multi(q2, tk, tv, tl, o=o2, lse=l2, scale=scale)
+
+    if w["Hq"] // w["Hkv"] * 2 <= 8:
+        time_steps(step2, 3, args.warmup, world)
+        g2 = capture_graph(step2)
+        ms2, _ = time_steps(g2.replay, steps, args.warmup, world)
+        eio.sync_status()
+        ms2 = max_over_ranks(ms2, world)
+        out["multi_token_2"] = {"metric": "decode KV GB/s, 2 new tokens per sequence",
+                                "value": whole_job_rate(kvb + q2.numel() * 4 + B * Hq * 8, ms2, world) / 1e9,
+                                "unit": "GB/s", "ms_per_step": ms2,
+                                "tokens_per_s": whole_job_rate(B * 2, ms2, world)}
+    del q2, o2, l2
     if with_e2e:
         # A decode step's input is the new query; the cache stays resident.
         hq_ = to_torch(q, pin=True)
@@ -581,7 +601,8 @@ def main():
                     "steps": d["steps"], "warmup": args.warmup, "ms_per_step": d["ms_per_step"],
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                     "data": "synthetic", "config": d["config"], "roofline": d["roofline"], "e2e": d["e2e"],
-                    "gpu_launches": d["gpu_launches"], "clocks": sampler.summary(), "cpu_baseline": None}
+                    "gpu_launches": d["gpu_launches"], "clocks": sampler.summary(), "cpu_baseline": None,
+                    "multi_token_2": d.get("multi_token_2")}
             print(json.dumps(line), flush=True)
         if world > 1:
             import torch.distributed as dist

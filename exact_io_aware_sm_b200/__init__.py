@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
         P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, I, P]
         L.attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P]
+        L.attn_decode_multi.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
         L.attn_frame_block_map.argtypes = [I, I, P]
         L.attn_classify.argtypes = [I, P, I, I, I, I, P]
         L.attn_plan.argtypes = [I, P, I, I, P, I, P, I, P, P]
@@ -61,7 +62,8 @@ def lib() -> ctypes.CDLL:
         L.attn_shutdown.argtypes = []
         L.attn_debug_fault.argtypes = [I]
         L.attn_version.restype = ctypes.c_char_p
-        for fn in (L.attn_fwd, L.attn_decode, L.attn_frame_block_map, L.attn_classify, L.attn_plan,
+        for fn in (L.attn_fwd, L.attn_decode, L.attn_decode_multi, L.attn_frame_block_map, L.attn_classify,
+                   L.attn_plan,
                    L.attn_sync_status, L.attn_last_error_detail, L.attn_shutdown, L.attn_debug_fault):
             fn.restype = I
         _lib = L
@@ -140,6 +142,26 @@ def attn_decode(q, k_cache, v_cache, seqlens, o=None, lse=None, scale=None, stre
     _check(lib().attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
                              o.data_ptr(), None if lse is None else lse.data_ptr(), B, Hq, Hkv, Lmax,
                              d, float(scale), _stream_ptr(stream)))
+    return o, lse
+
+
+def attn_decode_multi(q, k_cache, v_cache, seqlens, o=None, lse=None, scale=None, stream=None,
+                      want_lse=True):
+    """Decode of the Sq newest tokens per sequence.  q [B,Sq,Hq,d] bf16;
+    caches [B,Lmax,Hkv,d] bf16; seqlens int32 [B] on the device (including
+    the Sq new tokens).  Returns o [B,Sq,Hq,d] and lse [B,Hq,Sq]."""
+    import torch
+    B, Sq, Hq, d = q.shape
+    Lmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(lib().attn_decode_multi(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+                                   o.data_ptr(), None if lse is None else lse.data_ptr(), B, Sq, Hq, Hkv,
+                                   Lmax, d, float(scale), _stream_ptr(stream)))
     return o, lse
 
 

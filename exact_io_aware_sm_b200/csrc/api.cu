@@ -344,16 +344,20 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   return e == cudaSuccess ? ATTN_OK : cuda_err(e, "prefill launch");
 }
 
-int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
-                void* o, float* lse, int B, int Hq, int Hkv, int Lmax, int d, float scale,
-                void* stream) {
+int attn_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                      void* o, float* lse, int B, int Sq, int Hq, int Hkv, int Lmax, int d, float scale,
+                      void* stream) {
   if (!q || !k_cache || !v_cache || !seqlens || !o)
     return set_err(ATTN_ERR_NULL, "q, k_cache, v_cache, seqlens and o must be non-NULL");
-  if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1) return set_err(ATTN_ERR_SHAPE, "B, Hq, Hkv, Lmax must be >= 1");
+  if (B < 1 || Sq < 1 || Hq < 1 || Hkv < 1 || Lmax < 1)
+    return set_err(ATTN_ERR_SHAPE, "B, Sq, Hq, Hkv, Lmax must be >= 1");
   if (Hq % Hkv != 0) return set_err(ATTN_ERR_SHAPE, "Hq (%d) is not a multiple of Hkv (%d)", Hq, Hkv);
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8)
     return set_err(ATTN_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1, 2, 4, 8}, got %d", G);
+  if (G * Sq > 8)
+    return set_err(ATTN_ERR_UNSUPPORTED, "decode needs (Hq/Hkv) * Sq <= 8, got %d * %d", G, Sq);
+  if (static_cast<long long>(B) * Sq * Hq > (1ll << 30)) return set_err(ATTN_ERR_SHAPE, "too many query rows");
   if (d != 64 && d != 128) return set_err(ATTN_ERR_UNSUPPORTED, "decode needs d in {64, 128}");
   if (!(scale > 0.f) || !std::isfinite(scale))
     return set_err(ATTN_ERR_SHAPE, "scale must be positive and finite");
@@ -367,7 +371,7 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   std::lock_guard<std::mutex> lk(g_mu);
   DevWs* ws;
   if (int rc = get_ws(&ws)) return rc;
-  const size_t need = decode_partial_floats(B, Hq, Lmax, d);
+  const size_t need = decode_partial_floats(B * Sq, Hq, Lmax, d);
   if (ws->part_floats < need) {
     cudaDeviceSynchronize();
     cudaFree(ws->d_part);
@@ -386,9 +390,10 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   a.lse = lse;
   a.nsplit = (Lmax + kDecodeChunk - 1) / kDecodeChunk;
   a.opart = ws->d_part;
-  a.lpart = ws->d_part + static_cast<size_t>(B) * Hq * a.nsplit * d;
+  a.lpart = ws->d_part + static_cast<size_t>(B) * Sq * Hq * a.nsplit * d;
   a.err = ws->d_err;
   a.counter = ws->d_err + 1;
+  a.Sq = Sq;
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;
@@ -396,6 +401,12 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   a.scale_log2 = scale * 1.4426950408889634f;
   cudaError_t e = launch_decode(d, G, a, s);
   return e == cudaSuccess ? ATTN_OK : cuda_err(e, "decode launch");
+}
+
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                void* o, float* lse, int B, int Hq, int Hkv, int Lmax, int d, float scale,
+                void* stream) {
+  return attn_decode_multi(q, k_cache, v_cache, seqlens, o, lse, B, 1, Hq, Hkv, Lmax, d, scale, stream);
 }
 
 int attn_frame_block_map(int n_frames, int frame_len, uint8_t* out) {

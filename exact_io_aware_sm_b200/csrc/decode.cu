@@ -5,19 +5,21 @@
 // keep HBM streaming and to spend as few instructions per byte as possible:
 //
 //   decode_split_kernel   persistent, one CTA per SM, four warps.  A work
-//     item is (sequence b, KV head, split of 512 keys); only splits below the
+//     item is (sequence b, KV head, split of 512 keys), for the Sq newest
+//     query tokens of the sequence (Sq = 1: plain decode; Sq > 1: several
+//     tokens at once, each seeing the keys up to its own position); only splits below the
 //     sequence's length exist.  Every CTA counts the live splits from seqlens
 //     (prefix sums in shared memory); warps draw items one at a time from a
 //     global counter, so the work evens out to within one item per warp
 //     (the combine kernel zeroes the counter for the next call).
 //     Each warp is its own pipeline: a ring of 32-key stages (K and V tiles
 //     brought in by TMA, 128-byte swizzle) that it refills as it consumes, so
-//     every warp keeps up to 48 KB of loads in flight.  The G query heads of
-//     the item share every K/V tile:
-//       S^T (16 keys x 8 heads) = K (16 x d) q^T      mma.m16n8k16, K by ldmatrix
+//     every warp keeps up to 48 KB of loads in flight.  The G query heads x Sq
+//     tokens of the item (at most 8) share every K/V tile:
+//       S^T (16 keys x 8 columns) = K (16 x d) q^T     mma.m16n8k16, K by ldmatrix
 //       online softmax on the fragment (max over the 16 keys by 3 shuffles)
-//       O^T (d x 8 heads) += V^T (d x 16) P^T        V by ldmatrix.trans, P^T by movmatrix
-//     Heads past G are zero columns.  The output is a normalised partial O
+//       O^T (d x 8 columns) += V^T (d x 16) P^T       V by ldmatrix.trans, P^T by movmatrix
+//     Columns past G * Sq are zero.  The output is a normalised partial O
 //     and its log2-sum-exp per (sequence, query head, split).
 //   decode_combine_kernel  one CTA per (sequence, query head): merges the
 //     splits with the block rule of the FlashAttention page, section 2
@@ -111,6 +113,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   using C = DCfg<D>;
   constexpr int R = C::R, KB = C::KB;
   constexpr int NK = D / 16;  // k-steps of S, m-tiles of O
+  const int NC = G * a.Sq;    // live columns of the 8: (head, token) pairs of the group
   extern __shared__ uint8_t dsmem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
 
@@ -182,7 +185,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     if (cur.k >= cur.kend && !fetch(cur)) return false;
     const int nvalid = min(kStageKeys, cur.kend - cur.k);
     const int flags = (cur.k == cur.split * kDecodeChunk ? 1 : 0) | (cur.k + kStageKeys >= cur.kend ? 2 : 0);
-    if (lane == 0) meta[slot] = make_int4(cur.b, cur.hkv, cur.split, nvalid | (flags << 16));
+    const int stage = (cur.k - cur.split * kDecodeChunk) / kStageKeys;  // stage of the split, < 16
+    if (lane == 0) meta[slot] = make_int4(cur.b, cur.hkv, cur.split, nvalid | (flags << 16) | (stage << 20));
     const int nbox = nvalid > kBoxRows ? 2 : 1;
     uint8_t* st = ring + slot * C::kStageBytes;
     fence_proxy_async_smem();  // earlier generic writes to this slot come first
@@ -222,17 +226,22 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     }
     const int4 md = meta[slot];
     const int b = md.x, hkv = md.y, split = md.z;
-    const int nvalid = md.w & 0xffff, flags = md.w >> 16;
+    const int nvalid = md.w & 0xffff, flags = (md.w >> 16) & 3;
+    const int k0 = split * kDecodeChunk + (md.w >> 20) * kStageKeys;  // first key of the stage
     const uint32_t kt = ring_u32 + slot * C::kStageBytes;
     const uint32_t vt = kt + C::kTileBytes;
 
     if (flags & 1) {  // first stage of an item: this item's queries, fresh state
+      // Column g of q^T is (head g / Sq, token g % Sq) of this KV group.
+      const bool live = g < NC;
+      const int gc = live ? g : 0;
       const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                                  (static_cast<size_t>(b) * a.Hq + hkv * G + (g < G ? g : 0)) * D + 2 * t;
+                                  ((static_cast<size_t>(b) * a.Sq + gc % a.Sq) * a.Hq + hkv * G + gc / a.Sq) * D +
+                                  2 * t;
 #pragma unroll
       for (int ks = 0; ks < NK; ++ks) {
-        qf[ks][0] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks) : 0u;
-        qf[ks][1] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8) : 0u;
+        qf[ks][0] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks) : 0u;
+        qf[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8) : 0u;
       }
 #pragma unroll
       for (int mt = 0; mt < NK; ++mt)
@@ -253,6 +262,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     }
 
     const int nch = nvalid > 16 ? 2 : 1;
+    // Keys of this stage visible to the lane's two columns 2t, 2t+1: token s
+    // (of Sq, the last at position len - 1) sees keys 0 .. len - Sq + s.
+    int lim[2] = {nvalid, nvalid};
+    if (a.Sq > 1) {
+      const int len = lens[b];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) lim[j] = min(nvalid, len - a.Sq + (2 * t + j) % a.Sq + 1 - k0);
+    }
     float s[2][4];
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
@@ -268,11 +285,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
           mma_16816(s[ch], af, qf[ks][0], qf[ks][1]);
         }
       }
-      // keys past the valid ones carry no weight
+      // keys past the valid ones, and past each token's own position, carry no weight
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int key = ch * 16 + g + (i >> 1) * 8;
-        if (key >= nvalid) s[ch][i] = -INFINITY;
+        if (key >= lim[i & 1]) s[ch][i] = -INFINITY;
       }
     }
 
@@ -302,7 +319,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
         float p[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          p[i] = ex2(fmaf(s[ch][i], sl2, -m[i & 1]));
+          // a column that has seen no key yet keeps m = -inf: its p are 0
+          p[i] = ex2(fmaf(s[ch][i], sl2, m[i & 1] == -INFINITY ? 0.f : -m[i & 1]));
           l[i & 1] += p[i];
         }
         const uint32_t b0 = movmatrix_trans(pack_bf16x2(p[0], p[1]));
@@ -330,17 +348,19 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       }
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        const int head = 2 * t + j;
-        if (head < G) {
-          const size_t p = (static_cast<size_t>(b) * a.Hq + hkv * G + head) * a.nsplit + split;
-          const float inv = 1.f / lt[j];
+        const int col = 2 * t + j;
+        if (col < NC) {
+          const size_t row = (static_cast<size_t>(b) * a.Sq + col % a.Sq) * a.Hq + hkv * G + col / a.Sq;
+          const size_t p = row * a.nsplit + split;
+          // a token may see no key of this split (its position precedes it)
+          const float inv = lt[j] > 0.f ? 1.f / lt[j] : 0.f;
           float* op = a.opart + p * D;
 #pragma unroll
           for (int mt = 0; mt < NK; ++mt) {
             op[16 * mt + g] = acc[mt][j] * inv;
             op[16 * mt + g + 8] = acc[mt][j + 2] * inv;
           }
-          if (g == 0) a.lpart[p] = m[j] + __log2f(lt[j]);
+          if (g == 0) a.lpart[p] = lt[j] > 0.f ? m[j] + __log2f(lt[j]) : -INFINITY;
         }
       }
     }
@@ -362,8 +382,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
 
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
-  const int bh = blockIdx.x;
-  const int b = bh / a.Hq;
+  const int bh = blockIdx.x;  // query row (b, token, head) of [B, Sq, Hq]
+  const int b = bh / (a.Sq * a.Hq);
+  const int lse_at = (b * a.Hq + bh % a.Hq) * a.Sq + (bh / a.Hq) % a.Sq;  // LSE is [B, Hq, Sq]
   const int t = threadIdx.x;
   // The split kernels of this call have finished: zero their item counters
   // for the next call.
@@ -371,15 +392,15 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
   const int len = checked_len(a, b);
   const int ns = (len + kDecodeChunk - 1) / kDecodeChunk;
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.o) + static_cast<size_t>(bh) * D;
-  if (ns == 0) {
-    o[t] = __float2bfloat16_rn(0.f);
-    if (t == 0 && a.lse != nullptr) a.lse[bh] = -INFINITY;
-    return;
-  }
   const float* lp = a.lpart + static_cast<size_t>(bh) * a.nsplit;
   const float* op = a.opart + static_cast<size_t>(bh) * a.nsplit * D;
   float M = -INFINITY;
   for (int s = 0; s < ns; ++s) M = fmaxf(M, lp[s]);
+  if (M == -INFINITY) {  // no key visible to this query row
+    o[t] = __float2bfloat16_rn(0.f);
+    if (t == 0 && a.lse != nullptr) a.lse[lse_at] = -INFINITY;
+    return;
+  }
   float W = 0.f, O = 0.f;
   for (int s = 0; s < ns; ++s) {
     const float w = ex2(lp[s] - M);
@@ -387,7 +408,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
     O = fmaf(w, op[static_cast<size_t>(s) * D + t], O);
   }
   o[t] = __float2bfloat16_rn(O / W);
-  if (t == 0 && a.lse != nullptr) a.lse[bh] = (M + __log2f(W)) * kLn2;
+  if (t == 0 && a.lse != nullptr) a.lse[lse_at] = (M + __log2f(W)) * kLn2;
 }
 
 
@@ -412,13 +433,13 @@ cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
     DecodeArgs c = a;
     c.B = min(kMaxB, a.B - b0);
     const size_t cache_off = static_cast<size_t>(b0) * a.Lmax * a.Hkv * D * 2;
-    c.q = static_cast<const uint8_t*>(a.q) + static_cast<size_t>(b0) * a.Hq * D * 2;
+    c.q = static_cast<const uint8_t*>(a.q) + static_cast<size_t>(b0) * a.Sq * a.Hq * D * 2;
     c.kc = static_cast<const uint8_t*>(a.kc) + cache_off;
     c.vc = static_cast<const uint8_t*>(a.vc) + cache_off;
     c.seqlens = a.seqlens + b0;
     c.counter = a.counter + b0 / kMaxB;
-    c.opart = a.opart + static_cast<size_t>(b0) * a.Hq * a.nsplit * D;
-    c.lpart = a.lpart + static_cast<size_t>(b0) * a.Hq * a.nsplit;
+    c.opart = a.opart + static_cast<size_t>(b0) * a.Sq * a.Hq * a.nsplit * D;
+    c.lpart = a.lpart + static_cast<size_t>(b0) * a.Sq * a.Hq * a.nsplit;
     CUtensorMap tk, tv;
     if (!encode_bf16_map(&tk, c.kc, c.B, a.Lmax, a.Hkv, D, kBoxRows) ||
         !encode_bf16_map(&tv, c.vc, c.B, a.Lmax, a.Hkv, D, kBoxRows))
@@ -430,7 +451,7 @@ cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  decode_combine_kernel<D><<<a.B * a.Hq, D, 0, s>>>(a);
+  decode_combine_kernel<D><<<a.B * a.Sq * a.Hq, D, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -108,6 +108,7 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
   a.lpart = a.opart + static_cast<size_t>(B) * Hq * a.nsplit * d;
   a.err = err;
   a.counter = err + 1;  // zero at load, and zeroed again at the end of every call
+  a.Sq = 1;
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;

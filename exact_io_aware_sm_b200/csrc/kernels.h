@@ -52,17 +52,18 @@ cudaError_t launch_prefill_f32(int d, const PrefillF32Args& a, cudaStream_t s);
 // Split-KV decode.
 constexpr int kDecodeChunk = 512;
 struct DecodeArgs {
-  const void* q;    // [B, Hq, d] bf16
+  const void* q;    // [B, Sq, Hq, d] bf16
   const void* kc;   // [B, Lmax, Hkv, d] bf16
   const void* vc;
   const int32_t* seqlens;
-  void* o;          // [B, Hq, d] bf16
-  float* lse;       // [B, Hq] or nullptr
-  float* opart;     // [B, Hq, nsplit, d]
-  float* lpart;     // [B, Hq, nsplit]  (log2 domain)
+  void* o;          // [B, Sq, Hq, d] bf16
+  float* lse;       // [B, Hq, Sq] or nullptr
+  float* opart;     // [B, Sq, Hq, nsplit, d]
+  float* lpart;     // [B, Sq, Hq, nsplit]  (log2 domain)
   int* err;
   int* counter;     // work-item counters, one per group of 2048 sequences; zero before the call, zeroed after
   int B, Hq, Hkv, Lmax, nsplit;
+  int Sq;           // query tokens per sequence (the newest Sq positions); G * Sq <= 8
   float scale_log2;
 };
 constexpr int kDecodeMaxCounters = 63;  // sequence groups one call may need (B <= 65535)

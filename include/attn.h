@@ -128,6 +128,30 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
                 void* stream);
 
 /*
+ * attn_decode_multi -- decode of the Sq newest tokens of each sequence at
+ * once (several tokens per step, e.g. multi-token prediction), over the same
+ * KV cache read once for all of them.
+ *
+ * Passage: as attn_decode; the tokens' own K/V rows are already in the cache
+ * (positions seqlens[b]-Sq .. seqlens[b]-1), and token s (0-based) attends to
+ * rows 0 .. seqlens[b]-Sq+s: the last Sq rows of a causal prefill with
+ * Nq = Sq and Nkv = seqlens[b] (bottom-right aligned causal mask).
+ *
+ *   q         device, [B, Sq, Hq, d] bf16
+ *   k_cache, v_cache, seqlens   as attn_decode
+ *   o         device, [B, Sq, Hq, d] bf16 (written)
+ *   lse       device, [B, Hq, Sq] fp32 (written); may be NULL
+ * A token that sees no row (seqlens[b] - Sq + s < 0) gets O = 0, LSE = -inf.
+ * Limits: as attn_decode, and (Hq / Hkv) * Sq <= 8 (the query heads of a KV
+ * group times the tokens share one 8-column MMA operand), else
+ * ATTN_ERR_UNSUPPORTED.  Sq = 1 is attn_decode.
+ * Scratch: B*Sq*Hq*ceil(Lmax/512)*(d+1) floats of library workspace.
+ */
+int attn_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                      void* o, float* lse, int B, int Sq, int Hq, int Hkv, int Lmax, int d, float scale,
+                      void* stream);
+
+/*
  * attn_frame_block_map -- block map of the frame-aligned video mask.
  *
  * Passage: TPU attention guide, step 3 (the mask's live region follows frame

@@ -226,6 +226,70 @@ def test_decode_small(case):
     check(o, lse, ro, rl, str(case))
 
 
+def oracle_decode_multi(q, kc, vc, lens, scale):
+    """Sq newest tokens per sequence = the last Sq rows of a causal prefill
+    with Nq = Sq, Nkv = len (bottom-right alignment)."""
+    B, Sq, Hq, d = q.shape
+    o = np.zeros((B, Sq, Hq, d))
+    lse = np.full((B, Hq, Sq), -np.inf)
+    for b in range(B):
+        L = int(lens[b])
+        if L == 0:
+            continue
+        ob, lb = oracle.attn_fwd(q[b:b + 1], kc[b:b + 1, :L], vc[b:b + 1, :L], scale, oracle.MASK_CAUSAL, None)
+        o[b], lse[b] = ob[0], lb[0]
+    return o, lse
+
+
+DECODE_MULTI = [
+    # B, Sq, Hq, Hkv, Lmax, d, lens
+    (3, 2, 8, 2, 1100, 128, [1100, 513, 1]),
+    (4, 4, 4, 2, 700, 64, [700, 3, 512, 2]),
+    (2, 8, 2, 2, 600, 64, [600, 5]),
+    (3, 2, 2, 1, 64, 128, [64, 0, 33]),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_MULTI)
+def test_decode_multi_token(case):
+    B, Sq, Hq, Hkv, Lmax, d, lens = case
+    lens = np.array(lens, np.int32)
+    seed = 2300 + DECODE_MULTI.index(case)
+    q = synthetic.tensor(seed, synthetic.TID_Q, (B, Sq, Hq, d))
+    kc = synthetic.kv_cache(seed, synthetic.TID_K, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)  # NaN past len
+    vc = synthetic.kv_cache(seed, synthetic.TID_V, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
+    o, lse = eio.attn_decode_multi(dev_bf16(q), dev_bf16(kc), dev_bf16(vc), torch.from_numpy(lens).cuda(),
+                                   scale=1 / math.sqrt(d))
+    eio.sync_status()
+    ro, rl = oracle_decode_multi(q, kc, vc, lens, 1 / math.sqrt(d))
+    check(o, lse, ro, rl, str(case))
+
+
+def test_decode_multi_equals_single_at_sq1():
+    B, Hq, Hkv, Lmax, d = 4, 8, 2, 900, 128
+    lens = np.array([900, 1, 511, 512], np.int32)
+    q = synthetic.tensor(2400, synthetic.TID_Q, (B, Hq, d))
+    kc = dev_bf16(synthetic.kv_cache(2400, synthetic.TID_K, B, Lmax, Hkv, d, lens))
+    vc = dev_bf16(synthetic.kv_cache(2400, synthetic.TID_V, B, Lmax, Hkv, d, lens))
+    tl = torch.from_numpy(lens).cuda()
+    o1, l1 = eio.attn_decode(dev_bf16(q), kc, vc, tl)
+    o2, l2 = eio.attn_decode_multi(dev_bf16(q).reshape(B, 1, Hq, d), kc, vc, tl)
+    eio.sync_status()
+    assert torch.equal(o1, o2.reshape(B, Hq, d)) and torch.equal(l1, l2.reshape(B, Hq))
+
+
+def test_decode_multi_full_size_mtp2():
+    B, Sq, Hq, Hkv, Lmax, d = 64, 2, 32, 8, 8192, 128
+    lens = synthetic.seqlens(2005, B)
+    q = synthetic.tensor(1005, synthetic.TID_Q, (B, Sq, Hq, d))
+    kc = synthetic.kv_cache(1005, synthetic.TID_K, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
+    vc = synthetic.kv_cache(1005, synthetic.TID_V, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
+    o, lse = eio.attn_decode_multi(dev_bf16(q), dev_bf16(kc), dev_bf16(vc), torch.from_numpy(lens).cuda())
+    eio.sync_status()
+    ro, rl = oracle_decode_multi(q, kc, vc, lens, 1 / math.sqrt(d))
+    check(o, lse, ro, rl, "mtp2 full size")
+
+
 def test_decode_more_sequences_than_one_launch_holds():
     # more than 2048 sequences: the split kernel runs in sequence groups
     B, Hq, Hkv, Lmax, d = 2100, 4, 2, 40, 64
