@@ -48,6 +48,7 @@ def lib() -> ctypes.CDLL:
         P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
         L.ora_attn_rows.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, P, P, I, P, P]
         L.ora_attn_fwd.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, P, P, P]
+        L.ora_attn_bwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, D, I, P, P, P, P]
         L.ora_decode.argtypes = [P, P, P, I, P, I, I, I, I, I, D, P, P]
         L.ora_online_softmax.argtypes = [P, P, I, P, P, P, P, P]
         L.ora_merge_partials.argtypes = [P, P, I, I, P, P]
@@ -96,6 +97,25 @@ def attn_fwd(q, k, v, scale, mask_kind=MASK_NONE, block_map=None):
     if rc != 0:
         raise ValueError("ora_attn_fwd rejected its arguments")
     return o, lse
+
+
+def attn_bwd(q, k, v, dout, scale, mask_kind=MASK_NONE, block_map=None):
+    """Gradients (dQ, dK, dV) in fp64 for the upstream gradient dout of O.
+    q, dout [B,Nq,Hq,d]; k, v [B,Nkv,Hkv,d] (one dtype: bf16 bits, fp32, fp64)."""
+    q, k, v, dout = (np.ascontiguousarray(x) for x in (q, k, v, dout))
+    B, Nq, Hq, d = q.shape
+    Nkv, Hkv = k.shape[1], k.shape[2]
+    dt = _dtype_code(q)
+    assert all(_dtype_code(x) == dt for x in (k, v, dout))
+    dq = np.zeros((B, Nq, Hq, d), np.float64)
+    dk = np.zeros((B, Nkv, Hkv, d), np.float64)
+    dv = np.zeros((B, Nkv, Hkv, d), np.float64)
+    bm = _bm(block_map)
+    rc = lib().ora_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), dt, B, Hq, Hkv, Nq, Nkv, d, float(scale),
+                            mask_kind, _ptr(bm), _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise ValueError("ora_attn_bwd rejected its arguments")
+    return dq, dk, dv
 
 
 def attn_rows(q, k, v, scale, rows, mask_kind=MASK_NONE, block_map=None):

@@ -393,3 +393,95 @@ int ora_check_schedule(int mask_kind, const uint8_t *block_map, int Nq, int Nkv,
   free(colseen);
   return rc;
 }
+
+/*
+ * Gradients of attention for a given upstream gradient dO ("FlashAttention:
+ * memory-saving exact attention", section 4: the backward needs S and P,
+ * which the fast path recomputes from Q, K, V and the saved (m, l); the
+ * oracle simply materialises them again from the definition).  For one
+ * (b, hq) with hkv = hq / G and allowed pairs (i, j):
+ *
+ *   P[i][j]  = exp(S[i][j] - m_i) / l_i        (the forward's softmax)
+ *   dV[j]   += P[i][j] * dO[i]                 (O = P V)
+ *   dP[i][j] = dO[i] . V[j]
+ *   D_i      = sum_j P[i][j] * dP[i][j]        (softmax Jacobian: dS = P (dP - D))
+ *   dS[i][j] = P[i][j] * (dP[i][j] - D_i)
+ *   dQ[i]    = scale * sum_j dS[i][j] * K[j]   (S = scale Q K^T)
+ *   dK[j]   += scale * dS[i][j] * Q[i]
+ *
+ * dK and dV of a KV head sum over the G query heads that share it.  Masked
+ * pairs carry no gradient; a row without allowed keys has dQ = 0.
+ * Layouts: q, dO [B,Nq,Hq,d]; k, v [B,Nkv,Hkv,d] (dtype as ora_attn_fwd);
+ * dq [B,Nq,Hq,d], dk and dv [B,Nkv,Hkv,d], all fp64.  Returns 0, or -1 on bad
+ * arguments.
+ */
+int ora_attn_bwd(const void *q, const void *k, const void *v, const void *dout, int dtype, int B,
+                 int Hq, int Hkv, int Nq, int Nkv, int d, double scale, int mask_kind,
+                 const uint8_t *block_map, double *dq, double *dk, double *dv) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || Nq < 0 || Nkv < 0) return -1;
+  if (mask_kind == ORA_MASK_BLOCK && !block_map) return -1;
+  int G = Hq / Hkv;
+  memset(dq, 0, sizeof(double) * (size_t)B * Nq * Hq * d);
+  memset(dk, 0, sizeof(double) * (size_t)B * Nkv * Hkv * d);
+  memset(dv, 0, sizeof(double) * (size_t)B * Nkv * Hkv * d);
+  long slices = (long)B * Hkv;
+#pragma omp parallel
+  {
+    size_t n = (size_t)(Nkv > 0 ? Nkv : 1);
+    double *S = (double *)malloc(sizeof(double) * n);
+    double *P = (double *)malloc(sizeof(double) * n);
+    double *dP = (double *)malloc(sizeof(double) * n);
+#pragma omp for schedule(dynamic, 1)
+    for (long sl = 0; sl < slices; ++sl) {  /* one (b, hkv): its dK, dV are private to it */
+      int b = (int)(sl / Hkv), hkv = (int)(sl % Hkv);
+      size_t kv_base = ((size_t)b * Nkv * Hkv + hkv) * d, kv_stride = (size_t)Hkv * d;
+      for (int g = 0; g < G; ++g) {
+        int hq = hkv * G + g;
+        for (int i = 0; i < Nq; ++i) {
+          size_t q_off = (((size_t)b * Nq + i) * Hq + hq) * d;
+          double m = -INFINITY;
+          for (int j = 0; j < Nkv; ++j) {
+            if (!ora_allowed(mask_kind, block_map, Nq, Nkv, i, j)) {
+              S[j] = -INFINITY;
+              continue;
+            }
+            double acc = 0.0;
+            for (int t = 0; t < d; ++t)
+              acc += ld(q, dtype, q_off + t) * ld(k, dtype, kv_base + (size_t)j * kv_stride + t);
+            S[j] = acc * scale;
+            if (S[j] > m) m = S[j];
+          }
+          if (m == -INFINITY) continue; /* no allowed key: no gradient */
+          double l = 0.0;
+          for (int j = 0; j < Nkv; ++j) {
+            P[j] = S[j] == -INFINITY ? 0.0 : exp(S[j] - m);
+            l += P[j];
+          }
+          double D = 0.0;
+          for (int j = 0; j < Nkv; ++j) {
+            P[j] /= l;
+            dP[j] = 0.0;
+            if (P[j] == 0.0 && S[j] == -INFINITY) continue;
+            for (int t = 0; t < d; ++t)
+              dP[j] += ld(dout, dtype, q_off + t) * ld(v, dtype, kv_base + (size_t)j * kv_stride + t);
+            D += P[j] * dP[j];
+          }
+          for (int j = 0; j < Nkv; ++j) {
+            if (S[j] == -INFINITY) continue;
+            double ds = P[j] * (dP[j] - D);
+            size_t kj = kv_base + (size_t)j * kv_stride;
+            for (int t = 0; t < d; ++t) {
+              dq[q_off + t] += scale * ds * ld(k, dtype, kj + t);
+              dk[kj + t] += scale * ds * ld(q, dtype, q_off + t);
+              dv[kj + t] += P[j] * ld(dout, dtype, q_off + t);
+            }
+          }
+        }
+      }
+    }
+    free(S);
+    free(P);
+    free(dP);
+  }
+  return 0;
+}

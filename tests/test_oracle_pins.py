@@ -401,3 +401,85 @@ def test_check_schedule_detects_planted_mistakes():
     # a diagonal tile claimed full
     assert oracle.check_schedule(oracle.MASK_CAUSAL, None, N, N, good_q,
                                  [(0, 32, 0), (0, 32, 0), (32, 32, 1)]) == 4
+
+
+# --------------------------------------------------------------------------
+# Gradients (the backward pass): torch autograd, finite differences, invariants
+# --------------------------------------------------------------------------
+
+def _sdpa_grads(q, k, v, dout, scale, allowed):
+    """dQ, dK, dV of torch SDPA (fp64, CPU, math path, torch's own GQA
+    mapping) for the upstream gradient dout."""
+    Q, K, V = (torch.from_numpy(x).permute(0, 2, 1, 3).clone().requires_grad_(True) for x in (q, k, v))
+    G = Q.shape[1] // K.shape[1]
+    O = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=torch.from_numpy(allowed),
+                                                         scale=scale, enable_gqa=G > 1)
+    O.backward(torch.from_numpy(dout).permute(0, 2, 1, 3))
+    return tuple(t.grad.permute(0, 2, 1, 3).numpy() for t in (Q, K, V))
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_oracle_gradients_match_torch_autograd(case):
+    B, Hq, Hkv, Nq, Nkv, d, kind = case
+    seed = (hash(case) & 0xFFFF) + 17
+    q, k, v = rnd((B, Nq, Hq, d), seed), rnd((B, Nkv, Hkv, d), seed + 1), rnd((B, Nkv, Hkv, d), seed + 2)
+    dout = rnd((B, Nq, Hq, d), seed + 3)
+    bm = None
+    if kind == oracle.MASK_BLOCK:
+        rng = np.random.default_rng(seed)
+        bm = (rng.random(((Nq + 15) // 16, (Nkv + 15) // 16)) < 0.6).astype(np.uint8)
+        bm[:, 0] = 1
+    if kind == oracle.MASK_CAUSAL and Nq > Nkv:
+        pytest.skip("rows without keys are pinned separately")
+    scale = 1.0 / math.sqrt(d)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, scale, kind, bm)
+    rq, rk, rv = _sdpa_grads(q, k, v, dout, scale, _allowed_matrix(kind, bm, Nq, Nkv))
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        np.testing.assert_allclose(got, ref, atol=1e-11, rtol=1e-10)
+
+
+def test_oracle_gradients_match_finite_differences():
+    # central differences of the forward oracle's loss sum(O * dout)
+    B, Hq, Hkv, Nq, Nkv, d = 1, 4, 2, 6, 9, 3
+    rng = np.random.default_rng(5)
+    q, k, v, dout = (rng.standard_normal(s) for s in ((B, Nq, Hq, d), (B, Nkv, Hkv, d), (B, Nkv, Hkv, d),
+                                                        (B, Nq, Hq, d)))
+    scale, kind = 0.7, oracle.MASK_CAUSAL
+    grads = oracle.attn_bwd(q, k, v, dout, scale, kind)
+
+    def loss(q_, k_, v_):
+        return float((oracle.attn_fwd(q_, k_, v_, scale, kind)[0] * dout).sum())
+
+    h = 1e-5
+    for which, x in enumerate((q, k, v)):
+        for flat in rng.choice(x.size, size=6, replace=False):
+            idx = np.unravel_index(flat, x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p, args_m = [q, k, v], [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - grads[which][idx]) <= 1e-7 + 1e-6 * abs(fd), (which, idx, fd, grads[which][idx])
+
+
+def test_oracle_gradient_invariants():
+    B, Hq, Hkv, Nq, Nkv, d = 2, 6, 3, 40, 70, 16
+    q, k, v, dout = rnd((B, Nq, Hq, d), 71), rnd((B, Nkv, Hkv, d), 72), rnd((B, Nkv, Hkv, d), 73), \
+        rnd((B, Nq, Hq, d), 74)
+    scale = 0.25
+    # bottom-right causal: rows see keys up to i + 30, so keys 0..30 are seen by every row
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, scale, oracle.MASK_CAUSAL)
+    # each row's dS sums to zero over its keys (softmax is shift invariant), so sum_j dK_j = 0
+    np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-11)
+    # with dout = 1 every row's probabilities sum to one: sum_j dV_j = rows x query heads
+    _, _, dv1 = oracle.attn_bwd(q, k, v, np.ones_like(dout), scale, oracle.MASK_CAUSAL)
+    np.testing.assert_allclose(dv1.sum(axis=1), Nq * (Hq // Hkv), rtol=1e-12)
+    # keys that no row may see get no gradient; neither does a row that sees no key
+    bm = np.ones(((Nq + 15) // 16, (Nkv + 15) // 16), np.uint8)
+    bm[:, 2] = 0           # keys 32..47 masked for everyone
+    bm[1, :] = 0           # rows 16..31 see nothing
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, scale, oracle.MASK_BLOCK, bm)
+    assert not dk[:, 32:48].any() and not dv[:, 32:48].any()
+    assert not dq[:, 16:32].any()
+    assert dk[:, :32].any() and dq[:, :16].any()
