@@ -54,6 +54,7 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, I, P]
         L.attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P]
         L.attn_decode_multi.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+        L.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
         L.attn_frame_block_map.argtypes = [I, I, P]
         L.attn_classify.argtypes = [I, P, I, I, I, I, P]
         L.attn_plan.argtypes = [I, P, I, I, P, I, P, I, P, P]
@@ -62,7 +63,8 @@ def lib() -> ctypes.CDLL:
         L.attn_shutdown.argtypes = []
         L.attn_debug_fault.argtypes = [I]
         L.attn_version.restype = ctypes.c_char_p
-        for fn in (L.attn_fwd, L.attn_decode, L.attn_decode_multi, L.attn_frame_block_map, L.attn_classify,
+        for fn in (L.attn_fwd, L.attn_decode, L.attn_decode_multi, L.attn_bwd, L.attn_frame_block_map,
+                   L.attn_classify,
                    L.attn_plan,
                    L.attn_sync_status, L.attn_last_error_detail, L.attn_shutdown, L.attn_debug_fault):
             fn.restype = I
@@ -163,6 +165,24 @@ def attn_decode_multi(q, k_cache, v_cache, seqlens, o=None, lse=None, scale=None
                                    o.data_ptr(), None if lse is None else lse.data_ptr(), B, Sq, Hq, Hkv,
                                    Lmax, d, float(scale), _stream_ptr(stream)))
     return o, lse
+
+
+def attn_bwd(q, k, v, o, lse, dout, scale=None, mask_kind=MASK_NONE, stream=None):
+    """Gradients of attn_fwd (bf16): q, o, dout [B,Nq,Hq,d]; k, v [B,Nkv,Hkv,d];
+    lse [B,Hq,Nq] fp32 from the forward.  Returns (dq, dk, dv) like q, k, v."""
+    import torch
+    for t in (q, k, v, o, dout):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v, o, dout must be contiguous bf16 CUDA tensors")
+    B, Nq, Hq, d = q.shape
+    Nkv, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    _check(lib().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nkv, d, float(scale),
+                          mask_kind, _stream_ptr(stream)))
+    return dq, dk, dv
 
 
 def frame_block_map(n_frames: int, frame_len: int) -> np.ndarray:

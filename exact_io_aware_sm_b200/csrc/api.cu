@@ -409,6 +409,61 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   return attn_decode_multi(q, k_cache, v_cache, seqlens, o, lse, B, 1, Hq, Hkv, Lmax, d, scale, stream);
 }
 
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nkv, int d, float scale,
+             int mask_kind, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv)
+    return set_err(ATTN_ERR_NULL, "every tensor of attn_bwd must be non-NULL");
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nkv < 1) return set_err(ATTN_ERR_SHAPE, "sizes must be >= 1");
+  if (Hq % Hkv != 0) return set_err(ATTN_ERR_SHAPE, "Hq (%d) is not a multiple of Hkv (%d)", Hq, Hkv);
+  if (d != 64 && d != 128) return set_err(ATTN_ERR_UNSUPPORTED, "attn_bwd needs d in {64, 128}");
+  if (mask_kind != ATTN_MASK_NONE && mask_kind != ATTN_MASK_CAUSAL)
+    return set_err(ATTN_ERR_UNSUPPORTED, "attn_bwd supports ATTN_MASK_NONE and ATTN_MASK_CAUSAL");
+  if (!(scale > 0.f) || !std::isfinite(scale)) return set_err(ATTN_ERR_SHAPE, "scale must be positive and finite");
+  if (B > 65535 || Hq > 65535 || static_cast<long long>(B) * Hq * Nq >= (1ll << 31))
+    return set_err(ATTN_ERR_SHAPE, "too many rows");
+  for (const void* p : {q, k, v, o, dout, static_cast<const void*>(lse), static_cast<const void*>(dq),
+                        static_cast<const void*>(dk), static_cast<const void*>(dv)})
+    if (!aligned16(p)) return set_err(ATTN_ERR_ALIGN, "device pointers must be 16-byte aligned");
+  if (int rc = check_device_sm100()) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevWs* ws;
+  if (int rc = get_ws(&ws)) return rc;
+  const size_t need = 2 * static_cast<size_t>(B) * Hq * Nq;  // D and LSE * log2(e)
+  if (ws->part_floats < need) {
+    cudaDeviceSynchronize();
+    cudaFree(ws->d_part);
+    ws->d_part = nullptr;
+    ws->part_floats = 0;
+    cudaError_t e = cudaMalloc(&ws->d_part, need * sizeof(float));
+    if (e != cudaSuccess) return set_err(ATTN_ERR_WORKSPACE, "backward scratch: %s", cudaGetErrorString(e));
+    ws->part_floats = need;
+  }
+  BwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.dout = dout;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dvec = ws->d_part;
+  a.lse2 = ws->d_part + need / 2;
+  a.err = ws->d_err;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nkv = Nkv;
+  a.causal = mask_kind == ATTN_MASK_CAUSAL;
+  a.scale = scale;
+  cudaError_t e = launch_bwd(d, a, s);
+  return e == cudaSuccess ? ATTN_OK : cuda_err(e, "backward launch");
+}
+
 int attn_frame_block_map(int n_frames, int frame_len, uint8_t* out) {
   if (!out) return set_err(ATTN_ERR_NULL, "out must be non-NULL");
   if (n_frames < 1 || frame_len < 1) return set_err(ATTN_ERR_SHAPE, "n_frames and frame_len must be >= 1");

@@ -29,6 +29,7 @@
 
 #include "kernels.h"
 #include "ptx_sm100.cuh"
+#include "warp_mma.cuh"
 
 namespace eio {
 namespace {
@@ -53,44 +54,6 @@ struct DCfg {
   static constexpr int kOffPre = kOffMeta + kWarps * R * 16;  // int[kMaxB + 1] prefix, int[kMaxB] lengths
   static constexpr int kSmem = kOffPre + (2 * kMaxB + 1) * 4 + 1024;  // + slack to align the base to 1 KB
 };
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
-// D (16x8 f32) += A (16x16 bf16, row) * B (16x8 bf16, col).
-__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ int checked_len(const DecodeArgs& a, int b) {
   const int len = a.seqlens[b];
@@ -302,7 +265,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
       v *= sl2;
       if (v > m[j] + kRebase) {  // move the base (always on the first stage)
-        const float alpha = ex2(m[j] - v);
+        const float alpha = wm_ex2(m[j] - v);
         l[j] *= alpha;
 #pragma unroll
         for (int mt = 0; mt < NK; ++mt) {
@@ -320,11 +283,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           // a column that has seen no key yet keeps m = -inf: its p are 0
-          p[i] = ex2(fmaf(s[ch][i], sl2, m[i & 1] == -INFINITY ? 0.f : -m[i & 1]));
+          p[i] = wm_ex2(fmaf(s[ch][i], sl2, m[i & 1] == -INFINITY ? 0.f : -m[i & 1]));
           l[i & 1] += p[i];
         }
-        const uint32_t b0 = movmatrix_trans(pack_bf16x2(p[0], p[1]));
-        const uint32_t b1 = movmatrix_trans(pack_bf16x2(p[2], p[3]));
+        const uint32_t b0 = movmatrix_trans(wm_pack_bf16x2(p[0], p[1]));
+        const uint32_t b1 = movmatrix_trans(wm_pack_bf16x2(p[2], p[3]));
         const int r = ch * 16 + (lane >> 4) * 8 + (lane & 7);
 #pragma unroll
         for (int mt = 0; mt < NK; ++mt) {
@@ -403,7 +366,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
   }
   float W = 0.f, O = 0.f;
   for (int s = 0; s < ns; ++s) {
-    const float w = ex2(lp[s] - M);
+    const float w = wm_ex2(lp[s] - M);
     W += w;
     O = fmaf(w, op[static_cast<size_t>(s) * D + t], O);
   }

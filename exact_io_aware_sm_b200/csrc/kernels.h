@@ -70,6 +70,25 @@ constexpr int kDecodeMaxCounters = 63;  // sequence groups one call may need (B 
 cudaError_t launch_decode(int d, int G, const DecodeArgs& a, cudaStream_t s);
 size_t decode_partial_floats(int B, int Hq, int Lmax, int d);
 
+// Backward (dQ, dK, dV) for an upstream dO; bf16 tensors, d in {64, 128}.
+struct BwdArgs {
+  const void* q;      // [B, Nq, Hq, d]
+  const void* k;      // [B, Nkv, Hkv, d]
+  const void* v;
+  const void* o;      // [B, Nq, Hq, d] forward output
+  const void* dout;   // [B, Nq, Hq, d]
+  const float* lse;   // [B, Hq, Nq] forward LSE (natural log)
+  void* dq;           // [B, Nq, Hq, d] (written)
+  void* dk;           // [B, Nkv, Hkv, d] (written)
+  void* dv;
+  float* dvec;        // scratch [B, Hq, Nq]: rowsum(dO * O)
+  float* lse2;        // scratch [B, Hq, Nq]: LSE * log2(e)
+  int* err;
+  int B, Hq, Hkv, Nq, Nkv, causal;
+  float scale;
+};
+cudaError_t launch_bwd(int d, const BwdArgs& a, cudaStream_t s);
+
 // TMA map of a [B, N, H, d] bf16 array as {d, H, N, B} with a {64, 1, box_rows, 1}
 // box and 128-byte swizzle; rows past N read as zeros.  False (with the error
 // detail set) if the driver refuses it.

@@ -240,6 +240,31 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                         int Lmax, int d, float scale, void* stream);
 
 /*
+ * attn_bwd -- gradients of attn_fwd (bf16) for an upstream gradient dO.
+ *
+ * Passage: "FlashAttention: memory-saving exact attention", section 4: the
+ * backward keeps only O and the row statistics of the forward and recomputes
+ * S and P from Q, K and those statistics, block by block, in on-chip memory.
+ * With P = exp(S - LSE), D_i = rowsum(dO_i * O_i):
+ *   dV = P^T dO,  dS = P * (dO V^T - D),  dQ = scale dS K,  dK = scale dS^T Q,
+ * dK and dV of a KV head summing over its Hq/Hkv query heads.
+ *
+ *   q, o, dout  device, [B, Nq, Hq, d] bf16 (o: the forward output)
+ *   k, v        device, [B, Nkv, Hkv, d] bf16
+ *   lse         device, [B, Hq, Nq] fp32, the forward LSE (natural log)
+ *   dq          device, [B, Nq, Hq, d] bf16 (written)
+ *   dk, dv      device, [B, Nkv, Hkv, d] bf16 (written)
+ *   mask_kind   ATTN_MASK_NONE or ATTN_MASK_CAUSAL (as attn_fwd)
+ * Limits: d == 64 or 128; all pointers 16-byte aligned.
+ * Scratch: 2*B*Hq*Nq floats of library workspace.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED (other masks or d), CUDA, WORKSPACE;
+ * a bounded wait that runs out latches ATTN_ERR_DEVICE_TIMEOUT.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nkv, int d, float scale,
+             int mask_kind, void* stream);
+
+/*
  * attn_debug_fault -- test hook for the device time-out path.
  *
  * kind 1: the next bf16 attn_fwd call on this thread makes CTA 0 skip its

@@ -193,6 +193,65 @@ def test_config4_frame_block_sparse_full_size():
     check_rows(o, lse, ro, rl, rows, "config4")
 
 
+# ------------------------------------------------------------------ backward
+# Gradients are bf16 outputs of products whose P and dS operands are rounded to
+# bf16 (relative 2^-9 each) and D = rowsum(dO * O) uses the bf16 O of the
+# forward; the bound is relative to each gradient's own scale.
+GRAD_MAX_REL, GRAD_MEAN_REL = 2e-2, 1e-2
+
+
+def check_grad(got, ref, where):
+    g = host_f64(got).reshape(ref.shape)
+    assert np.isfinite(g).all(), f"{where}: non-finite gradient"
+    err = np.abs(g - ref)
+    scale_max, scale_mean = np.abs(ref).max(), np.abs(ref).mean()
+    assert err.max() <= GRAD_MAX_REL * scale_max + 1e-6, f"{where}: max err {err.max():.3e} vs {scale_max:.3e}"
+    assert err.mean() <= GRAD_MEAN_REL * scale_mean + 1e-7, f"{where}: mean err {err.mean():.3e} vs {scale_mean:.3e}"
+
+
+BWD_CASES = [
+    # B, Hq, Hkv, Nq, Nkv, d, causal
+    (1, 2, 2, 128, 128, 64, False),
+    (2, 4, 2, 200, 200, 128, True),
+    (1, 4, 1, 77, 130, 64, True),
+    (1, 2, 1, 130, 77, 128, True),   # rows that see no key
+    (1, 3, 3, 300, 300, 128, False),
+    (2, 8, 2, 64, 64, 64, True),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES)
+def test_backward_small(case):
+    B, Hq, Hkv, Nq, Nkv, d, causal = case
+    seed = 3100 + BWD_CASES.index(case)
+    q, k, v = make_inputs(seed, B, Hq, Hkv, Nq, Nkv, d)
+    dout = synthetic.tensor(seed, 9, (B, Nq, Hq, d))
+    kind = eio.MASK_CAUSAL if causal else eio.MASK_NONE
+    scale = 1 / math.sqrt(d)
+    tq, tk, tv, tdo = dev_bf16(q), dev_bf16(k), dev_bf16(v), dev_bf16(dout)
+    o, lse = eio.attn_fwd(tq, tk, tv, scale=scale, mask_kind=kind)
+    dq, dk, dv = eio.attn_bwd(tq, tk, tv, o, lse, tdo, scale=scale, mask_kind=kind)
+    eio.sync_status()
+    rq, rk, rv = oracle.attn_bwd(q, k, v, dout, scale, kind)
+    check_grad(dq, rq, f"{case} dq")
+    check_grad(dk, rk, f"{case} dk")
+    check_grad(dv, rv, f"{case} dv")
+
+
+def test_backward_gpt2_shape_first_batch_element():
+    B, H, N, d = 8, 12, 1024, 64
+    q, k, v = make_inputs(1002, B, H, H, N, N, d)
+    dout = synthetic.tensor(1002, 9, (B, N, H, d))
+    tq, tk, tv, tdo = dev_bf16(q), dev_bf16(k), dev_bf16(v), dev_bf16(dout)
+    o, lse = eio.attn_fwd(tq, tk, tv, mask_kind=eio.MASK_CAUSAL)
+    dq, dk, dv = eio.attn_bwd(tq, tk, tv, o, lse, tdo, mask_kind=eio.MASK_CAUSAL)
+    eio.sync_status()
+    rq, rk, rv = oracle.attn_bwd(q[:1], k[:1], v[:1], dout[:1], 1 / math.sqrt(d), oracle.MASK_CAUSAL)
+    check_grad(dq[:1], rq, "gpt2 dq")
+    check_grad(dk[:1], rk, "gpt2 dk")
+    check_grad(dv[:1], rv, "gpt2 dv")
+
+
 # ------------------------------------------------------------------ decode
 def run_decode(q, kc, vc, lens, scale):
     o, lse = eio.attn_decode(dev_bf16(q), dev_bf16(kc), dev_bf16(vc),
