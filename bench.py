@@ -431,6 +431,48 @@ def bench_prefill(w, args, world, rank, peaks, with_e2e=True):
     return out
 
 
+def bench_backward(w, args, world, rank, peaks):
+    """attn_bwd on a prefill workload (bf16; O and LSE from attn_fwd, computed
+    once).  FLOPs: the five products of the backward over the allowed pairs,
+    2.5x the forward's (the usual convention; the recomputation of S and P in
+    both kernels is not counted)."""
+    import torch
+
+    import exact_io_aware_sm_b200 as eio
+    seed = rank_seed(w["seed"], rank)
+    q, k, v = host_prefill_inputs(w, seed)
+    dout = synthetic.tensor(seed, 9, q.shape, w["dtype"])
+    tq, tk, tv, tdo = (to_torch(x, "cuda") for x in (q, k, v, dout))
+    mk, _ = mask_of(w)
+    scale = 1.0 / math.sqrt(w["d"])
+    o, lse = eio.attn_fwd(tq, tk, tv, scale=scale, mask_kind=mk)
+    dq, dk, dv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
+
+    def step():
+        eio.lib().attn_bwd(tq.data_ptr(), tk.data_ptr(), tv.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           tdo.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), w["B"], w["Hq"], w["Hkv"],
+                           w["N"], w["N"], w["d"], scale, mk, torch.cuda.current_stream().cuda_stream)
+
+    flush = make_flush()
+    time_steps(step, 3, args.warmup, world, flush)
+    graph = capture_graph(step)
+    ms, _ = time_steps(graph.replay, max(5, args.steps // 2), args.warmup, world, flush)
+    eio.sync_status()
+    ms = max_over_ranks(ms, world)
+    flops = 2.5 * prefill_flops(w)
+    tflops = whole_job_rate(flops, ms, world) / 1e12
+    peak = peaks["bf16_tflops"]
+    out = {"metric": "attention backward TFLOP/s", "value": tflops, "unit": "TFLOP/s", "ms_per_step": ms,
+           "config": {"workload": w["desc"] + ", backward (dQ, dK, dV)"},
+           "roofline": {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                        "frac": flops / (ms * 1e-3) / 1e12 / peak, "peak_source": f"{peaks['source']} bf16 burst",
+                        "kernel": "bwd_prep + bwd_dq + bwd_dkdv (one call)"},
+           "gpu_launches": 3 * max(5, args.steps // 2)}
+    del tq, tk, tv, tdo, o, lse, dq, dk, dv
+    torch.cuda.empty_cache()
+    return out
+
+
 def args_key(w):
     return f"{w['mask']}_d{w['d']}_n{w['N']}"
 
@@ -669,6 +711,8 @@ def main():
         extra = {}
         if not args.no_extra:
             extra["decode"] = bench_decode(WORKLOADS["decode"], args, world, rank, peaks)
+            if w["mask"] in ("none", "causal"):
+                extra["backward"] = bench_backward(w, args, world, rank, peaks)
             for name in ("long", "frame"):
                 if name == args.workload:
                     continue

@@ -39,12 +39,13 @@ struct BCfg {
   static constexpr int KB = D / 64;                  // 128-byte column blocks per row
   static constexpr int kBlock = kBT * 128;           // one column block of a 64-row tile
   static constexpr int kTile = KB * kBlock;          // a 64 x D bf16 tile
-  static constexpr int R = D == 64 ? 3 : 2;          // ring stages (two tiles each)
+  static constexpr int kCtas = D == 64 ? 2 : 1;       // CTAs per SM (d = 128: registers for the accumulators)
+  static constexpr int R = D == 64 ? 3 : 4;          // ring stages (two tiles each)
   static constexpr int kOffRing = 2 * kTile;         // after the two resident tiles
   static constexpr int kOffVec = kOffRing + R * 2 * kTile;  // per stage: lse2[64], D[64]
   static constexpr int kOffBars = kOffVec + R * 2 * kBT * 4;
   static constexpr int kSmem = kOffBars + 8 * (2 * R + 1) + 16 + 1024;
-  static_assert(kSmem <= 113 * 1024, "two CTAs per SM");
+  static_assert(kSmem <= (kCtas == 2 ? 113 : 227) * 1024, "shared memory per CTA");
 };
 
 __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBThreads, 2)
+__global__ void __launch_bounds__(kBThreads, BCfg<D>::kCtas)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const BwdArgs a) {
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kBThreads, 2)
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBThreads, 2)
+__global__ void __launch_bounds__(kBThreads, BCfg<D>::kCtas)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const BwdArgs a) {
