@@ -420,7 +420,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   if (mask_kind != ATTN_MASK_NONE && mask_kind != ATTN_MASK_CAUSAL)
     return set_err(ATTN_ERR_UNSUPPORTED, "attn_bwd supports ATTN_MASK_NONE and ATTN_MASK_CAUSAL");
   if (!(scale > 0.f) || !std::isfinite(scale)) return set_err(ATTN_ERR_SHAPE, "scale must be positive and finite");
-  if (B > 65535 || Hq > 65535 || static_cast<long long>(B) * Hq * Nq >= (1ll << 31))
+  if (B > 65535 || Hq > 65535 || static_cast<long long>(B) * Hq * Nq >= (1ll << 31) ||
+      static_cast<long long>(B) * Hkv * Nkv >= (1ll << 31))
     return set_err(ATTN_ERR_SHAPE, "too many rows");
   for (const void* p : {q, k, v, o, dout, static_cast<const void*>(lse), static_cast<const void*>(dq),
                         static_cast<const void*>(dk), static_cast<const void*>(dv)})

@@ -217,6 +217,9 @@ BWD_CASES = [
     (1, 2, 1, 130, 77, 128, True),   # rows that see no key
     (1, 3, 3, 300, 300, 128, False),
     (2, 8, 2, 64, 64, 64, True),
+    (1, 4, 2, 400, 333, 64, True),    # several 128-row tiles, ragged, rows that see no key
+    (1, 8, 2, 520, 520, 128, True),   # GQA group of 4 over five Q and KV tiles
+    (2, 2, 2, 256, 384, 64, False),
 ]
 
 
