@@ -431,7 +431,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   std::lock_guard<std::mutex> lk(g_mu);
   DevWs* ws;
   if (int rc = get_ws(&ws)) return rc;
-  const size_t need = 2 * static_cast<size_t>(B) * Hq * Nq;  // D and LSE * log2(e)
+  // D and LSE * log2(e), rows padded to whole 128-row tiles
+  const size_t need = 2 * static_cast<size_t>(B) * Hq * ((static_cast<size_t>(Nq) + 127) / 128 * 128);
   if (ws->part_floats < need) {
     cudaDeviceSynchronize();
     cudaFree(ws->d_part);

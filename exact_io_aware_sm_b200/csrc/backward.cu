@@ -8,32 +8,45 @@
 //   P = exp(S - LSE),  dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
 //   dQ = scale dS K,   dK = scale dS^T Q
 //
-// Three kernels:
-//   bwd_prep_kernel   D and LSE * log2(e) per (b, head, row), into scratch.
-//   bwd_dkdv_kernel   one CTA per (128-key tile, KV head, b): K and V stay in
-//                     shared memory while the Q / dO tiles of every query
-//                     head of the group stream through a TMA ring, so dK and
-//                     dV of a KV head sum over its G query heads without
-//                     atomics.  Per Q tile, on the tensor core:
-//                       S^T  = K Q^T,   dP^T = V dO^T       (shared x shared)
-//                       dV  += P^T dO,  dK  += dS^T Q       (TMEM x shared)
-//   bwd_dq_kernel     one CTA per (128-row Q tile, query head, b): Q and dO
-//                     stay while the K / V tiles stream through; per K/V tile
-//                       S = Q K^T,  dP = dO V^T,  dQ += dS K.
-// S and dP are recomputed by both stream kernels (seven products instead of
-// five) so that neither needs atomics or a second pass over an fp32 dQ.
+// Two kernels, launched in this order:
+//   bwd_dq_kernel     one CTA per (128-row Q tile, query head, b): Q, dO and
+//                     O stay in shared memory while the K / V tiles stream
+//                     through a TMA ring; per K/V tile, on the tensor core,
+//                       S = Q K^T,  dP = dO V^T       (shared x shared)
+//                       dQ += dS K                    (TMEM x shared)
+//                     Its element-wise threads compute D from the O and dO
+//                     tiles (while dP of the first tile is on the tensor
+//                     core) and leave D and LSE*log2(e) in a scratch whose
+//                     rows are padded to whole tiles (lse2 = +inf, D = 0).
+//                     The dK/dV kernel fetches 128-row runs of both with bulk
+//                     copies on the same barrier as its Q / dO tiles.
+//   bwd_dkdv_kernel   one CTA per (128-key tile, KV head, b): K and V stay
+//                     while the Q / dO tiles of every query head of the group
+//                     stream through, so dK and dV of a KV head sum over its
+//                     G query heads without atomics; per Q tile
+//                       S^T = K Q^T,  dP^T = V dO^T
+//                       dV += P^T dO,  dK += dS^T Q
+// S and dP are recomputed by both kernels (seven products instead of five)
+// so that neither needs atomics or a second pass over an fp32 dQ.
 //
-// Roles (192 threads): warp 0 issues the TMA copies, warp 1 owns TMEM and
-// issues the tcgen05 MMAs from an elect.sync-chosen lane, warps 2..5 are the
-// element-wise warps (thread <-> TMEM lane <-> key row in the dK/dV kernel,
-// query row in the dQ kernel).  An element-wise thread loads its S row from
-// TMEM, writes P (bf16 pairs) over the first 64 columns of that row, then
-// turns each 32-column chunk of its dP row into dS and writes it (bf16
-// pairs) over the front of the dP row: the TMEM-operand MMAs read P and dS
-// from there.
+// Roles (320 threads): warp 0 issues the TMA copies, warp 1 owns TMEM and
+// issues the tcgen05 MMAs from an elect.sync-chosen lane, warps 2..9 are two
+// element-wise warpgroups: warpgroup h takes columns [64h, 64h+64) of every
+// S and dP row (thread <-> TMEM lane <-> key row in the dK/dV kernel, query
+// row in the dQ kernel).  A thread loads its 64 S values, writes P (bf16
+// pairs, 32 columns) over the front of that same column range, then turns
+// its dP values into dS and writes them (32 columns) behind P: dK/dV reads P
+// from columns [64h, 64h+32) and dS from [64h+32, 64h+64); the dQ kernel
+// keeps only dS, at [64h, 64h+32).  No warpgroup writes a column that the
+// other still has to read, and dP is never written, so dP(t+1) may start as
+// soon as both warpgroups have read dP(t).
 //
-// TMEM columns: S [0,128), dP [128,256), accumulators from 256 (dV then dK,
-// or dQ), d columns each.
+// S is double-buffered in TMEM where the columns allow (dQ kernel; dK/dV
+// kernel at d = 64): S(t+1) then runs on the tensor core while the
+// element-wise warps still work on tile t.
+//   dQ:         S0 [0,128) S1 [128,256) dP [256,384) dQ [384, 384+d)
+//   dK/dV d=64: S0 [0,128) S1 [128,256) dP [256,384) dV [384,448) dK [448,512)
+//   dK/dV d=128: S [0,128) dP [128,256) dV [256,384) dK [384,512)
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -44,7 +57,8 @@ namespace eio {
 namespace {
 
 constexpr int kT = 128;  // rows of a Q tile, keys of a KV tile: the MMA's M
-constexpr int kBThreads = 192;
+constexpr int kBThreads = 320;
+constexpr int kEW = 8;   // element-wise warps
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -54,45 +68,26 @@ struct BCfg {
   static constexpr int kTile = NCH * kChunk;         // a 128 x D bf16 tile
   static constexpr int R = D == 64 ? 4 : 2;          // ring stages (two tiles each)
   static constexpr int kOffRing = 2 * kTile;         // after the two resident tiles
-  static constexpr int kOffVec = kOffRing + R * 2 * kTile;  // per stage: lse2[128], D[128]
-  static constexpr int kOffBar = kOffVec + R * 2 * kT * 4;
-  // fixed_full, full[R], empty[R], s_full, dp_full, p_full, ds_full, mma_done, mma_idle
-  static constexpr int kNumBars = 1 + 2 * R + 6;
-  static constexpr int kSmem = kOffBar + 8 * kNumBars + 16 + 1024;
-  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+  // dK/dV kernel: per stage lse2[128], D[128]; dQ kernel: the O tile
+  static constexpr int kOffX = kOffRing + R * 2 * kTile;
+  static constexpr int kOffBarKV = kOffX + R * 2 * kT * 4;
+  static constexpr int kOffBarQ = kOffX + kTile;
+  // fixed_full, full[R], empty[R], s_full[2], dp_full, p_full, ds_full, mma_done, mma_idle
+  static constexpr int kNumBars = 1 + 2 * R + 7;
+  static constexpr int kSmemKV = kOffBarKV + 8 * kNumBars + 16 + 1024;
+  static constexpr int kSmemQ = kOffBarQ + 8 * kNumBars + 16 + 1024;
+  static_assert(kSmemKV <= 227 * 1024 && kSmemQ <= 227 * 1024, "shared memory per CTA");
+  static constexpr int kVecBytes = 2 * kT * 4;
+  // S buffers in TMEM (dK/dV kernel; the dQ kernel always has two)
+  static constexpr int kSBufKV = D == 64 ? 2 : 1;
 };
 
 __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// D and lse2 for every (b, head, row), one warp per row.
-template <int D>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const long long rows = static_cast<long long>(a.B) * a.Hq * a.Nq;
-  if (row >= rows) return;
-  const int i = static_cast<int>(row % a.Nq);
-  const int hq = static_cast<int>((row / a.Nq) % a.Hq);
-  const int b = static_cast<int>(row / (static_cast<long long>(a.Nq) * a.Hq));
-  const size_t off = ((static_cast<size_t>(b) * a.Nq + i) * a.Hq + hq) * D;
-  constexpr int E = D / 32;  // elements per lane
-  const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(a.o) + off + lane * E;
-  const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(a.dout) + off + lane * E;
-  float acc = 0.f;
-#pragma unroll
-  for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(o[e]), __bfloat162float(g[e]), acc);
-#pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) {
-    a.dvec[row] = acc;
-    a.lse2[row] = a.lse[row] * kLog2e;
-  }
-}
-
-// acc (+)= A B^T over d for two 128-row K-major tiles in shared memory
-// (A the M side, B the N side; both 128-byte swizzled, 64-column chunks).
+// acc = A B^T over d for two 128-row K-major tiles in shared memory (A the M
+// side, B the N side; both 128-byte swizzled, 64-column chunks).
 template <int D>
 __device__ __forceinline__ void issue_ss(uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
   constexpr uint32_t id = idesc_bf16_f32(128, 128, 0, 0);
@@ -105,23 +100,25 @@ __device__ __forceinline__ void issue_ss(uint32_t d_tmem, uint32_t a_base, uint3
 }
 
 // acc (+)= A B over 128 rows: A (128 x 128 bf16) from TMEM, B the 128 x D
-// tile in shared memory read with its rows as the reduction (MN-major).
+// tile in shared memory read with its rows as the reduction (MN-major).  A's
+// 64 packed columns sit in two runs of 32: [a, a+32) for reduction rows
+// 0..63 and [a+64, a+96) for rows 64..127.
 template <int D>
 __device__ __forceinline__ void issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool accumulate) {
   constexpr uint32_t id = idesc_bf16_f32(128, D, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < kT / 16; ++kk)
-    mma_bf16_ts_elect(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_base + kk * 2048, BCfg<D>::kChunk, 1024), id,
-                      (accumulate || kk > 0) ? 1u : 0u);
+    mma_bf16_ts_elect(d_tmem, a_tmem + kk * 8 + (kk >= 4 ? 32 : 0),
+                      sdesc_sw128(b_base + kk * 2048, BCfg<D>::kChunk, 1024), id, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// One thread's TMEM row of D fp32 values (times mul) to a bf16 row in HBM;
-// dst == nullptr skips the store, have == false stores zeros.  Warp-uniform
-// `have`: the TMEM loads are warp-collective.
-template <int D>
-__device__ __forceinline__ void store_row(uint32_t t, __nv_bfloat16* dst, float mul, bool have) {
+// NC columns of one thread's TMEM row (times mul) to bf16 in HBM; dst ==
+// nullptr skips the store, have == false stores zeros.  `have` is
+// warp-uniform: the TMEM loads are warp-collective.
+template <int NC>
+__device__ __forceinline__ void store_cols(uint32_t t, __nv_bfloat16* dst, float mul, bool have) {
 #pragma unroll
-  for (int c = 0; c < D; c += 32) {
+  for (int c = 0; c < NC; c += 32) {
     uint32_t r[32];
     if (have) {
       tmem_ld32(t + c, r);
@@ -142,26 +139,22 @@ __device__ __forceinline__ void store_row(uint32_t t, __nv_bfloat16* dst, float 
   }
 }
 
-// dS = P * (dP - D) for one thread's row, 32 columns at a time: dP is read
-// from TMEM at t_dp and dS written back (bf16 pairs) over the front of the
-// same row, behind the columns still to be read.  dvals(c) gives D for
-// column c.
+// dS = P * (dP - D) for one thread's 64 columns: dP read from TMEM at t_dp,
+// dS written (bf16 pairs, 32 columns) at t_ds.  dvals(c) gives D for the
+// columns c, c + 1.
 template <typename DFn>
-__device__ __forceinline__ void write_ds(uint32_t t_dp, const float* p, DFn dvals) {
+__device__ __forceinline__ void write_ds(uint32_t t_dp, uint32_t t_ds, const float* p, DFn dvals) {
+  uint32_t dr[64], pk[32];
+  tmem_ld32(t_dp, dr);
+  tmem_ld32(t_dp + 32, dr + 32);
+  tmem_wait_ld();
 #pragma unroll
-  for (int c4 = 0; c4 < 4; ++c4) {
-    uint32_t dr[32], pk[16];
-    tmem_ld32(t_dp + 32 * c4, dr);
-    tmem_wait_ld();
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int c = 32 * c4 + 2 * j;
-      const float2 dd = dvals(c);
-      pk[j] = wm_pack_bf16x2(p[c] * (__uint_as_float(dr[2 * j]) - dd.x),
-                             p[c + 1] * (__uint_as_float(dr[2 * j + 1]) - dd.y));
-    }
-    tmem_st16(t_dp + 16 * c4, pk);
+  for (int j = 0; j < 32; ++j) {
+    const float2 dd = dvals(2 * j);
+    pk[j] = wm_pack_bf16x2(p[2 * j] * (__uint_as_float(dr[2 * j]) - dd.x),
+                           p[2 * j + 1] * (__uint_as_float(dr[2 * j + 1]) - dd.y));
   }
+  tmem_st32(t_ds, pk);
 }
 
 // ----------------------------------------------------------------- dK, dV
@@ -171,22 +164,23 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const BwdArgs a) {
   using C = BCfg<D>;
-  constexpr int R = C::R;
+  constexpr int R = C::R, NB = C::kSBufKV;
+  constexpr uint32_t kColDP = 128 * NB, kColDV = kColDP + 128, kColDK = kColDV + D;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBarKV);
   uint64_t* fixed_full = bars;
   uint64_t* full = bars + 1;
   uint64_t* empty = full + R;
-  uint64_t* s_full = empty + R;
-  uint64_t* dp_full = s_full + 1;
+  uint64_t* s_full = empty + R;  // [2]
+  uint64_t* dp_full = s_full + 2;
   uint64_t* p_full = dp_full + 1;
   uint64_t* ds_full = p_full + 1;
   uint64_t* mma_done = ds_full + 1;
   uint64_t* mma_idle = mma_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* vec = reinterpret_cast<float*>(smem + C::kOffVec);  // [R][2][128]: lse2, D
+  float* vec = reinterpret_cast<float*>(smem + C::kOffX);  // [R][2][128]: lse2, D
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Linear grid, KV tile slowest: under a causal mask the first tiles have
@@ -198,6 +192,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const int k0 = kt * kT;
   const int off = a.Nkv - a.Nq;  // bottom-right causal alignment
   const int n_qt = (a.Nq + kT - 1) / kT;
+  const int nq_pad = n_qt * kT;  // rows per (b, head) of the lse2 / D scratch
   // causal: row i sees key k0 iff i >= k0 - off; earlier Q tiles see none of these keys
   const int first_qt = a.causal ? min(n_qt, max(0, k0 - off) / kT) : 0;
   const int per_head = n_qt - first_qt;
@@ -207,12 +202,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(fixed_full, 1);
     for (int s = 0; s < R; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // the MMA commit, and each element-wise warp after reading the vectors
+      mbar_init(&empty[s], 1 + kEW);  // the MMA commit, and each element-wise warp after reading the vectors
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(ds_full, 4);
+    mbar_init(p_full, kEW);
+    mbar_init(ds_full, kEW);
     mbar_init(mma_done, 1);
     mbar_init(mma_idle, 1);
     *abort_flag = 0;
@@ -257,24 +253,17 @@ __global__ void __launch_bounds__(kBThreads, 1)
         break;
       }
       const int hq = hkv * G + u / per_head, qt = first_qt + u % per_head;
-      // This stage's 128 lse2 and D values; rows past Nq get lse2 = +inf,
-      // which makes their P exactly 0.
-      const size_t vrow = (static_cast<size_t>(b) * a.Hq + hq) * a.Nq;
-      float* vs = vec + s * 2 * kT;
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const int i = qt * kT + lane + 32 * h;
-        vs[lane + 32 * h] = i < a.Nq ? a.lse2[vrow + i] : INFINITY;
-        vs[kT + lane + 32 * h] = i < a.Nq ? a.dvec[vrow + i] : 0.f;
-      }
-      __syncwarp();
       uint8_t* st = smem + C::kOffRing + s * 2 * C::kTile;
-      mbar_arrive_expect_tx_elect(&full[s], 2 * C::kTile);
+      mbar_arrive_expect_tx_elect(&full[s], 2 * C::kTile + C::kVecBytes);
 #pragma unroll
       for (int ch = 0; ch < C::NCH; ++ch) {
         tma_load_4d_elect(st + ch * C::kChunk, &tmQ, &full[s], 64 * ch, hq, qt * kT, b);
         tma_load_4d_elect(st + C::kTile + ch * C::kChunk, &tmDO, &full[s], 64 * ch, hq, qt * kT, b);
       }
+      // the tile's 128 lse2 and D values (padded rows: lse2 = +inf, D = 0)
+      const size_t vrow = (static_cast<size_t>(b) * a.Hq + hq) * nq_pad + static_cast<size_t>(qt) * kT;
+      bulk_load_elect(vec + s * 2 * kT, a.lse2 + vrow, kT * 4, &full[s]);
+      bulk_load_elect(vec + s * 2 * kT + kT, a.dvec + vrow, kT * 4, &full[s]);
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
     // Every copy lands before the CTA retires.
@@ -282,36 +271,60 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (int w = u > R ? u - R : 0; w < u; ++w) mbar_wait(&full[w % R], (w / R) & 1);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order per step t: S(t+1) (two S buffers), dV(t), dK(t), then
+    // dP(t+1) -- the element-wise warps have read dP(t) by then.
     const uint32_t sK = smem_u32(smem), sV = sK + C::kTile;
-    bool ok = wwait(fixed_full, 0);
-    for (int u = 0; ok && u < steps; ++u) {
-      const int s = u % R;
-      const uint32_t sQ = smem_u32(smem + C::kOffRing + s * 2 * C::kTile), sdO = sQ + C::kTile;
-      // S and dP are rewritten once the previous step's dV / dK MMAs have
-      // read P and dS out of their columns.
-      if (!wwait(&full[s], (u / R) & 1) || (u > 0 && !wwait(mma_done, (u - 1) & 1))) {
-        ok = false;
-        break;
-      }
+    auto stage = [&](int t) { return smem_u32(smem + C::kOffRing + (t % R) * 2 * C::kTile); };
+    bool ok = wwait(fixed_full, 0) && (steps == 0 || wwait(&full[0], 0));
+    if (ok && steps > 0) {
       tc_fence_after();
-      issue_ss<D>(tmem, sK, sQ);  // S^T = K Q^T
-      mma_commit_elect(s_full);
-      issue_ss<D>(tmem + 128, sV, sdO);  // dP^T = V dO^T
+      issue_ss<D>(tmem, sK, stage(0));  // S^T = K Q^T
+      mma_commit_elect(&s_full[0]);
+      issue_ss<D>(tmem + kColDP, sV, stage(0) + C::kTile);  // dP^T = V dO^T
       mma_commit_elect(dp_full);
+    }
+    for (int u = 0; ok && u < steps; ++u) {
+      const int s = u % R, x = u % NB;
+      const uint32_t sQ = stage(u), sdO = sQ + C::kTile;
+      const bool next = u + 1 < steps;
+      if (NB == 2 && next) {
+        // S buffer (u+1)%2 was last read by dV(u-1) / dK(u-1)
+        if (!wwait(&full[(u + 1) % R], ((u + 1) / R) & 1) || (u >= 1 && !wwait(mma_done, (u - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_ss<D>(tmem + 128 * ((u + 1) % NB), sK, stage(u + 1));
+        mma_commit_elect(&s_full[(u + 1) % NB]);
+      }
       if (!wwait(p_full, u & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      issue_ts<D>(tmem + 256, tmem, sdO, u > 0);  // dV += P^T dO
+      issue_ts<D>(tmem + kColDV, tmem + 128 * x, sdO, u > 0);  // dV += P^T dO
       if (!wwait(ds_full, u & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      issue_ts<D>(tmem + 256 + D, tmem + 128, sQ, u > 0);  // dK += dS^T Q
+      issue_ts<D>(tmem + kColDK, tmem + 128 * x + 32, sQ, u > 0);  // dK += dS^T Q
       mma_commit_elect(&empty[s]);
       mma_commit_elect(mma_done);
+      if (next) {
+        if (NB == 1) {
+          // one S buffer: S(u+1) after dV(u) / dK(u) have read it
+          if (!wwait(&full[(u + 1) % R], ((u + 1) / R) & 1) || !wwait(mma_done, u & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_ss<D>(tmem, sK, stage(u + 1));
+          mma_commit_elect(&s_full[0]);
+        }
+        issue_ss<D>(tmem + kColDP, sV, stage(u + 1) + C::kTile);
+        mma_commit_elect(dp_full);
+      }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
     // Every MMA issued above has finished before TMEM is released.
@@ -319,32 +332,34 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_wait(mma_idle, 0);
   } else {
     // ------------------------------------------------------------ element-wise
+    const int h = (warp - 2) >> 2;  // column half
     const int quarter = warp & 3;
     const int key = k0 + quarter * 32 + lane;  // this thread's key (TMEM lane)
     const uint32_t lo = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t t_s = tmem + lo, t_dp = t_s + 128, t_dv = t_s + 256, t_dk = t_s + 256 + D;
+    const uint32_t t_row = tmem + lo;
     const float sl2 = a.scale * kLog2e;
     bool ok = true;
     for (int u = 0; u < steps; ++u) {
-      const int s = u % R;
-      const int q0 = (first_qt + u % per_head) * kT;
-      if (!wwait(&full[s], (u / R) & 1) || !wwait(s_full, u & 1)) {
+      const int s = u % R, x = u % NB;
+      const int q0 = (first_qt + u % per_head) * kT + 64 * h;  // query of this thread's first column
+      if (!wwait(&full[s], (u / R) & 1) || !wwait(&s_full[x], (u / NB) & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* vs = vec + s * 2 * kT;
-      float p[kT];
+      const float* vs = vec + s * 2 * kT + 64 * h;
+      const uint32_t t_s = t_row + 128 * x + 64 * h;
+      float p[64];
       {
-        uint32_t sr[kT];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, sr + 32 * c);
+        uint32_t sr[64];
+        tmem_ld32(t_s, sr);
+        tmem_ld32(t_s + 32, sr + 32);
         tmem_wait_ld();
         // causal: query q0 + c sees this key iff c >= key - off - q0
         const bool masked_tile = a.causal && k0 + kT - 1 > q0 + off;
         const int lim = masked_tile ? key - off - q0 : -1;
 #pragma unroll
-        for (int c = 0; c < kT; c += 4) {
+        for (int c = 0; c < 64; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(vs + c);
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
@@ -355,11 +370,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
       {
         uint32_t pk[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) pk[j] = wm_pack_bf16x2(p[64 * h + 2 * j], p[64 * h + 2 * j + 1]);
-          tmem_st32(t_s + 32 * h, pk);
-        }
+        for (int j = 0; j < 32; ++j) pk[j] = wm_pack_bf16x2(p[2 * j], p[2 * j + 1]);
+        tmem_st32(t_s, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -370,7 +382,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         break;
       }
       tc_fence_after();
-      write_ds(t_dp, p, [&](int c) { return *reinterpret_cast<const float2*>(vs + kT + c); });
+      write_ds(t_row + kColDP + 64 * h, t_s + 32, p,
+               [&](int c) { return *reinterpret_cast<const float2*>(vs + kT + c); });
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -384,10 +397,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tc_fence_after();
     }
     if (ok) {
-      const size_t o = ((static_cast<size_t>(b) * a.Nkv + key) * a.Hkv + hkv) * D;
+      // each warpgroup stores half of the columns of dV and dK
+      constexpr int HC = D / 2;
+      const size_t o = ((static_cast<size_t>(b) * a.Nkv + key) * a.Hkv + hkv) * D + HC * h;
       const bool valid = key < a.Nkv;
-      store_row<D>(t_dv, valid ? reinterpret_cast<__nv_bfloat16*>(a.dv) + o : nullptr, 1.f, steps > 0);
-      store_row<D>(t_dk, valid ? reinterpret_cast<__nv_bfloat16*>(a.dk) + o : nullptr, a.scale, steps > 0);
+      store_cols<HC>(t_row + kColDV + HC * h, valid ? reinterpret_cast<__nv_bfloat16*>(a.dv) + o : nullptr, 1.f,
+                     steps > 0);
+      store_cols<HC>(t_row + kColDK + HC * h, valid ? reinterpret_cast<__nv_bfloat16*>(a.dk) + o : nullptr,
+                     a.scale, steps > 0);
     } else if (lane == 0) {
       fail(kErrDeviceTimeout);
     }
@@ -404,17 +421,18 @@ template <int D>
 __global__ void __launch_bounds__(kBThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  const BwdArgs a) {
+                  const __grid_constant__ CUtensorMap tmO, const BwdArgs a) {
   using C = BCfg<D>;
   constexpr int R = C::R;
+  constexpr uint32_t kColDP = 256, kColDQ = 384;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBarQ);
   uint64_t* fixed_full = bars;
   uint64_t* full = bars + 1;
   uint64_t* empty = full + R;
-  uint64_t* s_full = empty + R;
-  uint64_t* dp_full = s_full + 1;
+  uint64_t* s_full = empty + R;  // [2]
+  uint64_t* dp_full = s_full + 2;
   uint64_t* ds_full = dp_full + 2;  // p_full is unused here
   uint64_t* mma_done = ds_full + 1;
   uint64_t* mma_idle = mma_done + 1;
@@ -443,9 +461,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(dp_full, 1);
-    mbar_init(ds_full, 4);
+    mbar_init(ds_full, kEW);
     mbar_init(mma_done, 1);
     mbar_init(mma_idle, 1);
     *abort_flag = 0;
@@ -475,11 +494,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
-    mbar_arrive_expect_tx_elect(fixed_full, 2 * C::kTile);
+    mbar_arrive_expect_tx_elect(fixed_full, 3 * C::kTile);
 #pragma unroll
     for (int ch = 0; ch < C::NCH; ++ch) {
       tma_load_4d_elect(smem + ch * C::kChunk, &tmQ, fixed_full, 64 * ch, hq, q0, b);
       tma_load_4d_elect(smem + C::kTile + ch * C::kChunk, &tmDO, fixed_full, 64 * ch, hq, q0, b);
+      tma_load_4d_elect(smem + C::kOffX + ch * C::kChunk, &tmO, fixed_full, 64 * ch, hq, q0, b);
     }
     bool ok = true;
     int j = 0;
@@ -502,84 +522,136 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (int w = j > R ? j - R : 0; w < j; ++w) mbar_wait(&full[w % R], (w / R) & 1);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order per step t: S(t+1) into the other S buffer, dQ(t), then
+    // dP(t+1) -- the element-wise warps have read dP(t) by then.
     const uint32_t sQ = smem_u32(smem), sdO = sQ + C::kTile;
-    bool ok = wwait(fixed_full, 0);
-    for (int j = 0; ok && j < n_kv; ++j) {
-      const int s = j % R;
-      const uint32_t sK = smem_u32(smem + C::kOffRing + s * 2 * C::kTile), sV = sK + C::kTile;
-      // S is rewritten once the previous dQ MMA has read dS out of its columns.
-      if (!wwait(&full[s], (j / R) & 1) || (j > 0 && !wwait(mma_done, (j - 1) & 1))) {
-        ok = false;
-        break;
-      }
+    auto stage = [&](int t) { return smem_u32(smem + C::kOffRing + (t % R) * 2 * C::kTile); };
+    bool ok = wwait(fixed_full, 0) && (n_kv == 0 || wwait(&full[0], 0));
+    if (ok && n_kv > 0) {
       tc_fence_after();
-      issue_ss<D>(tmem, sQ, sK);  // S = Q K^T
-      mma_commit_elect(s_full);
-      issue_ss<D>(tmem + 128, sdO, sV);  // dP = dO V^T
+      issue_ss<D>(tmem, sQ, stage(0));  // S = Q K^T
+      mma_commit_elect(&s_full[0]);
+      issue_ss<D>(tmem + kColDP, sdO, stage(0) + C::kTile);  // dP = dO V^T
       mma_commit_elect(dp_full);
+    }
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int s = j % R, x = j & 1;
+      const bool next = j + 1 < n_kv;
+      if (next) {
+        // S buffer (j+1)%2 was last read by dQ(j-1)
+        if (!wwait(&full[(j + 1) % R], ((j + 1) / R) & 1) || (j >= 1 && !wwait(mma_done, (j - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_ss<D>(tmem + 128 * (x ^ 1), sQ, stage(j + 1));
+        mma_commit_elect(&s_full[x ^ 1]);
+      }
       if (!wwait(ds_full, j & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      issue_ts<D>(tmem + 256, tmem + 128, sK, j > 0);  // dQ += dS K
+      issue_ts<D>(tmem + kColDQ, tmem + 128 * x, stage(j), j > 0);  // dQ += dS K
       mma_commit_elect(&empty[s]);
       mma_commit_elect(mma_done);
+      if (next) {
+        issue_ss<D>(tmem + kColDP, sdO, stage(j + 1) + C::kTile);
+        mma_commit_elect(dp_full);
+      }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
     mma_commit_elect(mma_idle);
     mbar_wait(mma_idle, 0);
   } else {
     // ------------------------------------------------------------ element-wise
+    const int h = (warp - 2) >> 2;  // column half
     const int quarter = warp & 3;
     const int row = q0 + quarter * 32 + lane;  // this thread's query row (TMEM lane)
     const uint32_t lo = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t t_s = tmem + lo, t_dp = t_s + 128, t_dq = t_s + 256;
+    const uint32_t t_row = tmem + lo;
     const float sl2 = a.scale * kLog2e;
-    const size_t vrow = (static_cast<size_t>(b) * a.Hq + hq) * a.Nq;
     // rows past Nq: lse2 = +inf makes their P exactly 0
-    const float l2 = row < a.Nq ? a.lse2[vrow + row] : INFINITY;
-    const float dd = row < a.Nq ? a.dvec[vrow + row] : 0.f;
+    const float l2 = row < a.Nq ? a.lse[(static_cast<size_t>(b) * a.Hq + hq) * a.Nq + row] * kLog2e : INFINITY;
+    // D = rowsum(dO * O) from the resident O and dO tiles (zero rows past
+    // Nq); with lse2 it goes to the padded scratch for the dK/dV kernel.
+    float dd = 0.f;
+    auto compute_d = [&]() -> bool {
+      if (!wwait(fixed_full, 0)) return false;
+      const int r = quarter * 32 + lane;
+#pragma unroll
+      for (int ch = 0; ch < C::NCH; ++ch)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int o = ch * C::kChunk + r * 128 + ((u ^ (r & 7)) << 4);
+          const uint4 ov = *reinterpret_cast<const uint4*>(smem + C::kOffX + o);
+          const uint4 gv = *reinterpret_cast<const uint4*>(smem + C::kTile + o);
+          const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float2 of = __bfloat1622float2(o2[w]), gf = __bfloat1622float2(g2[w]);
+            dd = fmaf(of.x, gf.x, dd);
+            dd = fmaf(of.y, gf.y, dd);
+          }
+        }
+      if (h == 0) {
+        const size_t vrow = (static_cast<size_t>(b) * a.Hq + hq) * (n_qt * kT) + row;
+        a.dvec[vrow] = dd;
+        a.lse2[vrow] = l2;
+      }
+      return true;
+    };
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      if (!wwait(s_full, j & 1)) {
+      const int x = j & 1;
+      if (!wwait(&s_full[x], (j >> 1) & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
       // keys at or past column lim are masked: past Nkv, and past the
       // causal diagonal (rows with no visible key get lim <= 0)
-      int lim = min(kT, a.Nkv - j * kT);
-      if (a.causal) lim = min(lim, row + off + 1 - j * kT);
-      float p[kT];
+      const int c0 = j * kT + 64 * h;  // key of this thread's first column
+      int lim = min(64, a.Nkv - c0);
+      if (a.causal) lim = min(lim, row + off + 1 - c0);
+      const uint32_t t_s = t_row + 128 * x + 64 * h;
+      float p[64];
       {
-        uint32_t sr[kT];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, sr + 32 * c);
+        uint32_t sr[64];
+        tmem_ld32(t_s, sr);
+        tmem_ld32(t_s + 32, sr + 32);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kT; ++c) p[c] = c < lim ? wm_ex2(fmaf(__uint_as_float(sr[c]), sl2, -l2)) : 0.f;
+        for (int c = 0; c < 64; ++c) p[c] = c < lim ? wm_ex2(fmaf(__uint_as_float(sr[c]), sl2, -l2)) : 0.f;
+      }
+      // D while dP(0) is on the tensor core
+      if (j == 0 && !compute_d()) {
+        ok = false;
+        break;
       }
       if (!wwait(dp_full, j & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      write_ds(t_dp, p, [&](int) { return make_float2(dd, dd); });
+      write_ds(t_row + kColDP + 64 * h, t_s, p, [&](int) { return make_float2(dd, dd); });
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
     }
+    if (ok && n_kv == 0) ok = compute_d();
     if (ok && n_kv > 0) {
       ok = wwait(mma_done, (n_kv - 1) & 1);
       tc_fence_after();
     }
     if (ok) {
+      constexpr int HC = D / 2;
       __nv_bfloat16* dst = row < a.Nq ? reinterpret_cast<__nv_bfloat16*>(a.dq) +
-                                            ((static_cast<size_t>(b) * a.Nq + row) * a.Hq + hq) * D
+                                            ((static_cast<size_t>(b) * a.Nq + row) * a.Hq + hq) * D + HC * h
                                       : nullptr;
-      store_row<D>(t_dq, dst, a.scale, n_kv > 0);
+      store_cols<HC>(t_row + kColDQ + HC * h, dst, a.scale, n_kv > 0);
     } else if (lane == 0) {
       fail(kErrDeviceTimeout);
     }
@@ -598,25 +670,23 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemQ);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+      e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemKV);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  CUtensorMap tq, tdo, tk, tv;
+  CUtensorMap tq, tdo, tk, tv, to;
   if (!encode_bf16_map(&tq, a.q, a.B, a.Nq, a.Hq, D, kT) || !encode_bf16_map(&tdo, a.dout, a.B, a.Nq, a.Hq, D, kT) ||
-      !encode_bf16_map(&tk, a.k, a.B, a.Nkv, a.Hkv, D, kT) || !encode_bf16_map(&tv, a.v, a.B, a.Nkv, a.Hkv, D, kT))
+      !encode_bf16_map(&tk, a.k, a.B, a.Nkv, a.Hkv, D, kT) || !encode_bf16_map(&tv, a.v, a.B, a.Nkv, a.Hkv, D, kT) ||
+      !encode_bf16_map(&to, a.o, a.B, a.Nq, a.Hq, D, kT))
     return cudaErrorInvalidValue;
-  const long long rows = static_cast<long long>(a.B) * a.Hq * a.Nq;
-  bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(a);
+  const long long n_qt = (a.Nq + kT - 1) / kT, n_kt = (a.Nkv + kT - 1) / kT;
+  // The dQ kernel also writes D and lse2, which the dK/dV kernel reads.
+  bwd_dq_kernel<D><<<static_cast<unsigned>(n_qt * a.Hq * a.B), kBThreads, C::kSmemQ, s>>>(tq, tdo, tk, tv, to, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long n_qt = (a.Nq + kT - 1) / kT, n_kt = (a.Nkv + kT - 1) / kT;
-  bwd_dq_kernel<D><<<static_cast<unsigned>(n_qt * a.Hq * a.B), kBThreads, C::kSmem, s>>>(tq, tdo, tk, tv, a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  bwd_dkdv_kernel<D><<<static_cast<unsigned>(n_kt * a.Hkv * a.B), kBThreads, C::kSmem, s>>>(tq, tdo, tk, tv, a);
+  bwd_dkdv_kernel<D><<<static_cast<unsigned>(n_kt * a.Hkv * a.B), kBThreads, C::kSmemKV, s>>>(tq, tdo, tk, tv, a);
   return cudaGetLastError();
 }
 
