@@ -8,8 +8,9 @@
 //   P = exp(S - LSE),  dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
 //   dQ = scale dS K,   dK = scale dS^T Q
 //
-// Two kernels, launched in this order:
-//   bwd_dq_kernel     one CTA per (128-row Q tile, query head, b): Q, dO and
+// Two persistent kernels (one CTA per SM, each walking a longest-first list
+// of work items dealt in rounds of alternating direction), in this order:
+//   bwd_dq_kernel     an item is a (128-row Q tile, query head, b): Q, dO and
 //                     O stay in shared memory while the K / V tiles stream
 //                     through a TMA ring; per K/V tile, on the tensor core,
 //                       S = Q K^T,  dP = dO V^T       (shared x shared)
@@ -20,7 +21,7 @@
 //                     rows are padded to whole tiles (lse2 = +inf, D = 0).
 //                     The dK/dV kernel fetches 128-row runs of both with bulk
 //                     copies on the same barrier as its Q / dO tiles.
-//   bwd_dkdv_kernel   one CTA per (128-key tile, KV head, b): K and V stay
+//   bwd_dkdv_kernel   an item is a (128-key tile, KV head, b): K and V stay
 //                     while the Q / dO tiles of every query head of the group
 //                     stream through, so dK and dV of a KV head sum over its
 //                     G query heads without atomics; per Q tile
@@ -28,6 +29,12 @@
 //                       dV += P^T dO,  dK += dS^T Q
 // S and dP are recomputed by both kernels (seven products instead of five)
 // so that neither needs atomics or a second pass over an fp32 dQ.
+//
+// Across items: the producer loads the next item's resident tiles as soon as
+// the current item's last S / dP MMAs have read them, its first stream tiles
+// queue in the ring behind the current ones, and the next item's first S and
+// dP run on the tensor core while the element-wise warps write the current
+// item's gradients out of TMEM.
 //
 // Roles (320 threads): warp 0 issues the TMA copies, warp 1 owns TMEM and
 // issues the tcgen05 MMAs from an elect.sync-chosen lane, warps 2..9 are two
@@ -45,6 +52,7 @@
 // kernel at d = 64): S(t+1) then runs on the tensor core while the
 // element-wise warps still work on tile t.
 //   dQ:         S0 [0,128) S1 [128,256) dP [256,384) dQ [384, 384+d)
+//               (d = 64: a second dQ at [448,512), alternating by item)
 //   dK/dV d=64: S0 [0,128) S1 [128,256) dP [256,384) dV [384,448) dK [448,512)
 //   dK/dV d=128: S [0,128) dP [128,256) dV [256,384) dK [384,512)
 #include <cuda_bf16.h>
@@ -72,15 +80,78 @@ struct BCfg {
   static constexpr int kOffX = kOffRing + R * 2 * kTile;
   static constexpr int kOffBarKV = kOffX + R * 2 * kT * 4;
   static constexpr int kOffBarQ = kOffX + kTile;
-  // fixed_full, full[R], empty[R], s_full[2], dp_full, p_full, ds_full, mma_done, mma_idle
-  static constexpr int kNumBars = 1 + 2 * R + 7;
+  // fixed_full, fixed_empty, full[R], empty[R], s_full[2], dp_full, p_full, ds_full,
+  // mma_done, acc_free[2], mma_idle
+  static constexpr int kNumBars = 2 * R + 11;
   static constexpr int kSmemKV = kOffBarKV + 8 * kNumBars + 16 + 1024;
   static constexpr int kSmemQ = kOffBarQ + 8 * kNumBars + 16 + 1024;
   static_assert(kSmemKV <= 227 * 1024 && kSmemQ <= 227 * 1024, "shared memory per CTA");
   static constexpr int kVecBytes = 2 * kT * 4;
   // S buffers in TMEM (dK/dV kernel; the dQ kernel always has two)
   static constexpr int kSBufKV = D == 64 ? 2 : 1;
+  static constexpr int kAccQ = D == 64 ? 2 : 1;  // dQ accumulators in TMEM
 };
+
+// Barriers shared by both kernels' layouts (p_full is unused by the dQ kernel).
+struct BBars {
+  uint64_t *fixed_full, *fixed_empty, *full, *empty, *s_full, *dp_full, *p_full, *ds_full, *mma_done, *acc_free,
+      *mma_idle;
+  __device__ BBars(uint64_t* b, int R)
+      : fixed_full(b), fixed_empty(b + 1), full(b + 2), empty(b + 2 + R), s_full(b + 2 + 2 * R),
+        dp_full(b + 4 + 2 * R), p_full(b + 5 + 2 * R), ds_full(b + 6 + 2 * R), mma_done(b + 7 + 2 * R),
+        acc_free(b + 8 + 2 * R), mma_idle(b + 10 + 2 * R) {}
+};
+
+// The k-th item of this CTA, or -1: items are numbered longest first and
+// dealt in rounds of gridDim.x, alternating direction.
+__device__ __forceinline__ long long bwd_item(long long k, long long n_items) {
+  const long long g = gridDim.x, base = k * g;
+  if (base >= n_items) return -1;
+  const long long idx = (k & 1) ? base + (g - 1 - blockIdx.x) : base + blockIdx.x;
+  return idx < n_items ? idx : -1;
+}
+
+// dK/dV item: KV tile slowest (under a causal mask the first tiles visit the
+// most Q tiles).
+struct KvItem {
+  int b, hkv, k0, first_qt, per_head, steps;
+};
+__device__ __forceinline__ KvItem kv_item(const BwdArgs& a, long long w) {
+  KvItem it;
+  const int per_kt = a.Hkv * a.B;
+  const int r = static_cast<int>(w % per_kt);
+  it.k0 = static_cast<int>(w / per_kt) * kT;
+  it.hkv = r / a.B;
+  it.b = r % a.B;
+  const int n_qt = (a.Nq + kT - 1) / kT;
+  // causal: row i sees key k0 iff i >= k0 - off; earlier Q tiles see none of these keys
+  it.first_qt = a.causal ? min(n_qt, max(0, it.k0 - (a.Nkv - a.Nq)) / kT) : 0;
+  it.per_head = n_qt - it.first_qt;
+  it.steps = (a.Hq / a.Hkv) * it.per_head;
+  return it;
+}
+
+// dQ item: Q tile slowest, last tile first (under a causal mask the last
+// tiles visit the most K/V tiles).
+struct QItem {
+  int b, hq, q0, n_kv;
+};
+__device__ __forceinline__ QItem q_item(const BwdArgs& a, long long w) {
+  QItem it;
+  const int per_qt = a.Hq * a.B;
+  const int n_qt = (a.Nq + kT - 1) / kT;
+  const int r = static_cast<int>(w % per_qt);
+  it.q0 = (n_qt - 1 - static_cast<int>(w / per_qt)) * kT;
+  it.hq = r / a.B;
+  it.b = r % a.B;
+  int n_kv = (a.Nkv + kT - 1) / kT;
+  if (a.causal) {
+    const int last = min(it.q0 + kT - 1, a.Nq - 1) + (a.Nkv - a.Nq);  // largest key any row may see
+    n_kv = last < 0 ? 0 : min(n_kv, last / kT + 1);
+  }
+  it.n_kv = n_kv;
+  return it;
+}
 
 __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -168,49 +239,34 @@ __global__ void __launch_bounds__(kBThreads, 1)
   constexpr uint32_t kColDP = 128 * NB, kColDV = kColDP + 128, kColDK = kColDV + D;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBarKV);
-  uint64_t* fixed_full = bars;
-  uint64_t* full = bars + 1;
-  uint64_t* empty = full + R;
-  uint64_t* s_full = empty + R;  // [2]
-  uint64_t* dp_full = s_full + 2;
-  uint64_t* p_full = dp_full + 1;
-  uint64_t* ds_full = p_full + 1;
-  uint64_t* mma_done = ds_full + 1;
-  uint64_t* mma_idle = mma_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  uint64_t* bar_base = reinterpret_cast<uint64_t*>(smem + C::kOffBarKV);
+  const BBars br(bar_base, R);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_base + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* vec = reinterpret_cast<float*>(smem + C::kOffX);  // [R][2][128]: lse2, D
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Linear grid, KV tile slowest: under a causal mask the first tiles have
-  // the most Q tiles to visit, so the longest CTAs start first.
-  const int per_kt = a.Hkv * a.B;
-  const int kt = static_cast<int>(blockIdx.x) / per_kt;
-  const int hkv = (static_cast<int>(blockIdx.x) % per_kt) / a.B, b = static_cast<int>(blockIdx.x) % a.B;
   const int G = a.Hq / a.Hkv;
-  const int k0 = kt * kT;
   const int off = a.Nkv - a.Nq;  // bottom-right causal alignment
-  const int n_qt = (a.Nq + kT - 1) / kT;
-  const int nq_pad = n_qt * kT;  // rows per (b, head) of the lse2 / D scratch
-  // causal: row i sees key k0 iff i >= k0 - off; earlier Q tiles see none of these keys
-  const int first_qt = a.causal ? min(n_qt, max(0, k0 - off) / kT) : 0;
-  const int per_head = n_qt - first_qt;
-  const int steps = G * per_head;
+  const int nq_pad = (a.Nq + kT - 1) / kT * kT;  // rows per (b, head) of the lse2 / D scratch
+  const long long n_items = static_cast<long long>((a.Nkv + kT - 1) / kT) * a.Hkv * a.B;
 
   if (threadIdx.x == 0) {
-    mbar_init(fixed_full, 1);
+    mbar_init(br.fixed_full, 1);
+    mbar_init(br.fixed_empty, 1);
     for (int s = 0; s < R; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + kEW);  // the MMA commit, and each element-wise warp after reading the vectors
+      mbar_init(&br.full[s], 1);
+      mbar_init(&br.empty[s], 1 + kEW);  // the MMA commit, and each element-wise warp after reading the vectors
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(dp_full, 1);
-    mbar_init(p_full, kEW);
-    mbar_init(ds_full, kEW);
-    mbar_init(mma_done, 1);
-    mbar_init(mma_idle, 1);
+    mbar_init(&br.s_full[0], 1);
+    mbar_init(&br.s_full[1], 1);
+    mbar_init(br.dp_full, 1);
+    mbar_init(br.p_full, kEW);
+    mbar_init(br.ds_full, kEW);
+    mbar_init(br.mma_done, 1);
+    mbar_init(&br.acc_free[0], kEW);
+    mbar_init(&br.acc_free[1], kEW);
+    mbar_init(br.mma_idle, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -231,183 +287,226 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const bool mine = !*abort_flag && mbar_wait(bar, parity);
     return __all_sync(0xffffffffu, mine);
   };
+  auto stage = [&](uint32_t t) { return smem + C::kOffRing + (t % R) * 2 * C::kTile; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmDO);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
     }
-    mbar_arrive_expect_tx_elect(fixed_full, 2 * C::kTile);
-#pragma unroll
-    for (int ch = 0; ch < C::NCH; ++ch) {
-      tma_load_4d_elect(smem + ch * C::kChunk, &tmK, fixed_full, 64 * ch, hkv, k0, b);
-      tma_load_4d_elect(smem + C::kTile + ch * C::kChunk, &tmV, fixed_full, 64 * ch, hkv, k0, b);
-    }
+    uint32_t g = 0, nfix = 0;
     bool ok = true;
-    int u = 0;
-    for (; u < steps; ++u) {
-      const int s = u % R;
-      if (u >= R && !wwait(&empty[s], ((u / R) - 1) & 1)) {
+    for (long long k = 0; ok; ++k) {
+      const long long w = bwd_item(k, n_items);
+      if (w < 0) break;
+      const KvItem it = kv_item(a, w);
+      // K and V of the previous item are free once its last S and dP have run
+      if (k > 0 && !wwait(br.fixed_empty, (k - 1) & 1)) {
         ok = false;
         break;
       }
-      const int hq = hkv * G + u / per_head, qt = first_qt + u % per_head;
-      uint8_t* st = smem + C::kOffRing + s * 2 * C::kTile;
-      mbar_arrive_expect_tx_elect(&full[s], 2 * C::kTile + C::kVecBytes);
+      mbar_arrive_expect_tx_elect(br.fixed_full, 2 * C::kTile);
 #pragma unroll
       for (int ch = 0; ch < C::NCH; ++ch) {
-        tma_load_4d_elect(st + ch * C::kChunk, &tmQ, &full[s], 64 * ch, hq, qt * kT, b);
-        tma_load_4d_elect(st + C::kTile + ch * C::kChunk, &tmDO, &full[s], 64 * ch, hq, qt * kT, b);
+        tma_load_4d_elect(smem + ch * C::kChunk, &tmK, br.fixed_full, 64 * ch, it.hkv, it.k0, it.b);
+        tma_load_4d_elect(smem + C::kTile + ch * C::kChunk, &tmV, br.fixed_full, 64 * ch, it.hkv, it.k0, it.b);
       }
-      // the tile's 128 lse2 and D values (padded rows: lse2 = +inf, D = 0)
-      const size_t vrow = (static_cast<size_t>(b) * a.Hq + hq) * nq_pad + static_cast<size_t>(qt) * kT;
-      bulk_load_elect(vec + s * 2 * kT, a.lse2 + vrow, kT * 4, &full[s]);
-      bulk_load_elect(vec + s * 2 * kT + kT, a.dvec + vrow, kT * 4, &full[s]);
+      ++nfix;
+      for (int u = 0; u < it.steps; ++u, ++g) {
+        const int s = g % R;
+        if (g >= R && !wwait(&br.empty[s], ((g / R) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        const int hq = it.hkv * G + u / it.per_head, qt = it.first_qt + u % it.per_head;
+        uint8_t* st = stage(g);
+        mbar_arrive_expect_tx_elect(&br.full[s], 2 * C::kTile + C::kVecBytes);
+#pragma unroll
+        for (int ch = 0; ch < C::NCH; ++ch) {
+          tma_load_4d_elect(st + ch * C::kChunk, &tmQ, &br.full[s], 64 * ch, hq, qt * kT, it.b);
+          tma_load_4d_elect(st + C::kTile + ch * C::kChunk, &tmDO, &br.full[s], 64 * ch, hq, qt * kT, it.b);
+        }
+        // the tile's 128 lse2 and D values (padded rows: lse2 = +inf, D = 0)
+        const size_t vrow = (static_cast<size_t>(it.b) * a.Hq + hq) * nq_pad + static_cast<size_t>(qt) * kT;
+        bulk_load_elect(vec + s * 2 * kT, a.lse2 + vrow, kT * 4, &br.full[s]);
+        bulk_load_elect(vec + s * 2 * kT + kT, a.dvec + vrow, kT * 4, &br.full[s]);
+      }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
     // Every copy lands before the CTA retires.
-    mbar_wait(fixed_full, 0);
-    for (int w = u > R ? u - R : 0; w < u; ++w) mbar_wait(&full[w % R], (w / R) & 1);
+    if (nfix > 0) mbar_wait(br.fixed_full, (nfix - 1) & 1);
+    for (uint32_t t = g > R ? g - R : 0; t < g; ++t) mbar_wait(&br.full[t % R], (t / R) & 1);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // Issue order per step t: S(t+1) (two S buffers), dV(t), dK(t), then
     // dP(t+1) -- the element-wise warps have read dP(t) by then.
     const uint32_t sK = smem_u32(smem), sV = sK + C::kTile;
-    auto stage = [&](int t) { return smem_u32(smem + C::kOffRing + (t % R) * 2 * C::kTile); };
-    bool ok = wwait(fixed_full, 0) && (steps == 0 || wwait(&full[0], 0));
-    if (ok && steps > 0) {
-      tc_fence_after();
-      issue_ss<D>(tmem, sK, stage(0));  // S^T = K Q^T
-      mma_commit_elect(&s_full[0]);
-      issue_ss<D>(tmem + kColDP, sV, stage(0) + C::kTile);  // dP^T = V dO^T
-      mma_commit_elect(dp_full);
-    }
-    for (int u = 0; ok && u < steps; ++u) {
-      const int s = u % R, x = u % NB;
-      const uint32_t sQ = stage(u), sdO = sQ + C::kTile;
-      const bool next = u + 1 < steps;
-      if (NB == 2 && next) {
-        // S buffer (u+1)%2 was last read by dV(u-1) / dK(u-1)
-        if (!wwait(&full[(u + 1) % R], ((u + 1) / R) & 1) || (u >= 1 && !wwait(mma_done, (u - 1) & 1))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        issue_ss<D>(tmem + 128 * ((u + 1) % NB), sK, stage(u + 1));
-        mma_commit_elect(&s_full[(u + 1) % NB]);
+    uint32_t g = 0;
+    bool ok = true;
+    for (long long k = 0; ok; ++k) {
+      const long long w = bwd_item(k, n_items);
+      if (w < 0) break;
+      const KvItem it = kv_item(a, w);
+      if (!wwait(br.fixed_full, k & 1)) {
+        ok = false;
+        break;
       }
-      if (!wwait(p_full, u & 1)) {
+      if (it.steps == 0) {
+        mma_commit_elect(br.fixed_empty);
+        continue;
+      }
+      // every earlier MMA has completed: both S buffers and dP are free
+      if (!wwait(&br.full[g % R], (g / R) & 1) || (g > 0 && !wwait(br.mma_done, (g - 1) & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      issue_ts<D>(tmem + kColDV, tmem + 128 * x, sdO, u > 0);  // dV += P^T dO
-      if (!wwait(ds_full, u & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      issue_ts<D>(tmem + kColDK, tmem + 128 * x + 32, sQ, u > 0);  // dK += dS^T Q
-      mma_commit_elect(&empty[s]);
-      mma_commit_elect(mma_done);
-      if (next) {
-        if (NB == 1) {
-          // one S buffer: S(u+1) after dV(u) / dK(u) have read it
-          if (!wwait(&full[(u + 1) % R], ((u + 1) / R) & 1) || !wwait(mma_done, u & 1)) {
+      issue_ss<D>(tmem + 128 * (g % NB), sK, smem_u32(stage(g)));  // S^T = K Q^T
+      mma_commit_elect(&br.s_full[g % NB]);
+      issue_ss<D>(tmem + kColDP, sV, smem_u32(stage(g)) + C::kTile);  // dP^T = V dO^T
+      mma_commit_elect(br.dp_full);
+      if (it.steps == 1) mma_commit_elect(br.fixed_empty);
+      for (int u = 0; u < it.steps; ++u, ++g) {
+        const int s = g % R, x = g % NB;
+        const uint32_t sQ = smem_u32(stage(g)), sdO = sQ + C::kTile;
+        const bool next = u + 1 < it.steps;
+        if (NB == 2 && next) {
+          // S buffer (g+1)%2 was last read by dV(g-1) / dK(g-1)
+          if (!wwait(&br.full[(g + 1) % R], ((g + 1) / R) & 1) || (u >= 1 && !wwait(br.mma_done, (g - 1) & 1))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_ss<D>(tmem, sK, stage(u + 1));
-          mma_commit_elect(&s_full[0]);
+          issue_ss<D>(tmem + 128 * ((g + 1) % NB), sK, smem_u32(stage(g + 1)));
+          mma_commit_elect(&br.s_full[(g + 1) % NB]);
         }
-        issue_ss<D>(tmem + kColDP, sV, stage(u + 1) + C::kTile);
-        mma_commit_elect(dp_full);
+        // dV / dK of the previous item have been read out of TMEM
+        if (!wwait(br.p_full, g & 1) || (u == 0 && k > 0 && !wwait(&br.acc_free[0], (k - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_ts<D>(tmem + kColDV, tmem + 128 * x, sdO, u > 0);  // dV += P^T dO
+        if (!wwait(br.ds_full, g & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_ts<D>(tmem + kColDK, tmem + 128 * x + 32, sQ, u > 0);  // dK += dS^T Q
+        mma_commit_elect(&br.empty[s]);
+        mma_commit_elect(br.mma_done);
+        if (next) {
+          if (NB == 1) {
+            // one S buffer: S(g+1) after dV(g) / dK(g) have read it
+            if (!wwait(&br.full[(g + 1) % R], ((g + 1) / R) & 1) || !wwait(br.mma_done, g & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_ss<D>(tmem, sK, smem_u32(stage(g + 1)));
+            mma_commit_elect(&br.s_full[0]);
+          }
+          issue_ss<D>(tmem + kColDP, sV, smem_u32(stage(g + 1)) + C::kTile);
+          mma_commit_elect(br.dp_full);
+          if (u + 2 == it.steps) mma_commit_elect(br.fixed_empty);  // the item's last S and dP
+        }
       }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
     // Every MMA issued above has finished before TMEM is released.
-    mma_commit_elect(mma_idle);
-    mbar_wait(mma_idle, 0);
+    mma_commit_elect(br.mma_idle);
+    mbar_wait(br.mma_idle, 0);
   } else {
     // ------------------------------------------------------------ element-wise
     const int h = (warp - 2) >> 2;  // column half
     const int quarter = warp & 3;
-    const int key = k0 + quarter * 32 + lane;  // this thread's key (TMEM lane)
     const uint32_t lo = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t t_row = tmem + lo;
     const float sl2 = a.scale * kLog2e;
+    uint32_t g = 0;
     bool ok = true;
-    for (int u = 0; u < steps; ++u) {
-      const int s = u % R, x = u % NB;
-      const int q0 = (first_qt + u % per_head) * kT + 64 * h;  // query of this thread's first column
-      if (!wwait(&full[s], (u / R) & 1) || !wwait(&s_full[x], (u / NB) & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float* vs = vec + s * 2 * kT + 64 * h;
-      const uint32_t t_s = t_row + 128 * x + 64 * h;
-      float p[64];
-      {
-        uint32_t sr[64];
-        tmem_ld32(t_s, sr);
-        tmem_ld32(t_s + 32, sr + 32);
-        tmem_wait_ld();
-        // causal: query q0 + c sees this key iff c >= key - off - q0
-        const bool masked_tile = a.causal && k0 + kT - 1 > q0 + off;
-        const int lim = masked_tile ? key - off - q0 : -1;
+    for (long long k = 0; ok; ++k) {
+      const long long w = bwd_item(k, n_items);
+      if (w < 0) break;
+      const KvItem it = kv_item(a, w);
+      const int key = it.k0 + quarter * 32 + lane;  // this thread's key (TMEM lane)
+      for (int u = 0; u < it.steps; ++u, ++g) {
+        const int s = g % R, x = g % NB;
+        const int q0 = (it.first_qt + u % it.per_head) * kT + 64 * h;  // query of this thread's first column
+        if (!wwait(&br.full[s], (g / R) & 1) || !wwait(&br.s_full[x], (g / NB) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float* vs = vec + s * 2 * kT + 64 * h;
+        const uint32_t t_s = t_row + 128 * x + 64 * h;
+        float p[64];
+        {
+          uint32_t sr[64];
+          tmem_ld32(t_s, sr);
+          tmem_ld32(t_s + 32, sr + 32);
+          tmem_wait_ld();
+          // causal: query q0 + c sees this key iff c >= key - off - q0
+          const bool masked_tile = a.causal && it.k0 + kT - 1 > q0 + off;
+          const int lim = masked_tile ? key - off - q0 : -1;
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(vs + c);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          for (int c = 0; c < 64; c += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(vs + c);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            p[c + e] = c + e < lim ? 0.f : wm_ex2(fmaf(__uint_as_float(sr[c + e]), sl2, -lv[e]));
+            for (int e = 0; e < 4; ++e)
+              p[c + e] = c + e < lim ? 0.f : wm_ex2(fmaf(__uint_as_float(sr[c + e]), sl2, -lv[e]));
+          }
+        }
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pk[j] = wm_pack_bf16x2(p[2 * j], p[2 * j + 1]);
+          tmem_st32(t_s, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(br.p_full);
+        if (!wwait(br.dp_full, g & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        write_ds(t_row + kColDP + 64 * h, t_s + 32, p,
+                 [&](int c) { return *reinterpret_cast<const float2*>(vs + kT + c); });
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(br.ds_full);
+          mbar_arrive(&br.empty[s]);
         }
       }
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) pk[j] = wm_pack_bf16x2(p[2 * j], p[2 * j + 1]);
-        tmem_st32(t_s, pk);
+      if (!ok) break;
+      if (it.steps > 0) {
+        if (!wwait(br.mma_done, (g - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-      if (!wwait(dp_full, u & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      write_ds(t_row + kColDP + 64 * h, t_s + 32, p,
-               [&](int c) { return *reinterpret_cast<const float2*>(vs + kT + c); });
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(ds_full);
-        mbar_arrive(&empty[s]);
-      }
-    }
-    if (ok && steps > 0) {
-      ok = wwait(mma_done, (steps - 1) & 1);
-      tc_fence_after();
-    }
-    if (ok) {
       // each warpgroup stores half of the columns of dV and dK
       constexpr int HC = D / 2;
-      const size_t o = ((static_cast<size_t>(b) * a.Nkv + key) * a.Hkv + hkv) * D + HC * h;
+      const size_t o = ((static_cast<size_t>(it.b) * a.Nkv + key) * a.Hkv + it.hkv) * D + HC * h;
       const bool valid = key < a.Nkv;
       store_cols<HC>(t_row + kColDV + HC * h, valid ? reinterpret_cast<__nv_bfloat16*>(a.dv) + o : nullptr, 1.f,
-                     steps > 0);
-      store_cols<HC>(t_row + kColDK + HC * h, valid ? reinterpret_cast<__nv_bfloat16*>(a.dk) + o : nullptr,
-                     a.scale, steps > 0);
-    } else if (lane == 0) {
-      fail(kErrDeviceTimeout);
+                     it.steps > 0);
+      store_cols<HC>(t_row + kColDK + HC * h, valid ? reinterpret_cast<__nv_bfloat16*>(a.dk) + o : nullptr, a.scale,
+                     it.steps > 0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&br.acc_free[0]);
     }
+    if (!ok && lane == 0) fail(kErrDeviceTimeout);
   }
 
   tc_fence_before();
@@ -423,50 +522,36 @@ __global__ void __launch_bounds__(kBThreads, 1)
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmO, const BwdArgs a) {
   using C = BCfg<D>;
-  constexpr int R = C::R;
+  constexpr int R = C::R, NA = C::kAccQ;
   constexpr uint32_t kColDP = 256, kColDQ = 384;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1k(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBarQ);
-  uint64_t* fixed_full = bars;
-  uint64_t* full = bars + 1;
-  uint64_t* empty = full + R;
-  uint64_t* s_full = empty + R;  // [2]
-  uint64_t* dp_full = s_full + 2;
-  uint64_t* ds_full = dp_full + 2;  // p_full is unused here
-  uint64_t* mma_done = ds_full + 1;
-  uint64_t* mma_idle = mma_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  uint64_t* bar_base = reinterpret_cast<uint64_t*>(smem + C::kOffBarQ);
+  const BBars br(bar_base, R);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_base + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Linear grid, Q tile slowest and last tile first: under a causal mask the
-  // last tiles visit the most K/V tiles.
-  const int per_qt = a.Hq * a.B;
-  const int n_qt = (a.Nq + kT - 1) / kT;
-  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x) / per_qt;
-  const int hq = (static_cast<int>(blockIdx.x) % per_qt) / a.B, b = static_cast<int>(blockIdx.x) % a.B;
-  const int hkv = hq / (a.Hq / a.Hkv);
-  const int q0 = qt * kT;
+  const int G = a.Hq / a.Hkv;
   const int off = a.Nkv - a.Nq;
-  int n_kv = (a.Nkv + kT - 1) / kT;
-  if (a.causal) {
-    const int last = min(q0 + kT - 1, a.Nq - 1) + off;  // largest key any row may see
-    n_kv = last < 0 ? 0 : min(n_kv, last / kT + 1);
-  }
+  const int nq_pad = (a.Nq + kT - 1) / kT * kT;
+  const long long n_items = static_cast<long long>((a.Nq + kT - 1) / kT) * a.Hq * a.B;
 
   if (threadIdx.x == 0) {
-    mbar_init(fixed_full, 1);
+    mbar_init(br.fixed_full, 1);
+    mbar_init(br.fixed_empty, 1 + kEW);  // the MMA commit, and each element-wise warp after reading O and dO
     for (int s = 0; s < R; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&br.full[s], 1);
+      mbar_init(&br.empty[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(dp_full, 1);
-    mbar_init(ds_full, kEW);
-    mbar_init(mma_done, 1);
-    mbar_init(mma_idle, 1);
+    mbar_init(&br.s_full[0], 1);
+    mbar_init(&br.s_full[1], 1);
+    mbar_init(br.dp_full, 1);
+    mbar_init(br.ds_full, kEW);
+    mbar_init(br.mma_done, 1);
+    mbar_init(&br.acc_free[0], kEW);
+    mbar_init(&br.acc_free[1], kEW);
+    mbar_init(br.mma_idle, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -487,174 +572,228 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const bool mine = !*abort_flag && mbar_wait(bar, parity);
     return __all_sync(0xffffffffu, mine);
   };
+  auto stage = [&](uint32_t t) { return smem + C::kOffRing + (t % R) * 2 * C::kTile; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmDO);
+      tma_prefetch_desc(&tmO);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
-    mbar_arrive_expect_tx_elect(fixed_full, 3 * C::kTile);
-#pragma unroll
-    for (int ch = 0; ch < C::NCH; ++ch) {
-      tma_load_4d_elect(smem + ch * C::kChunk, &tmQ, fixed_full, 64 * ch, hq, q0, b);
-      tma_load_4d_elect(smem + C::kTile + ch * C::kChunk, &tmDO, fixed_full, 64 * ch, hq, q0, b);
-      tma_load_4d_elect(smem + C::kOffX + ch * C::kChunk, &tmO, fixed_full, 64 * ch, hq, q0, b);
-    }
+    uint32_t g = 0, nfix = 0;
     bool ok = true;
-    int j = 0;
-    for (; j < n_kv; ++j) {
-      const int s = j % R;
-      if (j >= R && !wwait(&empty[s], ((j / R) - 1) & 1)) {
+    for (long long k = 0; ok; ++k) {
+      const long long w = bwd_item(k, n_items);
+      if (w < 0) break;
+      const QItem it = q_item(a, w);
+      // Q, dO and O of the previous item are free once its last S and dP
+      // have run and D has been computed
+      if (k > 0 && !wwait(br.fixed_empty, (k - 1) & 1)) {
         ok = false;
         break;
       }
-      uint8_t* st = smem + C::kOffRing + s * 2 * C::kTile;
-      mbar_arrive_expect_tx_elect(&full[s], 2 * C::kTile);
+      mbar_arrive_expect_tx_elect(br.fixed_full, 3 * C::kTile);
 #pragma unroll
       for (int ch = 0; ch < C::NCH; ++ch) {
-        tma_load_4d_elect(st + ch * C::kChunk, &tmK, &full[s], 64 * ch, hkv, j * kT, b);
-        tma_load_4d_elect(st + C::kTile + ch * C::kChunk, &tmV, &full[s], 64 * ch, hkv, j * kT, b);
+        tma_load_4d_elect(smem + ch * C::kChunk, &tmQ, br.fixed_full, 64 * ch, it.hq, it.q0, it.b);
+        tma_load_4d_elect(smem + C::kTile + ch * C::kChunk, &tmDO, br.fixed_full, 64 * ch, it.hq, it.q0, it.b);
+        tma_load_4d_elect(smem + C::kOffX + ch * C::kChunk, &tmO, br.fixed_full, 64 * ch, it.hq, it.q0, it.b);
+      }
+      ++nfix;
+      const int hkv = it.hq / G;
+      for (int j = 0; j < it.n_kv; ++j, ++g) {
+        const int s = g % R;
+        if (g >= R && !wwait(&br.empty[s], ((g / R) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = stage(g);
+        mbar_arrive_expect_tx_elect(&br.full[s], 2 * C::kTile);
+#pragma unroll
+        for (int ch = 0; ch < C::NCH; ++ch) {
+          tma_load_4d_elect(st + ch * C::kChunk, &tmK, &br.full[s], 64 * ch, hkv, j * kT, it.b);
+          tma_load_4d_elect(st + C::kTile + ch * C::kChunk, &tmV, &br.full[s], 64 * ch, hkv, j * kT, it.b);
+        }
       }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
-    mbar_wait(fixed_full, 0);
-    for (int w = j > R ? j - R : 0; w < j; ++w) mbar_wait(&full[w % R], (w / R) & 1);
+    if (nfix > 0) mbar_wait(br.fixed_full, (nfix - 1) & 1);
+    for (uint32_t t = g > R ? g - R : 0; t < g; ++t) mbar_wait(&br.full[t % R], (t / R) & 1);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // Issue order per step t: S(t+1) into the other S buffer, dQ(t), then
     // dP(t+1) -- the element-wise warps have read dP(t) by then.
     const uint32_t sQ = smem_u32(smem), sdO = sQ + C::kTile;
-    auto stage = [&](int t) { return smem_u32(smem + C::kOffRing + (t % R) * 2 * C::kTile); };
-    bool ok = wwait(fixed_full, 0) && (n_kv == 0 || wwait(&full[0], 0));
-    if (ok && n_kv > 0) {
+    uint32_t g = 0;
+    bool ok = true;
+    for (long long k = 0; ok; ++k) {
+      const long long w = bwd_item(k, n_items);
+      if (w < 0) break;
+      const QItem it = q_item(a, w);
+      const int acc = static_cast<int>(k % NA);
+      if (!wwait(br.fixed_full, k & 1)) {
+        ok = false;
+        break;
+      }
+      if (it.n_kv == 0) {
+        mma_commit_elect(br.fixed_empty);
+        continue;
+      }
+      // every earlier MMA has completed: both S buffers and dP are free
+      if (!wwait(&br.full[g % R], (g / R) & 1) || (g > 0 && !wwait(br.mma_done, (g - 1) & 1))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      issue_ss<D>(tmem, sQ, stage(0));  // S = Q K^T
-      mma_commit_elect(&s_full[0]);
-      issue_ss<D>(tmem + kColDP, sdO, stage(0) + C::kTile);  // dP = dO V^T
-      mma_commit_elect(dp_full);
-    }
-    for (int j = 0; ok && j < n_kv; ++j) {
-      const int s = j % R, x = j & 1;
-      const bool next = j + 1 < n_kv;
-      if (next) {
-        // S buffer (j+1)%2 was last read by dQ(j-1)
-        if (!wwait(&full[(j + 1) % R], ((j + 1) / R) & 1) || (j >= 1 && !wwait(mma_done, (j - 1) & 1))) {
+      issue_ss<D>(tmem + 128 * (g & 1), sQ, smem_u32(stage(g)));  // S = Q K^T
+      mma_commit_elect(&br.s_full[g & 1]);
+      issue_ss<D>(tmem + kColDP, sdO, smem_u32(stage(g)) + C::kTile);  // dP = dO V^T
+      mma_commit_elect(br.dp_full);
+      if (it.n_kv == 1) mma_commit_elect(br.fixed_empty);
+      for (int j = 0; j < it.n_kv; ++j, ++g) {
+        const int s = g % R, x = g & 1;
+        const bool next = j + 1 < it.n_kv;
+        if (next) {
+          // S buffer (g+1)%2 was last read by dQ(g-1)
+          if (!wwait(&br.full[(g + 1) % R], ((g + 1) / R) & 1) || (j >= 1 && !wwait(br.mma_done, (g - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_ss<D>(tmem + 128 * (x ^ 1), sQ, smem_u32(stage(g + 1)));
+          mma_commit_elect(&br.s_full[x ^ 1]);
+        }
+        // this dQ buffer was read out by the epilogue of item k - NA
+        if (!wwait(br.ds_full, g & 1) || (j == 0 && k >= NA && !wwait(&br.acc_free[acc], ((k / NA) - 1) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        issue_ss<D>(tmem + 128 * (x ^ 1), sQ, stage(j + 1));
-        mma_commit_elect(&s_full[x ^ 1]);
-      }
-      if (!wwait(ds_full, j & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      issue_ts<D>(tmem + kColDQ, tmem + 128 * x, stage(j), j > 0);  // dQ += dS K
-      mma_commit_elect(&empty[s]);
-      mma_commit_elect(mma_done);
-      if (next) {
-        issue_ss<D>(tmem + kColDP, sdO, stage(j + 1) + C::kTile);
-        mma_commit_elect(dp_full);
+        issue_ts<D>(tmem + kColDQ + D * acc, tmem + 128 * x, smem_u32(stage(g)), j > 0);  // dQ += dS K
+        mma_commit_elect(&br.empty[s]);
+        mma_commit_elect(br.mma_done);
+        if (next) {
+          issue_ss<D>(tmem + kColDP, sdO, smem_u32(stage(g + 1)) + C::kTile);
+          mma_commit_elect(br.dp_full);
+          if (j + 2 == it.n_kv) mma_commit_elect(br.fixed_empty);  // the item's last S and dP
+        }
       }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
-    mma_commit_elect(mma_idle);
-    mbar_wait(mma_idle, 0);
+    mma_commit_elect(br.mma_idle);
+    mbar_wait(br.mma_idle, 0);
   } else {
     // ------------------------------------------------------------ element-wise
     const int h = (warp - 2) >> 2;  // column half
     const int quarter = warp & 3;
-    const int row = q0 + quarter * 32 + lane;  // this thread's query row (TMEM lane)
+    const int r = quarter * 32 + lane;  // this thread's row of the tile (TMEM lane)
     const uint32_t lo = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t t_row = tmem + lo;
     const float sl2 = a.scale * kLog2e;
-    // rows past Nq: lse2 = +inf makes their P exactly 0
-    const float l2 = row < a.Nq ? a.lse[(static_cast<size_t>(b) * a.Hq + hq) * a.Nq + row] * kLog2e : INFINITY;
-    // D = rowsum(dO * O) from the resident O and dO tiles (zero rows past
-    // Nq); with lse2 it goes to the padded scratch for the dK/dV kernel.
-    float dd = 0.f;
-    auto compute_d = [&]() -> bool {
-      if (!wwait(fixed_full, 0)) return false;
-      const int r = quarter * 32 + lane;
-#pragma unroll
-      for (int ch = 0; ch < C::NCH; ++ch)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int o = ch * C::kChunk + r * 128 + ((u ^ (r & 7)) << 4);
-          const uint4 ov = *reinterpret_cast<const uint4*>(smem + C::kOffX + o);
-          const uint4 gv = *reinterpret_cast<const uint4*>(smem + C::kTile + o);
-          const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-          const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const float2 of = __bfloat1622float2(o2[w]), gf = __bfloat1622float2(g2[w]);
-            dd = fmaf(of.x, gf.x, dd);
-            dd = fmaf(of.y, gf.y, dd);
-          }
-        }
-      if (h == 0) {
-        const size_t vrow = (static_cast<size_t>(b) * a.Hq + hq) * (n_qt * kT) + row;
-        a.dvec[vrow] = dd;
-        a.lse2[vrow] = l2;
-      }
-      return true;
-    };
+    uint32_t g = 0;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int x = j & 1;
-      if (!wwait(&s_full[x], (j >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // keys at or past column lim are masked: past Nkv, and past the
-      // causal diagonal (rows with no visible key get lim <= 0)
-      const int c0 = j * kT + 64 * h;  // key of this thread's first column
-      int lim = min(64, a.Nkv - c0);
-      if (a.causal) lim = min(lim, row + off + 1 - c0);
-      const uint32_t t_s = t_row + 128 * x + 64 * h;
-      float p[64];
-      {
-        uint32_t sr[64];
-        tmem_ld32(t_s, sr);
-        tmem_ld32(t_s + 32, sr + 32);
-        tmem_wait_ld();
+    for (long long k = 0; ok; ++k) {
+      const long long w = bwd_item(k, n_items);
+      if (w < 0) break;
+      const QItem it = q_item(a, w);
+      const int acc = static_cast<int>(k % NA);
+      const int row = it.q0 + r;
+      // rows past Nq: lse2 = +inf makes their P exactly 0
+      const float l2 =
+          row < a.Nq ? a.lse[(static_cast<size_t>(it.b) * a.Hq + it.hq) * a.Nq + row] * kLog2e : INFINITY;
+      // D = rowsum(dO * O) from the resident O and dO tiles (zero rows past
+      // Nq); with lse2 it goes to the padded scratch for the dK/dV kernel.
+      float dd = 0.f;
+      auto compute_d = [&]() -> bool {
+        if (!wwait(br.fixed_full, k & 1)) return false;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) p[c] = c < lim ? wm_ex2(fmaf(__uint_as_float(sr[c]), sl2, -l2)) : 0.f;
+        for (int ch = 0; ch < C::NCH; ++ch)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int o = ch * C::kChunk + r * 128 + ((u ^ (r & 7)) << 4);
+            const uint4 ov = *reinterpret_cast<const uint4*>(smem + C::kOffX + o);
+            const uint4 gv = *reinterpret_cast<const uint4*>(smem + C::kTile + o);
+            const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 of = __bfloat1622float2(o2[e]), gf = __bfloat1622float2(g2[e]);
+              dd = fmaf(of.x, gf.x, dd);
+              dd = fmaf(of.y, gf.y, dd);
+            }
+          }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(br.fixed_empty);  // O and dO read
+        if (h == 0) {
+          const size_t vrow = (static_cast<size_t>(it.b) * a.Hq + it.hq) * nq_pad + row;
+          a.dvec[vrow] = dd;
+          a.lse2[vrow] = l2;
+        }
+        return true;
+      };
+      for (int j = 0; j < it.n_kv; ++j, ++g) {
+        const int x = g & 1;
+        if (!wwait(&br.s_full[x], (g >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // keys at or past column lim are masked: past Nkv, and past the
+        // causal diagonal (rows with no visible key get lim <= 0)
+        const int c0 = j * kT + 64 * h;  // key of this thread's first column
+        int lim = min(64, a.Nkv - c0);
+        if (a.causal) lim = min(lim, row + off + 1 - c0);
+        const uint32_t t_s = t_row + 128 * x + 64 * h;
+        float p[64];
+        {
+          uint32_t sr[64];
+          tmem_ld32(t_s, sr);
+          tmem_ld32(t_s + 32, sr + 32);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 64; ++c) p[c] = c < lim ? wm_ex2(fmaf(__uint_as_float(sr[c]), sl2, -l2)) : 0.f;
+        }
+        // D while dP of the first tile is on the tensor core
+        if (j == 0 && !compute_d()) {
+          ok = false;
+          break;
+        }
+        if (!wwait(br.dp_full, g & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        write_ds(t_row + kColDP + 64 * h, t_s, p, [&](int) { return make_float2(dd, dd); });
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(br.ds_full);
       }
-      // D while dP(0) is on the tensor core
-      if (j == 0 && !compute_d()) {
+      if (!ok) break;
+      if (it.n_kv == 0 && !compute_d()) {
         ok = false;
         break;
       }
-      if (!wwait(dp_full, j & 1)) {
-        ok = false;
-        break;
+      if (it.n_kv > 0) {
+        if (!wwait(br.mma_done, (g - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
       }
-      tc_fence_after();
-      write_ds(t_row + kColDP + 64 * h, t_s, p, [&](int) { return make_float2(dd, dd); });
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
-    }
-    if (ok && n_kv == 0) ok = compute_d();
-    if (ok && n_kv > 0) {
-      ok = wwait(mma_done, (n_kv - 1) & 1);
-      tc_fence_after();
-    }
-    if (ok) {
       constexpr int HC = D / 2;
       __nv_bfloat16* dst = row < a.Nq ? reinterpret_cast<__nv_bfloat16*>(a.dq) +
-                                            ((static_cast<size_t>(b) * a.Nq + row) * a.Hq + hq) * D + HC * h
+                                            ((static_cast<size_t>(it.b) * a.Nq + row) * a.Hq + it.hq) * D + HC * h
                                       : nullptr;
-      store_cols<HC>(t_row + kColDQ + HC * h, dst, a.scale, n_kv > 0);
-    } else if (lane == 0) {
-      fail(kErrDeviceTimeout);
+      store_cols<HC>(t_row + kColDQ + D * acc + HC * h, dst, a.scale, it.n_kv > 0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&br.acc_free[acc]);
     }
+    if (!ok && lane == 0) fail(kErrDeviceTimeout);
   }
 
   tc_fence_before();
@@ -666,13 +805,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
 template <int D>
 cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   using C = BCfg<D>;
-  static int attr_dev = -1;
+  static int attr_dev = -1, n_sm = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
     cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemQ);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemKV);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
@@ -681,12 +821,15 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
       !encode_bf16_map(&tk, a.k, a.B, a.Nkv, a.Hkv, D, kT) || !encode_bf16_map(&tv, a.v, a.B, a.Nkv, a.Hkv, D, kT) ||
       !encode_bf16_map(&to, a.o, a.B, a.Nq, a.Hq, D, kT))
     return cudaErrorInvalidValue;
-  const long long n_qt = (a.Nq + kT - 1) / kT, n_kt = (a.Nkv + kT - 1) / kT;
+  const long long n_q = static_cast<long long>((a.Nq + kT - 1) / kT) * a.Hq * a.B;
+  const long long n_kv = static_cast<long long>((a.Nkv + kT - 1) / kT) * a.Hkv * a.B;
   // The dQ kernel also writes D and lse2, which the dK/dV kernel reads.
-  bwd_dq_kernel<D><<<static_cast<unsigned>(n_qt * a.Hq * a.B), kBThreads, C::kSmemQ, s>>>(tq, tdo, tk, tv, to, a);
+  bwd_dq_kernel<D><<<static_cast<unsigned>(n_q < n_sm ? n_q : n_sm), kBThreads, C::kSmemQ, s>>>(tq, tdo, tk, tv, to,
+                                                                                                 a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dkdv_kernel<D><<<static_cast<unsigned>(n_kt * a.Hkv * a.B), kBThreads, C::kSmemKV, s>>>(tq, tdo, tk, tv, a);
+  bwd_dkdv_kernel<D><<<static_cast<unsigned>(n_kv < n_sm ? n_kv : n_sm), kBThreads, C::kSmemKV, s>>>(tq, tdo, tk, tv,
+                                                                                                     a);
   return cudaGetLastError();
 }
 
