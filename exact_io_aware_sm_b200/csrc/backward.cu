@@ -78,11 +78,17 @@ struct BCfg {
   static constexpr int kOffRing = 2 * kTile;         // after the two resident tiles
   // dK/dV kernel: per stage lse2[128], D[128]; dQ kernel: the O tile
   static constexpr int kOffX = kOffRing + R * 2 * kTile;
-  static constexpr int kOffBarKV = kOffX + R * 2 * kT * 4;
-  static constexpr int kOffBarQ = kOffX + kTile;
+  // d = 64: the gradients leave through 128-byte-swizzled staging tiles in
+  // shared memory and one TMA store per tile (dV and dK, or dQ), instead of
+  // one 16-byte store per row and thread.
+  static constexpr bool kStage = D == 64;
+  static constexpr int kOffStgKV = kOffX + R * 2 * kT * 4;
+  static constexpr int kOffBarKV = kOffStgKV + (kStage ? 2 * kTile : 0);
+  static constexpr int kOffStgQ = kOffX + kTile;
+  static constexpr int kOffBarQ = kOffStgQ + (kStage ? kTile : 0);
   // fixed_full, fixed_empty, full[R], empty[R], s_full[2], dp_full, p_full, ds_full,
-  // mma_done, acc_free[2], mma_idle
-  static constexpr int kNumBars = 2 * R + 11;
+  // mma_done, acc_free[2], mma_idle, stg_full, stg_free
+  static constexpr int kNumBars = 2 * R + 13;
   static constexpr int kSmemKV = kOffBarKV + 8 * kNumBars + 16 + 1024;
   static constexpr int kSmemQ = kOffBarQ + 8 * kNumBars + 16 + 1024;
   static_assert(kSmemKV <= 227 * 1024 && kSmemQ <= 227 * 1024, "shared memory per CTA");
@@ -95,12 +101,25 @@ struct BCfg {
 // Barriers shared by both kernels' layouts (p_full is unused by the dQ kernel).
 struct BBars {
   uint64_t *fixed_full, *fixed_empty, *full, *empty, *s_full, *dp_full, *p_full, *ds_full, *mma_done, *acc_free,
-      *mma_idle;
+      *mma_idle, *stg_full, *stg_free;
   __device__ BBars(uint64_t* b, int R)
       : fixed_full(b), fixed_empty(b + 1), full(b + 2), empty(b + 2 + R), s_full(b + 2 + 2 * R),
         dp_full(b + 4 + 2 * R), p_full(b + 5 + 2 * R), ds_full(b + 6 + 2 * R), mma_done(b + 7 + 2 * R),
-        acc_free(b + 8 + 2 * R), mma_idle(b + 10 + 2 * R) {}
+        acc_free(b + 8 + 2 * R), mma_idle(b + 10 + 2 * R), stg_full(b + 11 + 2 * R), stg_free(b + 12 + 2 * R) {}
 };
+
+// One element-wise thread's NC TMEM columns (times mul) as bf16 into a
+// 128-byte-swizzled staging row, at 16-byte unit u0 onwards.
+template <int NC>
+__device__ __forceinline__ void stage_row(uint8_t* stg, int r, int u0, const uint32_t* v, float mul) {
+#pragma unroll
+  for (int u = 0; u < NC / 8; ++u)
+    *reinterpret_cast<uint4*>(stg + r * 128 + (((u0 + u) ^ (r & 7)) << 4)) =
+        make_uint4(wm_pack_bf16x2(__uint_as_float(v[8 * u + 0]) * mul, __uint_as_float(v[8 * u + 1]) * mul),
+                   wm_pack_bf16x2(__uint_as_float(v[8 * u + 2]) * mul, __uint_as_float(v[8 * u + 3]) * mul),
+                   wm_pack_bf16x2(__uint_as_float(v[8 * u + 4]) * mul, __uint_as_float(v[8 * u + 5]) * mul),
+                   wm_pack_bf16x2(__uint_as_float(v[8 * u + 6]) * mul, __uint_as_float(v[8 * u + 7]) * mul));
+}
 
 // The k-th item of this CTA, or -1: items are numbered longest first and
 // dealt in rounds of gridDim.x, alternating direction.
@@ -233,6 +252,7 @@ template <int D>
 __global__ void __launch_bounds__(kBThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                     const BwdArgs a) {
   using C = BCfg<D>;
   constexpr int R = C::R, NB = C::kSBufKV;
@@ -267,6 +287,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(&br.acc_free[0], kEW);
     mbar_init(&br.acc_free[1], kEW);
     mbar_init(br.mma_idle, 1);
+    mbar_init(br.stg_full, kEW);
+    mbar_init(br.stg_free, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -426,6 +448,34 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint32_t lo = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t t_row = tmem + lo;
     const float sl2 = a.scale * kLog2e;
+    constexpr int STG = C::kOffStgKV;
+    // Staged output of the k-th item: wait until the previous item's TMA
+    // stores have read the staging tiles, write this thread's rows (fill),
+    // and have warp 2 store the tiles (issue) once every element-wise warp
+    // has written.  All waits are bounded.
+    auto stage_out = [&](long long k, auto fill, auto issue) -> bool {
+      uint8_t* stg = smem + STG;
+      if (k > 0) {
+        if (warp == 2) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(br.stg_free);
+        }
+        if (!wwait(br.stg_free, (k - 1) & 1)) return false;
+      }
+      fill(stg);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(br.stg_full);
+      if (warp == 2) {
+        if (!wwait(br.stg_full, k & 1)) return false;
+        if (lane == 0) {
+          issue(stg);
+          bulk_commit();
+        }
+      }
+      return true;
+    };
     uint32_t g = 0;
     bool ok = true;
     for (long long k = 0; ok; ++k) {
@@ -494,19 +544,45 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         tc_fence_after();
       }
-      // each warpgroup stores half of the columns of dV and dK
+      // each warpgroup writes half of the columns of dV and dK
       constexpr int HC = D / 2;
-      const size_t o = ((static_cast<size_t>(it.b) * a.Nkv + key) * a.Hkv + it.hkv) * D + HC * h;
-      const bool valid = key < a.Nkv;
-      store_cols<HC>(t_row + kColDV + HC * h, valid ? reinterpret_cast<__nv_bfloat16*>(a.dv) + o : nullptr, 1.f,
-                     it.steps > 0);
-      store_cols<HC>(t_row + kColDK + HC * h, valid ? reinterpret_cast<__nv_bfloat16*>(a.dk) + o : nullptr, a.scale,
-                     it.steps > 0);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&br.acc_free[0]);
+      if constexpr (C::kStage) {
+        uint32_t rv[HC], rk[HC];
+        if (it.steps > 0) {
+          tmem_ld32(t_row + kColDV + HC * h, rv);
+          tmem_ld32(t_row + kColDK + HC * h, rk);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < HC; ++i) rv[i] = rk[i] = 0u;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&br.acc_free[0]);
+        if (!stage_out(k, [&](uint8_t* stg) {
+              stage_row<HC>(stg, quarter * 32 + lane, 4 * h, rv, 1.f);
+              stage_row<HC>(stg + C::kTile, quarter * 32 + lane, 4 * h, rk, a.scale);
+            }, [&](uint8_t* stg) {
+              tma_store_4d(&tmDV, stg, 0, it.hkv, it.k0, it.b);
+              tma_store_4d(&tmDK, stg + C::kTile, 0, it.hkv, it.k0, it.b);
+            })) {
+          ok = false;
+          break;
+        }
+      } else {
+        const size_t o = ((static_cast<size_t>(it.b) * a.Nkv + key) * a.Hkv + it.hkv) * D + HC * h;
+        const bool valid = key < a.Nkv;
+        store_cols<HC>(t_row + kColDV + HC * h, valid ? reinterpret_cast<__nv_bfloat16*>(a.dv) + o : nullptr, 1.f,
+                       it.steps > 0);
+        store_cols<HC>(t_row + kColDK + HC * h, valid ? reinterpret_cast<__nv_bfloat16*>(a.dk) + o : nullptr,
+                       a.scale, it.steps > 0);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&br.acc_free[0]);
+      }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
+    if (C::kStage && warp == 2 && lane == 0) bulk_wait_all();  // stores done before the CTA retires
   }
 
   tc_fence_before();
@@ -520,7 +596,8 @@ template <int D>
 __global__ void __launch_bounds__(kBThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  const __grid_constant__ CUtensorMap tmO, const BwdArgs a) {
+                  const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmDQ,
+                  const BwdArgs a) {
   using C = BCfg<D>;
   constexpr int R = C::R, NA = C::kAccQ;
   constexpr uint32_t kColDP = 256, kColDQ = 384;
@@ -552,6 +629,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(&br.acc_free[0], kEW);
     mbar_init(&br.acc_free[1], kEW);
     mbar_init(br.mma_idle, 1);
+    mbar_init(br.stg_full, kEW);
+    mbar_init(br.stg_free, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -693,6 +772,34 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint32_t lo = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t t_row = tmem + lo;
     const float sl2 = a.scale * kLog2e;
+    constexpr int STG = C::kOffStgQ;
+    // Staged output of the k-th item: wait until the previous item's TMA
+    // stores have read the staging tiles, write this thread's rows (fill),
+    // and have warp 2 store the tiles (issue) once every element-wise warp
+    // has written.  All waits are bounded.
+    auto stage_out = [&](long long k, auto fill, auto issue) -> bool {
+      uint8_t* stg = smem + STG;
+      if (k > 0) {
+        if (warp == 2) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(br.stg_free);
+        }
+        if (!wwait(br.stg_free, (k - 1) & 1)) return false;
+      }
+      fill(stg);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(br.stg_full);
+      if (warp == 2) {
+        if (!wwait(br.stg_full, k & 1)) return false;
+        if (lane == 0) {
+          issue(stg);
+          bulk_commit();
+        }
+      }
+      return true;
+    };
     uint32_t g = 0;
     bool ok = true;
     for (long long k = 0; ok; ++k) {
@@ -785,15 +892,35 @@ __global__ void __launch_bounds__(kBThreads, 1)
         tc_fence_after();
       }
       constexpr int HC = D / 2;
-      __nv_bfloat16* dst = row < a.Nq ? reinterpret_cast<__nv_bfloat16*>(a.dq) +
-                                            ((static_cast<size_t>(it.b) * a.Nq + row) * a.Hq + it.hq) * D + HC * h
-                                      : nullptr;
-      store_cols<HC>(t_row + kColDQ + D * acc + HC * h, dst, a.scale, it.n_kv > 0);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&br.acc_free[acc]);
+      if constexpr (C::kStage) {
+        uint32_t rq[HC];
+        if (it.n_kv > 0) {
+          tmem_ld32(t_row + kColDQ + D * acc + HC * h, rq);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < HC; ++i) rq[i] = 0u;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&br.acc_free[acc]);
+        if (!stage_out(k, [&](uint8_t* stg) { stage_row<HC>(stg, r, 4 * h, rq, a.scale); },
+                       [&](uint8_t* stg) { tma_store_4d(&tmDQ, stg, 0, it.hq, it.q0, it.b); })) {
+          ok = false;
+          break;
+        }
+      } else {
+        __nv_bfloat16* dst = row < a.Nq ? reinterpret_cast<__nv_bfloat16*>(a.dq) +
+                                              ((static_cast<size_t>(it.b) * a.Nq + row) * a.Hq + it.hq) * D + HC * h
+                                        : nullptr;
+        store_cols<HC>(t_row + kColDQ + D * acc + HC * h, dst, a.scale, it.n_kv > 0);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&br.acc_free[acc]);
+      }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
+    if (C::kStage && warp == 2 && lane == 0) bulk_wait_all();  // stores done before the CTA retires
   }
 
   tc_fence_before();
@@ -816,20 +943,21 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  CUtensorMap tq, tdo, tk, tv, to;
+  CUtensorMap tq, tdo, tk, tv, to, tdq, tdk, tdv;
   if (!encode_bf16_map(&tq, a.q, a.B, a.Nq, a.Hq, D, kT) || !encode_bf16_map(&tdo, a.dout, a.B, a.Nq, a.Hq, D, kT) ||
       !encode_bf16_map(&tk, a.k, a.B, a.Nkv, a.Hkv, D, kT) || !encode_bf16_map(&tv, a.v, a.B, a.Nkv, a.Hkv, D, kT) ||
-      !encode_bf16_map(&to, a.o, a.B, a.Nq, a.Hq, D, kT))
+      !encode_bf16_map(&to, a.o, a.B, a.Nq, a.Hq, D, kT) || !encode_bf16_map(&tdq, a.dq, a.B, a.Nq, a.Hq, D, kT) ||
+      !encode_bf16_map(&tdk, a.dk, a.B, a.Nkv, a.Hkv, D, kT) || !encode_bf16_map(&tdv, a.dv, a.B, a.Nkv, a.Hkv, D, kT))
     return cudaErrorInvalidValue;
   const long long n_q = static_cast<long long>((a.Nq + kT - 1) / kT) * a.Hq * a.B;
   const long long n_kv = static_cast<long long>((a.Nkv + kT - 1) / kT) * a.Hkv * a.B;
   // The dQ kernel also writes D and lse2, which the dK/dV kernel reads.
   bwd_dq_kernel<D><<<static_cast<unsigned>(n_q < n_sm ? n_q : n_sm), kBThreads, C::kSmemQ, s>>>(tq, tdo, tk, tv, to,
-                                                                                                 a);
+                                                                                                 tdq, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bwd_dkdv_kernel<D><<<static_cast<unsigned>(n_kv < n_sm ? n_kv : n_sm), kBThreads, C::kSmemKV, s>>>(tq, tdo, tk, tv,
-                                                                                                     a);
+                                                                                                     tdk, tdv, a);
   return cudaGetLastError();
 }
 
