@@ -28,6 +28,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -106,8 +107,21 @@ def measured_peaks():
 
 
 def kernel_source_sha(fn):
-    with open(os.path.join(ROOT, "exact_io_aware_sm_b200", "csrc", fn), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of a kernel source together with the local headers it includes
+    (recursively), so that a change to a shared device helper also counts."""
+    csrc = os.path.join(ROOT, "exact_io_aware_sm_b200", "csrc")
+    h, seen, todo = hashlib.sha256(), set(), [fn]
+    while todo:
+        name = todo.pop(0)
+        path = os.path.join(csrc, name)
+        if name in seen or not os.path.exists(path):
+            continue
+        seen.add(name)
+        with open(path, "rb") as f:
+            data = f.read()
+        h.update(name.encode() + b"\0" + data)
+        todo += re.findall(r'^#include "([^"/]+)"', data.decode(), flags=re.M)
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(key):
@@ -462,12 +476,15 @@ def bench_backward(w, args, world, rank, peaks):
     flops = 2.5 * prefill_flops(w)
     tflops = whole_job_rate(flops, ms, world) / 1e12
     peak = peaks["bf16_tflops"]
+    # The kernels run seven products (S and dP in both), 3.5x the forward.
     out = {"metric": "attention backward TFLOP/s", "value": tflops, "unit": "TFLOP/s", "ms_per_step": ms,
            "config": {"workload": w["desc"] + ", backward (dQ, dK, dV)"},
            "roofline": {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
                         "frac": flops / (ms * 1e-3) / 1e12 / peak, "peak_source": f"{peaks['source']} bf16 burst",
-                        "kernel": "bwd_prep + bwd_dq + bwd_dkdv (one call)"},
-           "gpu_launches": 3 * max(5, args.steps // 2)}
+                        "executed_frac": 1.4 * flops / (ms * 1e-3) / 1e12 / peak,
+                        "kernel": "bwd_dq + bwd_dkdv (one call)",
+                        "traffic": recorded_traffic(f"backward_{args_key(w)}")},
+           "gpu_launches": 2 * max(5, args.steps // 2)}
     del tq, tk, tv, tdo, o, lse, dq, dk, dv
     torch.cuda.empty_cache()
     return out
@@ -666,6 +683,8 @@ def main():
     ap.add_argument("--workload", default="gpt2", choices=["gpt2", "long", "frame", "decode"])
     ap.add_argument("--no-extra", action="store_true", help="skip the decode / other prefill workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only attn_bwd on the chosen prefill workload (one JSON line)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -691,6 +710,20 @@ def main():
     w = WORKLOADS[args.workload]
 
     sampler = ClockSampler(torch.cuda.current_device())
+    if args.backward_only:
+        if w["mask"] not in ("none", "causal"):
+            raise SystemExit("--backward-only needs a workload without a block map")
+        with sampler:
+            d = bench_backward(w, args, world, rank, peaks)
+        if rank == 0:
+            d.update({"n_gpus": world, "steps": max(5, args.steps // 2), "warmup": args.warmup,
+                      "higher_is_better": True, "scaling": "weak",
+                      "dtype": "bf16", "data": "synthetic", "clocks": sampler.summary()})
+            print(json.dumps(d), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     if args.workload == "decode":
         with sampler:
             d = bench_decode(w, args, world, rank, peaks)

@@ -452,8 +452,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
-  a.dvec = ws->d_part;
-  a.lse2 = ws->d_part + need / 2;
+  a.neg_d = ws->d_part;
+  a.neg_lse2 = ws->d_part + need / 2;
   a.err = ws->d_err;
   a.B = B;
   a.Hq = Hq;

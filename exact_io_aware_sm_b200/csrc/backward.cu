@@ -17,8 +17,8 @@
 //                       dQ += dS K                    (TMEM x shared)
 //                     Its element-wise threads compute D from the O and dO
 //                     tiles (while dP of the first tile is on the tensor
-//                     core) and leave D and LSE*log2(e) in a scratch whose
-//                     rows are padded to whole tiles (lse2 = +inf, D = 0).
+//                     core) and leave -D and -LSE*log2(e) in a scratch whose
+//                     rows are padded to whole tiles (-inf and 0 there).
 //                     The dK/dV kernel fetches 128-row runs of both with bulk
 //                     copies on the same barrier as its Q / dO tiles.
 //   bwd_dkdv_kernel   an item is a (128-key tile, KV head, b): K and V stay
@@ -57,6 +57,7 @@
 //   dK/dV d=128: S [0,128) dP [128,256) dV [256,384) dK [384,512)
 #include <cuda_bf16.h>
 
+#include "fastmath.cuh"
 #include "kernels.h"
 #include "ptx_sm100.cuh"
 #include "warp_mma.cuh"
@@ -68,6 +69,11 @@ constexpr int kT = 128;  // rows of a Q tile, keys of a KV tile: the MMA's M
 constexpr int kBThreads = 320;
 constexpr int kEW = 8;   // element-wise warps
 constexpr float kLog2e = 1.4426950408889634f;
+// Of every 8 column pairs, this many take the polynomial 2^x on the FMA pipe
+// instead of the MUFU unit (measured: 1 at d = 64 and 2 at d = 128 were
+// best, by about 1 %; 0 to 3 all lie within 2 %).
+template <int D>
+constexpr int kPolyPairsB = D == 64 ? 1 : 2;
 
 template <int D>
 struct BCfg {
@@ -76,7 +82,7 @@ struct BCfg {
   static constexpr int kTile = NCH * kChunk;         // a 128 x D bf16 tile
   static constexpr int R = D == 64 ? 4 : 2;          // ring stages (two tiles each)
   static constexpr int kOffRing = 2 * kTile;         // after the two resident tiles
-  // dK/dV kernel: per stage lse2[128], D[128]; dQ kernel: the O tile
+  // dK/dV kernel: per stage -lse2[128], -D[128]; dQ kernel: the O tile
   static constexpr int kOffX = kOffRing + R * 2 * kTile;
   // d = 64: the gradients leave through 128-byte-swizzled staging tiles in
   // shared memory and one TMA store per tile (dV and dK, or dQ), instead of
@@ -229,20 +235,39 @@ __device__ __forceinline__ void store_cols(uint32_t t, __nv_bfloat16* dst, float
   }
 }
 
+// p = 2^(s * sl2 - lse2) for one thread's 64 columns (sr: the S values as
+// loaded from TMEM); nl(c) gives -lse2 for the columns c, c + 1.  MASK:
+// columns outside [lo, hi) are 0.
+template <int NP, bool MASK, typename NLFn>
+__device__ __forceinline__ void p_row(float* p, const uint32_t* sr, float sl2, NLFn nl, int lo, int hi) {
+  const float2 sl = make_float2(sl2, sl2);
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    float2 e = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl, nl(c));
+    if (MASK) {
+      if (c < lo || c >= hi) e.x = -INFINITY;
+      if (c + 1 < lo || c + 1 >= hi) e.y = -INFINITY;
+    }
+    const float2 v = ((c >> 1) & 7) < NP ? exp2_poly2(e) : make_float2(wm_ex2(e.x), wm_ex2(e.y));
+    p[c] = v.x;
+    p[c + 1] = v.y;
+  }
+}
+
 // dS = P * (dP - D) for one thread's 64 columns: dP read from TMEM at t_dp,
-// dS written (bf16 pairs, 32 columns) at t_ds.  dvals(c) gives D for the
+// dS written (bf16 pairs, 32 columns) at t_ds.  nd(c) gives -D for the
 // columns c, c + 1.
 template <typename DFn>
-__device__ __forceinline__ void write_ds(uint32_t t_dp, uint32_t t_ds, const float* p, DFn dvals) {
+__device__ __forceinline__ void write_ds(uint32_t t_dp, uint32_t t_ds, const float* p, DFn nd) {
   uint32_t dr[64], pk[32];
   tmem_ld32(t_dp, dr);
   tmem_ld32(t_dp + 32, dr + 32);
   tmem_wait_ld();
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
-    const float2 dd = dvals(2 * j);
-    pk[j] = wm_pack_bf16x2(p[2 * j] * (__uint_as_float(dr[2 * j]) - dd.x),
-                           p[2 * j + 1] * (__uint_as_float(dr[2 * j + 1]) - dd.y));
+    const float2 d = fadd2(make_float2(__uint_as_float(dr[2 * j]), __uint_as_float(dr[2 * j + 1])), nd(2 * j));
+    const float2 ds = fmul2(make_float2(p[2 * j], p[2 * j + 1]), d);
+    pk[j] = wm_pack_bf16x2(ds.x, ds.y);
   }
   tmem_st32(t_ds, pk);
 }
@@ -263,7 +288,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const BBars br(bar_base, R);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_base + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* vec = reinterpret_cast<float*>(smem + C::kOffX);  // [R][2][128]: lse2, D
+  float* vec = reinterpret_cast<float*>(smem + C::kOffX);  // [R][2][128]: -lse2, -D
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.Hq / a.Hkv;
@@ -351,10 +376,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
           tma_load_4d_elect(st + ch * C::kChunk, &tmQ, &br.full[s], 64 * ch, hq, qt * kT, it.b);
           tma_load_4d_elect(st + C::kTile + ch * C::kChunk, &tmDO, &br.full[s], 64 * ch, hq, qt * kT, it.b);
         }
-        // the tile's 128 lse2 and D values (padded rows: lse2 = +inf, D = 0)
+        // the tile's 128 -lse2 and -D values (padded rows: -lse2 = -inf, D = 0)
         const size_t vrow = (static_cast<size_t>(it.b) * a.Hq + hq) * nq_pad + static_cast<size_t>(qt) * kT;
-        bulk_load_elect(vec + s * 2 * kT, a.lse2 + vrow, kT * 4, &br.full[s]);
-        bulk_load_elect(vec + s * 2 * kT + kT, a.dvec + vrow, kT * 4, &br.full[s]);
+        bulk_load_elect(vec + s * 2 * kT, a.neg_lse2 + vrow, kT * 4, &br.full[s]);
+        bulk_load_elect(vec + s * 2 * kT + kT, a.neg_d + vrow, kT * 4, &br.full[s]);
       }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
@@ -500,16 +525,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
           tmem_ld32(t_s + 32, sr + 32);
           tmem_wait_ld();
           // causal: query q0 + c sees this key iff c >= key - off - q0
-          const bool masked_tile = a.causal && it.k0 + kT - 1 > q0 + off;
-          const int lim = masked_tile ? key - off - q0 : -1;
-#pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(vs + c);
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              p[c + e] = c + e < lim ? 0.f : wm_ex2(fmaf(__uint_as_float(sr[c + e]), sl2, -lv[e]));
-          }
+          auto nl = [&](int c) { return *reinterpret_cast<const float2*>(vs + c); };
+          if (a.causal && it.k0 + kT - 1 > q0 + off)
+            p_row<kPolyPairsB<D>, true>(p, sr, sl2, nl, key - off - q0, 64);
+          else
+            p_row<kPolyPairsB<D>, false>(p, sr, sl2, nl, 0, 64);
         }
         {
           uint32_t pk[32];
@@ -836,8 +856,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         if (lane == 0) mbar_arrive(br.fixed_empty);  // O and dO read
         if (h == 0) {
           const size_t vrow = (static_cast<size_t>(it.b) * a.Hq + it.hq) * nq_pad + row;
-          a.dvec[vrow] = dd;
-          a.lse2[vrow] = l2;
+          a.neg_d[vrow] = -dd;
+          a.neg_lse2[vrow] = -l2;
         }
         return true;
       };
@@ -860,8 +880,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
           tmem_ld32(t_s, sr);
           tmem_ld32(t_s + 32, sr + 32);
           tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 64; ++c) p[c] = c < lim ? wm_ex2(fmaf(__uint_as_float(sr[c]), sl2, -l2)) : 0.f;
+          auto nl = [&](int) { return make_float2(-l2, -l2); };
+          if (__any_sync(0xffffffffu, lim < 64))
+            p_row<kPolyPairsB<D>, true>(p, sr, sl2, nl, 0, lim);
+          else
+            p_row<kPolyPairsB<D>, false>(p, sr, sl2, nl, 0, 64);
         }
         // D while dP of the first tile is on the tensor core
         if (j == 0 && !compute_d()) {
@@ -873,7 +896,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
           break;
         }
         tc_fence_after();
-        write_ds(t_row + kColDP + 64 * h, t_s, p, [&](int) { return make_float2(dd, dd); });
+        write_ds(t_row + kColDP + 64 * h, t_s, p, [&](int) { return make_float2(-dd, -dd); });
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

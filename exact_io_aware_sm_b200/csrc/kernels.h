@@ -81,8 +81,8 @@ struct BwdArgs {
   void* dq;           // [B, Nq, Hq, d] (written)
   void* dk;           // [B, Nkv, Hkv, d] (written)
   void* dv;
-  float* dvec;        // scratch [B, Hq, Nq rounded up to 128]: rowsum(dO * O)
-  float* lse2;        // scratch, same layout: LSE * log2(e)
+  float* neg_d;       // scratch [B, Hq, Nq rounded up to 128]: -rowsum(dO * O)
+  float* neg_lse2;    // scratch, same layout: -LSE * log2(e)
   int* err;
   int B, Hq, Hkv, Nq, Nkv, causal;
   float scale;
