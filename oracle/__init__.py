@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.ora_count_allowed.restype = ctypes.c_longlong
         L.ora_check_schedule.argtypes = [I, P, I, I, P, I, P, I]
         L.ora_allowed.argtypes = [I, P, I, I, I, I]
+        L.ora_key_stats.argtypes = [P, I, I, I, I, I, P, P]
+        L.ora_attn_fwd_bound.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, P, P, P, D, P, P, P]
         _lib = L
     return _lib
 
@@ -213,3 +215,43 @@ def check_schedule(mask_kind, block_map, Nq, Nkv, qtiles, kvtiles):
     bm = _bm(block_map)
     return int(lib().ora_check_schedule(mask_kind, _ptr(bm), Nq, Nkv, _ptr(qt), qt.shape[0],
                                         _ptr(kt), kt.shape[0]))
+
+
+def key_stats(k):
+    """Per (b, KV head): mean key kbar [B,Hkv,d] and radius max_j ||k_j - kbar||
+    [B,Hkv] (TPU guide, step 4: mean-centring), fp64."""
+    k = np.ascontiguousarray(k)
+    B, Nkv, Hkv, d = k.shape
+    kbar = np.zeros((B, Hkv, d), np.float64)
+    radius = np.zeros((B, Hkv), np.float64)
+    if lib().ora_key_stats(_ptr(k), _dtype_code(k), B, Nkv, Hkv, d, _ptr(kbar), _ptr(radius)) != 0:
+        raise ValueError("ora_key_stats rejected its arguments")
+    return kbar, radius
+
+
+BOUND_LIMIT2 = 100.0  # a row uses the bound when 2*M*log2(e) <= this (P >= 2^-100)
+
+
+def attn_fwd_bound(q, k, v, scale, mask_kind=MASK_NONE, block_map=None, kbar=None, radius=None,
+                   limit2=BOUND_LIMIT2):
+    """Attention with the bound-based softmax (TPU guide, step 4) and a per-row
+    fallback to the exact max.  Returns (o, lse, bound_row)."""
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    B, Nq, Hq, d = q.shape
+    Nkv, Hkv = k.shape[1], k.shape[2]
+    if kbar is None or radius is None:
+        kbar, radius = key_stats(k)
+    kbar = np.ascontiguousarray(kbar, dtype=np.float64)
+    radius = np.ascontiguousarray(radius, dtype=np.float64)
+    o = np.zeros((B, Nq, Hq, d), np.float64)
+    lse = np.zeros((B, Hq, Nq), np.float64)
+    flags = np.zeros((B, Hq, Nq), np.int32)
+    bm = _bm(block_map)
+    rc = lib().ora_attn_fwd_bound(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hkv, Nq, Nkv, d, float(scale),
+                                  mask_kind, _ptr(bm), _ptr(kbar), _ptr(radius), float(limit2), _ptr(o), _ptr(lse),
+                                  _ptr(flags))
+    if rc != 0:
+        raise ValueError("ora_attn_fwd_bound rejected its arguments")
+    return o, lse, flags

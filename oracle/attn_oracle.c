@@ -30,7 +30,12 @@
  *   - a row with no allowed key has O = 0 and LSE = -inf;
  *   - LSE is the natural log-sum-exp of the scaled logits, m + ln(l);
  *   - BLOCK masks are 16x16-granular: allowed iff block_map[i/16][j/16] != 0;
- *   - the frame rule: query frame f sees key frames {0, f-1, f} (a set).
+ *   - the frame rule: query frame f sees key frames {0, f-1, f} (a set);
+ *   - bound-based softmax ("TPU attention optimisation guide", step 4): keys
+ *     are centred on the mean over all keys of their (b, KV head); a row uses
+ *     the bound where it keeps every P at or above 2^-limit2 and falls back to
+ *     its exact max otherwise (the guide checks eligibility per head; this is
+ *     the same test per row, and a head is eligible iff all its rows are).
  *
  * Inputs are read element by element and converted to double from exactly the
  * stored value (bf16 bit patterns, fp32 or fp64).
@@ -482,6 +487,118 @@ int ora_attn_bwd(const void *q, const void *k, const void *v, const void *dout, 
     free(S);
     free(P);
     free(dP);
+  }
+  return 0;
+}
+
+/*
+ * Bound-based softmax (TPU attention guide, step 4): the running max is
+ * replaced by a per-row upper bound of the scores, found from Cauchy-Schwarz
+ * after centring the keys on their mean.
+ *
+ * ora_key_stats: for every (b, hkv), kbar = (1/Nkv) sum_j k_j and
+ * radius = max_j ||k_j - kbar|| over all Nkv keys.  kbar [B,Hkv,d] fp64,
+ * radius [B,Hkv] fp64.
+ */
+int ora_key_stats(const void *k, int dtype, int B, int Nkv, int Hkv, int d, double *kbar,
+                  double *radius) {
+  if (B <= 0 || Nkv <= 0 || Hkv <= 0 || d <= 0) return -1;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hkv; ++h) {
+      double *m = kbar + ((size_t)b * Hkv + h) * d;
+      for (int t = 0; t < d; ++t) m[t] = 0.0;
+      for (int j = 0; j < Nkv; ++j)
+        for (int t = 0; t < d; ++t) m[t] += ld(k, dtype, (((size_t)b * Nkv + j) * Hkv + h) * d + t);
+      for (int t = 0; t < d; ++t) m[t] /= Nkv;
+      double r2 = 0.0;
+      for (int j = 0; j < Nkv; ++j) {
+        double s = 0.0;
+        for (int t = 0; t < d; ++t) {
+          double c = ld(k, dtype, (((size_t)b * Nkv + j) * Hkv + h) * d + t) - m[t];
+          s += c * c;
+        }
+        if (s > r2) r2 = s;
+      }
+      radius[(size_t)b * Hkv + h] = sqrt(r2);
+    }
+  return 0;
+}
+
+/*
+ * Prefill attention with the bound-based softmax.  For row i of query head
+ * hq (KV head hkv = hq / G), with centred keys k'_j = k_j - kbar:
+ *   S'_ij = scale * q_i . k'_j                (the centring shifts every score
+ *                                              of the row by the same amount)
+ *   M_i   = scale * ||q_i|| * radius          (>= S'_ij for every j)
+ *   if 2 * M_i * log2(e) <= limit2 (no P can fall below 2^-limit2, since
+ *   S'_ij >= -M_i as well): P_ij = exp(S'_ij - M_i), with no running max;
+ *   otherwise the row falls back to the exact max of its scores.
+ *   l_i = sum_j P_ij,  O_i = sum_j P_ij v_j / l_i,
+ *   LSE_i = scale * q_i . kbar + M_i + ln l_i  (the scores' own LSE).
+ * o [B,Nq,Hq,d] fp64, lse [B,Hq,Nq] fp64, bound_row [B,Hq,Nq] int32 (1 when
+ * the row used the bound, 0 for the fallback).  kbar/radius as ora_key_stats.
+ */
+int ora_attn_fwd_bound(const void *q, const void *k, const void *v, int dtype, int B, int Hq, int Hkv,
+                       int Nq, int Nkv, int d, double scale, int mask_kind, const uint8_t *block_map,
+                       const double *kbar, const double *radius, double limit2, double *o, double *lse,
+                       int32_t *bound_row) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || Nq < 0 || Nkv <= 0) return -1;
+  if (mask_kind == ORA_MASK_BLOCK && !block_map) return -1;
+  int G = Hq / Hkv;
+  long total = (long)B * Hq * Nq;
+#pragma omp parallel
+  {
+    double *P = (double *)malloc(sizeof(double) * (size_t)Nkv);
+#pragma omp for schedule(dynamic, 16)
+    for (long r = 0; r < total; ++r) {
+      int i = (int)(r % Nq);
+      int hq = (int)((r / Nq) % Hq);
+      int b = (int)(r / ((long)Nq * Hq));
+      int hkv = hq / G;
+      const double *m = kbar + ((size_t)b * Hkv + hkv) * d;
+      size_t q_off = (((size_t)b * Nq + i) * Hq + hq) * d;
+      size_t li = ((size_t)b * Hq + hq) * Nq + i;
+      double qn = 0.0, qm = 0.0;
+      for (int t = 0; t < d; ++t) {
+        double x = ld(q, dtype, q_off + t);
+        qn += x * x;
+        qm += x * m[t];
+      }
+      double M = scale * sqrt(qn) * radius[(size_t)b * Hkv + hkv];
+      int use_bound = 2.0 * M * 1.4426950408889634 <= limit2;
+      double base = M, smax = -INFINITY;
+      for (int j = 0; j < Nkv; ++j) {
+        if (!ora_allowed(mask_kind, block_map, Nq, Nkv, i, j)) {
+          P[j] = -INFINITY;
+          continue;
+        }
+        double acc = 0.0;
+        for (int t = 0; t < d; ++t)
+          acc += ld(q, dtype, q_off + t) * (ld(k, dtype, (((size_t)b * Nkv + j) * Hkv + hkv) * d + t) - m[t]);
+        P[j] = scale * acc; /* S'_ij */
+        if (P[j] > smax) smax = P[j];
+      }
+      if (!use_bound) base = smax; /* fallback: the exact max */
+      double *orow = o + q_off;
+      for (int t = 0; t < d; ++t) orow[t] = 0.0;
+      bound_row[li] = use_bound;
+      if (smax == -INFINITY) { /* no allowed key */
+        lse[li] = -INFINITY;
+        continue;
+      }
+      double l = 0.0;
+      for (int j = 0; j < Nkv; ++j) {
+        P[j] = P[j] == -INFINITY ? 0.0 : exp(P[j] - base);
+        l += P[j];
+      }
+      for (int j = 0; j < Nkv; ++j) {
+        if (P[j] == 0.0) continue;
+        for (int t = 0; t < d; ++t) orow[t] += P[j] * ld(v, dtype, (((size_t)b * Nkv + j) * Hkv + hkv) * d + t);
+      }
+      for (int t = 0; t < d; ++t) orow[t] /= l;
+      lse[li] = scale * qm + base + log(l);
+    }
+    free(P);
   }
   return 0;
 }
