@@ -490,6 +490,60 @@ def bench_backward(w, args, world, rank, peaks):
     return out
 
 
+def bench_bound(w, args, world, rank, peaks):
+    """attn_fwd_bound (bound-based softmax) on a prefill workload, next to the
+    online forward: the key statistics (attn_key_stats) and the forward are
+    timed separately, each as CUDA-graph replays with the L2 flushed between
+    steps; the rate is reported with and without the statistics."""
+    import torch
+
+    import exact_io_aware_sm_b200 as eio
+    seed = rank_seed(w["seed"], rank)
+    q, k, v = host_prefill_inputs(w, seed)
+    tq, tk, tv = (to_torch(x, "cuda") for x in (q, k, v))
+    mk, bm = mask_of(w)
+    scale = 1.0 / math.sqrt(w["d"])
+    o = torch.empty_like(tq)
+    lse = torch.empty((w["B"], w["Hq"], w["N"]), dtype=torch.float32, device="cuda")
+    kbar = torch.empty((w["B"], w["Hkv"], w["d"]), dtype=torch.float32, device="cuda")
+    radius = torch.empty((w["B"], w["Hkv"]), dtype=torch.float32, device="cuda")
+    nfb = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def stats():
+        eio.key_stats(tk, kbar, radius)
+
+    def fwd():
+        eio.attn_fwd_bound(tq, tk, tv, kbar, radius, o=o, lse=lse, scale=scale, mask_kind=mk, block_map=bm,
+                           n_fallback=nfb)
+
+    flush = make_flush()
+    steps = max(5, args.steps // 2)
+    stats()
+    time_steps(fwd, 3, args.warmup, world, flush)
+    g_stats, g_fwd = capture_graph(stats), capture_graph(fwd)
+    ms_stats, _ = time_steps(g_stats.replay, steps, args.warmup, world, flush)
+    ms_fwd, _ = time_steps(g_fwd.replay, steps, args.warmup, world, flush)
+    eio.sync_status()
+    ms_stats, ms_fwd = max_over_ranks(ms_stats, world), max_over_ranks(ms_fwd, world)
+    nfb.zero_()
+    fwd()  # one more call, to count its fallback rows
+    eio.sync_status()
+    flops = prefill_flops(w)
+    peak = peaks["bf16_tflops"]
+    out = {"metric": "prefill attn TFLOP/s (bound-based softmax)", "value": whole_job_rate(flops, ms_fwd, world) / 1e12,
+           "unit": "TFLOP/s", "ms_per_step": ms_fwd, "key_stats_ms": ms_stats,
+           "value_with_key_stats": whole_job_rate(flops, ms_fwd + ms_stats, world) / 1e12,
+           "fallback_rows": int(nfb.item()),
+           "config": {"workload": w["desc"] + ", attn_fwd_bound (key statistics precomputed)"},
+           "roofline": {"bound": "tensor", "achieved": flops / (ms_fwd * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                        "frac": flops / (ms_fwd * 1e-3) / 1e12 / peak, "peak_source": f"{peaks['source']} bf16 burst",
+                        "kernel": "prefill_bf16_kernel (bound mode)"},
+           "gpu_launches": 3 * steps}
+    del tq, tk, tv, o, lse
+    torch.cuda.empty_cache()
+    return out
+
+
 def args_key(w):
     return f"{w['mask']}_d{w['d']}_n{w['N']}"
 
@@ -685,6 +739,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only attn_bwd on the chosen prefill workload (one JSON line)")
+    ap.add_argument("--bound-only", action="store_true",
+                    help="time only attn_fwd_bound (and attn_key_stats) on the chosen prefill workload")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -710,11 +766,13 @@ def main():
     w = WORKLOADS[args.workload]
 
     sampler = ClockSampler(torch.cuda.current_device())
-    if args.backward_only:
-        if w["mask"] not in ("none", "causal"):
+    if args.backward_only or args.bound_only:
+        if args.workload == "decode":
+            raise SystemExit("--backward-only / --bound-only need a prefill workload")
+        if args.backward_only and w["mask"] not in ("none", "causal"):
             raise SystemExit("--backward-only needs a workload without a block map")
         with sampler:
-            d = bench_backward(w, args, world, rank, peaks)
+            d = (bench_backward if args.backward_only else bench_bound)(w, args, world, rank, peaks)
         if rank == 0:
             d.update({"n_gpus": world, "steps": max(5, args.steps // 2), "warmup": args.warmup,
                       "higher_is_better": True, "scaling": "weak",
@@ -746,6 +804,7 @@ def main():
             extra["decode"] = bench_decode(WORKLOADS["decode"], args, world, rank, peaks)
             if w["mask"] in ("none", "causal"):
                 extra["backward"] = bench_backward(w, args, world, rank, peaks)
+            extra["bound"] = bench_bound(w, args, world, rank, peaks)
             for name in ("long", "frame"):
                 if name == args.workload:
                     continue

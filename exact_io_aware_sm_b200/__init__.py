@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.attn_last_error_detail.argtypes = [ctypes.c_char_p, I]
         L.attn_shutdown.argtypes = []
         L.attn_debug_fault.argtypes = [I]
+        L.attn_key_stats.argtypes = [P, P, P, I, I, I, I, P]
+        L.attn_fwd_bound.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, P, P, P, P]
         L.attn_version.restype = ctypes.c_char_p
         for fn in (L.attn_fwd, L.attn_decode, L.attn_decode_multi, L.attn_bwd, L.attn_frame_block_map,
                    L.attn_classify,
@@ -125,6 +127,46 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, mask_kind=MASK_NONE, block_m
     _check(lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                           None if lse is None else lse.data_ptr(), B, Hq, Hkv, Nq, Nkv, d,
                           float(scale), mask_kind, _np_ptr(bm), dt, _stream_ptr(stream)))
+    return o, lse
+
+
+def key_stats(k, kbar=None, radius=None, stream=None):
+    """Key statistics for the bound-based softmax: kbar fp32 [B,Hkv,d] (mean
+    key) and radius fp32 [B,Hkv] (largest centred key norm) of a bf16
+    k [B,Nkv,Hkv,d] CUDA tensor."""
+    import torch
+    B, Nkv, Hkv, d = k.shape
+    if kbar is None:
+        kbar = torch.empty((B, Hkv, d), dtype=torch.float32, device=k.device)
+    if radius is None:
+        radius = torch.empty((B, Hkv), dtype=torch.float32, device=k.device)
+    _check(lib().attn_key_stats(k.data_ptr(), kbar.data_ptr(), radius.data_ptr(), B, Nkv, Hkv, d,
+                                _stream_ptr(stream)))
+    return kbar, radius
+
+
+def attn_fwd_bound(q, k, v, kbar, radius, o=None, lse=None, scale=None, mask_kind=MASK_NONE, block_map=None,
+                   n_fallback=None, stream=None):
+    """attn_fwd (bf16) with the bound-based softmax; kbar, radius from
+    key_stats(k).  n_fallback: optional int32 CUDA tensor of one element to
+    which the number of rows that kept the running max is added.
+    Returns (o, lse)."""
+    import torch
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    B, Nq, Hq, d = q.shape
+    Nkv, Hkv = k.shape[1], k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    bm = _bm(block_map)
+    _check(lib().attn_fwd_bound(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
+                                Nq, Nkv, d, float(scale), mask_kind, _np_ptr(bm), kbar.data_ptr(), radius.data_ptr(),
+                                None if n_fallback is None else n_fallback.data_ptr(), _stream_ptr(stream)))
     return o, lse
 
 

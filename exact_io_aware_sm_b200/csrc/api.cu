@@ -61,6 +61,8 @@ struct DevWs {
   int* d_err = nullptr;
   float* d_part = nullptr;
   size_t part_floats = 0;
+  float* d_stats = nullptr;  // key-statistics partial sums
+  size_t stats_floats = 0;
   std::list<DevPlan> plans;  // most recent first
 };
 
@@ -252,6 +254,56 @@ bool eio::encode_bf16_map(CUtensorMap* m, const void* base, int B, int N, int H,
   return true;
 }
 
+// The bf16 tensor-core forward; kbar != nullptr selects the bound-based
+// softmax.  Called with g_mu held and the arguments validated.
+static int fwd_bf16(DevWs& wsr, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+             int Nq, int Nkv, int d, float scale, int mask_kind, const uint8_t* block_map, const float* kbar,
+             const float* radius, int* n_fallback, cudaStream_t s) {
+  DevWs* ws = &wsr;
+  const int G = Hq / Hkv;
+  const int rows_mode = G == 1 ? 1 : 0;
+  DevPlan* pl = nullptr;
+  if (int rc = get_plan(*ws, mask_kind, block_map, Nq, Nkv, false, rows_mode, s, &pl)) return rc;
+  CUtensorMap tq, tk, tv;
+  if (int rc = make_map(&tq, q, B, Nq, Hq, d)) return rc;
+  if (int rc = make_map(&tk, k, B, Nkv, Hkv, d)) return rc;
+  if (int rc = make_map(&tv, v, B, Nkv, Hkv, d)) return rc;
+  CUtensorMap to;
+  if (!encode_bf16_map(&to, o, B, Nq, Hq, d, 16)) return ATTN_ERR_CUDA;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  PrefillArgs a{};
+  a.pairs = pl->d_pairs;
+  a.kvtiles = pl->d_pkv;
+  a.o = o;
+  a.lse = lse;
+  a.err = ws->d_err;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nkv = Nkv;
+  a.G = G;
+  a.HP = rows_mode ? 1 : (G + 1) / 2;
+  a.rows_mode = rows_mode;
+  a.n_items = static_cast<long long>(pl->n_pairs) * B * Hkv * a.HP;
+  a.num_ctas = sms > 0 ? sms : 148;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = mask_kind == ATTN_MASK_CAUSAL;
+  a.causal_off = Nkv - Nq;
+  a.stagger = pl->equal_pairs;
+  a.fault = g_fault_next;
+  g_fault_next = 0;
+  a.bound = kbar != nullptr;
+  a.q = q;
+  a.kbar = kbar;
+  a.radius = radius;
+  a.n_fallback = n_fallback;
+  cudaError_t e = launch_prefill_bf16(d, tq, tk, tv, to, a, s);
+  return e == cudaSuccess ? ATTN_OK : cuda_err(e, "prefill launch");
+}
+
 extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -305,43 +357,70 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     return e == cudaSuccess ? ATTN_OK : cuda_err(e, "fp32 prefill launch");
   }
 
-  const int G = Hq / Hkv;
-  const int rows_mode = G == 1 ? 1 : 0;
-  DevPlan* pl = nullptr;
-  if (int rc = get_plan(*ws, mask_kind, block_map, Nq, Nkv, false, rows_mode, s, &pl)) return rc;
-  CUtensorMap tq, tk, tv;
-  if (int rc = make_map(&tq, q, B, Nq, Hq, d)) return rc;
-  if (int rc = make_map(&tk, k, B, Nkv, Hkv, d)) return rc;
-  if (int rc = make_map(&tv, v, B, Nkv, Hkv, d)) return rc;
-  CUtensorMap to;
-  if (!encode_bf16_map(&to, o, B, Nq, Hq, d, 16)) return ATTN_ERR_CUDA;
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  PrefillArgs a{};
-  a.pairs = pl->d_pairs;
-  a.kvtiles = pl->d_pkv;
-  a.o = o;
-  a.lse = lse;
-  a.err = ws->d_err;
+  return fwd_bf16(*ws, q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, mask_kind, block_map, nullptr, nullptr, nullptr,
+                  s);
+}
+
+int attn_key_stats(const void* k, float* kbar, float* radius, int B, int Nkv, int Hkv, int d, void* stream) {
+  if (!k || !kbar || !radius) return set_err(ATTN_ERR_NULL, "k, kbar and radius must be non-NULL");
+  if (B < 1 || Nkv < 1 || Hkv < 1) return set_err(ATTN_ERR_SHAPE, "B, Nkv, Hkv must be >= 1");
+  if (d != 64 && d != 128) return set_err(ATTN_ERR_UNSUPPORTED, "attn_key_stats needs d in {64, 128}");
+  if (B > 65535 || Hkv > 65535 || static_cast<long long>(B) * Nkv * Hkv >= (1ll << 31))
+    return set_err(ATTN_ERR_SHAPE, "too many keys");
+  if (!aligned16(k) || !aligned16(kbar) || (reinterpret_cast<uintptr_t>(radius) & 3u))
+    return set_err(ATTN_ERR_ALIGN, "k and kbar must be 16-byte aligned, radius 4-byte aligned");
+  if (int rc = check_device_sm100()) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevWs* ws;
+  if (int rc = get_ws(&ws)) return rc;
+  const int nsplit = key_stats_splits(Nkv);
+  const size_t need = static_cast<size_t>(B) * Hkv * nsplit * d;
+  if (ws->stats_floats < need) {
+    cudaDeviceSynchronize();
+    cudaFree(ws->d_stats);
+    ws->d_stats = nullptr;
+    ws->stats_floats = 0;
+    cudaError_t e = cudaMalloc(&ws->d_stats, need * sizeof(float));
+    if (e != cudaSuccess) return set_err(ATTN_ERR_WORKSPACE, "key statistics scratch: %s", cudaGetErrorString(e));
+    ws->stats_floats = need;
+  }
+  KeyStatsArgs a{};
+  a.k = k;
+  a.part = ws->d_stats;
+  a.kbar = kbar;
+  a.radius = radius;
   a.B = B;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.Nq = Nq;
   a.Nkv = Nkv;
-  a.G = G;
-  a.HP = rows_mode ? 1 : (G + 1) / 2;
-  a.rows_mode = rows_mode;
-  a.n_items = static_cast<long long>(pl->n_pairs) * B * Hkv * a.HP;
-  a.num_ctas = sms > 0 ? sms : 148;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.causal = mask_kind == ATTN_MASK_CAUSAL;
-  a.causal_off = Nkv - Nq;
-  a.stagger = pl->equal_pairs;
-  a.fault = g_fault_next;
-  g_fault_next = 0;
-  cudaError_t e = launch_prefill_bf16(d, tq, tk, tv, to, a, s);
-  return e == cudaSuccess ? ATTN_OK : cuda_err(e, "prefill launch");
+  a.Hkv = Hkv;
+  a.nsplit = nsplit;
+  cudaError_t e = launch_key_stats(d, a, s);
+  return e == cudaSuccess ? ATTN_OK : cuda_err(e, "key statistics launch");
+}
+
+int attn_fwd_bound(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                   int Nkv, int d, float scale, int mask_kind, const uint8_t* block_map, const float* kbar,
+                   const float* radius, int* n_fallback, void* stream) {
+  if (!q || !k || !v || !o || !kbar || !radius)
+    return set_err(ATTN_ERR_NULL, "q, k, v, o, kbar and radius must be non-NULL");
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nkv < 1)
+    return set_err(ATTN_ERR_SHAPE, "B, Hq, Hkv, Nq, Nkv must be >= 1");
+  if (Hq % Hkv != 0) return set_err(ATTN_ERR_SHAPE, "Hq (%d) is not a multiple of Hkv (%d)", Hq, Hkv);
+  if (!(scale > 0.f) || !std::isfinite(scale))
+    return set_err(ATTN_ERR_SHAPE, "scale must be positive and finite");
+  if (int rc = check_mask_args(mask_kind, block_map)) return rc;
+  if (d != 64 && d != 128) return set_err(ATTN_ERR_UNSUPPORTED, "attn_fwd_bound needs d in {64, 128}");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)) ||
+      !aligned16(kbar) || (reinterpret_cast<uintptr_t>(radius) & 3u) ||
+      (reinterpret_cast<uintptr_t>(n_fallback) & 3u))
+    return set_err(ATTN_ERR_ALIGN, "device pointers must be 16-byte aligned (radius, n_fallback: 4-byte)");
+  if (int rc = check_device_sm100()) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevWs* ws;
+  if (int rc = get_ws(&ws)) return rc;
+  return fwd_bf16(*ws, q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, mask_kind, block_map, kbar, radius,
+                  n_fallback, s);
 }
 
 int attn_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
@@ -544,6 +623,7 @@ int attn_shutdown(void) {
     cudaDeviceSynchronize();
     for (auto& p : kv.second.plans) free_plan(p);
     cudaFree(kv.second.d_part);
+    cudaFree(kv.second.d_stats);
     cudaFree(kv.second.d_err);
   }
   g_ws.clear();

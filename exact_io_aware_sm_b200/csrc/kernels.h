@@ -28,7 +28,25 @@ struct PrefillArgs {
   int causal, causal_off;
   int stagger;          // 1: both slots of every pair visit the same number of KV tiles
   int fault;            // test hook: 1 = CTA 0 skips its first K load (a wait then runs out)
+  // Bound-based softmax (bound = 1): each row's exponent base is
+  // scale*log2(e)*(q.kbar + ||q|| radius) instead of the running max.
+  int bound;
+  const void* q;        // [B, Nq, Hq, d] bf16 (read for the row norms)
+  const float* kbar;    // [B, Hkv, d]
+  const float* radius;  // [B, Hkv]
+  int* n_fallback;      // rows that kept the running max are added here (may be null)
 };
+
+// Key statistics for the bound-based softmax.
+struct KeyStatsArgs {
+  const void* k;  // [B, Nkv, Hkv, d] bf16
+  float* part;    // scratch [B, Hkv, nsplit, d]
+  float* kbar;    // [B, Hkv, d] (written)
+  float* radius;  // [B, Hkv] (written)
+  int B, Nkv, Hkv, nsplit;
+};
+int key_stats_splits(int Nkv);
+cudaError_t launch_key_stats(int d, const KeyStatsArgs& a, cudaStream_t s);
 
 // bf16 tensor-core prefill (tcgen05 / TMA).  d in {64, 128}.
 // to: O as {d, Hq, Nq, B} with a {64, 1, 16, 1} box (used by the d = 64 epilogue).

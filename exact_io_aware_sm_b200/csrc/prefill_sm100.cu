@@ -56,6 +56,9 @@ constexpr int kRegsSoftmax = 216;  // warpgroups 1 and 2
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
               "register split must fit in the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Bound-based softmax: a row keeps the bound as its base only if no P can fall
+// below 2^-kBoundLimit2 (every centred score lies within +-bound).
+constexpr float kBoundLimit2 = 100.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
@@ -96,6 +99,44 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Bound-based softmax ("TPU attention optimisation guide", step 4): the
+// exponent base of a row, in log2 units, from the Cauchy-Schwarz bound on its
+// centred scores, q . (k_j - kbar) <= ||q|| radius:
+//   base = scale*log2(e) * (q . kbar + ||q|| radius).
+// The centring only shifts all scores of the row by q . kbar, so P, O and the
+// LSE are those of the plain definition.  Returns false (base untouched) when
+// 2 * scale*log2(e) * ||q|| radius exceeds kBoundLimit2, where the row keeps
+// the running max.  Rows past the tile's valid rows take base 0: their
+// results are discarded.
+template <int D>
+__device__ __forceinline__ bool bound_base(const PrefillArgs& a, int b, int head, int hkv, int grow, bool valid,
+                                           float sl2, float* base) {
+  if (!valid) {
+    *base = 0.f;
+    return true;
+  }
+  const uint4* qr = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.q) +
+                                                   ((static_cast<size_t>(b) * a.Nq + grow) * a.Hq + head) * D);
+  const float4* kb = reinterpret_cast<const float4*>(a.kbar + (static_cast<size_t>(b) * a.Hkv + hkv) * D);
+  float qk = 0.f, qq = 0.f;
+#pragma unroll 4
+  for (int e = 0; e < D / 8; ++e) {
+    const uint4 u = qr[e];
+    const float4 k0 = kb[2 * e], k1 = kb[2 * e + 1];
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
+    const float2 f2 = __bfloat1622float2(h2[2]), f3 = __bfloat1622float2(h2[3]);
+    qk = fmaf(f0.x, k0.x, fmaf(f0.y, k0.y, fmaf(f1.x, k0.z, fmaf(f1.y, k0.w, qk))));
+    qk = fmaf(f2.x, k1.x, fmaf(f2.y, k1.y, fmaf(f3.x, k1.z, fmaf(f3.y, k1.w, qk))));
+    qq = fmaf(f0.x, f0.x, fmaf(f0.y, f0.y, fmaf(f1.x, f1.x, fmaf(f1.y, f1.y, qq))));
+    qq = fmaf(f2.x, f2.x, fmaf(f2.y, f2.y, fmaf(f3.x, f3.x, fmaf(f3.y, f3.y, qq))));
+  }
+  const float m = sl2 * sqrtf(qq) * a.radius[static_cast<size_t>(b) * a.Hkv + hkv];
+  if (!(2.f * m <= kBoundLimit2)) return false;
+  *base = fmaf(sl2, qk, m);
+  return true;
 }
 
 // One work item, decoded identically by every role.
@@ -152,7 +193,8 @@ constexpr bool kFirstLoadsFirst = true;
 
 // STAGGER: both slots of every pair visit the same number of KV tiles, and
 // slot A starts each item after slot B's first exponentials (see below).
-template <int D, bool STAGGER>
+// BOUND: the bound-based softmax (see bound_base).
+template <int D, bool STAGGER, bool BOUND>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -441,6 +483,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // exponentials of its first tile.  Done when both slots of every pair
       // visit the same number of KV tiles (GQA head pairs, Q tiles inside one
       // frame); the offset then persists through the item.
+      const int grow = row0 + row;
+      float m_b = -INFINITY;  // exponent base, log2 units
+      // Bound-based softmax: rows with a fixed base skip the max; a warp whose
+      // rows all have one skips the row-max reduction entirely.  (Computed
+      // before the slot offset below, so that its loads overlap that wait.)
+      bool fixed = false;
+      if constexpr (BOUND) {
+        fixed = bound_base<D>(a, it.b, head, it.hkv, grow, row < nrows, sl2, &m_b);
+        const unsigned fb = __ballot_sync(0xffffffffu, !fixed);
+        if (lane == 0 && fb != 0u && a.n_fallback != nullptr) atomicAdd(a.n_fallback, __popc(fb));
+      }
+      const bool skip_max = BOUND && __all_sync(0xffffffffu, fixed);
       const bool stagger = STAGGER && it.nA > 0;
       if (stagger && x == 0) {
         if (!warp_wait(b_first, bcnt & 1)) {
@@ -449,9 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (stagger) bcnt++;
-      const int grow = row0 + row;
       const int4* kv = a.kvtiles + it.kv_first;
-      float m_b = -INFINITY;  // exponent base, log2 units
       float l = 0.f;
 
       for (int t = 0; t < nX; ++t) {
@@ -484,17 +536,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
         }
         // Row max: four independent chains of 3-input max.
-        float mx4[4];
+        float mx_s = -INFINITY;
+        if (!BOUND || !skip_max) {
+          float mx4[4];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          float m = __uint_as_float(sr[q4 * 32]);
+          for (int q4 = 0; q4 < 4; ++q4) {
+            float m = __uint_as_float(sr[q4 * 32]);
 #pragma unroll
-          for (int c = 1; c < 31; c += 2)
-            m = max3f(m, __uint_as_float(sr[q4 * 32 + c]), __uint_as_float(sr[q4 * 32 + c + 1]));
-          mx4[q4] = fmaxf(m, __uint_as_float(sr[q4 * 32 + 31]));
+            for (int c = 1; c < 31; c += 2)
+              m = max3f(m, __uint_as_float(sr[q4 * 32 + c]), __uint_as_float(sr[q4 * 32 + c + 1]));
+            mx4[q4] = fmaxf(m, __uint_as_float(sr[q4 * 32 + 31]));
+          }
+          mx_s = max3f(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * sl2;
         }
-        const float mx_s = max3f(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * sl2;
-        const bool upd = mx_s > m_b + kRescaleThreshold;
+        const bool upd = (!BOUND || !fixed) && mx_s > m_b + kRescaleThreshold;
         const float alpha = upd ? ex2(m_b - mx_s) : 1.f;  // 0 when m_b was -inf
         if (upd) m_b = mx_s;
         const float base = m_b == -INFINITY ? 0.f : m_b;
@@ -641,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D, bool STAGGER>
+template <int D, bool STAGGER, bool BOUND>
 cudaError_t launch_ds(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const CUtensorMap& to, const PrefillArgs& a, cudaStream_t s) {
   static int attr_dev = -1;
@@ -651,17 +706,17 @@ cudaError_t launch_ds(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
     // The warpgroup register split is only safe when every thread starts with
     // exactly kLaunchRegs registers.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, prefill_bf16_kernel<D, STAGGER>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, prefill_bf16_kernel<D, STAGGER, BOUND>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kLaunchRegs || fa.maxThreadsPerBlock < kThreads) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(prefill_bf16_kernel<D, STAGGER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(prefill_bf16_kernel<D, STAGGER, BOUND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg<D>::kSmem);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
   if (a.n_items == 0) return cudaSuccess;
   const long long grid = a.n_items < a.num_ctas ? a.n_items : a.num_ctas;
-  prefill_bf16_kernel<D, STAGGER>
+  prefill_bf16_kernel<D, STAGGER, BOUND>
       <<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmem, s>>>(tq, tk, tv, to, a);
   return cudaGetLastError();
 }
@@ -669,7 +724,9 @@ cudaError_t launch_ds(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& to, const PrefillArgs& a, cudaStream_t s) {
-  return a.stagger ? launch_ds<D, true>(tq, tk, tv, to, a, s) : launch_ds<D, false>(tq, tk, tv, to, a, s);
+  if (a.bound)
+    return a.stagger ? launch_ds<D, true, true>(tq, tk, tv, to, a, s) : launch_ds<D, false, true>(tq, tk, tv, to, a, s);
+  return a.stagger ? launch_ds<D, true, false>(tq, tk, tv, to, a, s) : launch_ds<D, false, false>(tq, tk, tv, to, a, s);
 }
 
 }  // namespace

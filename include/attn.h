@@ -35,9 +35,11 @@
  *     [0, Lmax]) are latched in a device word and returned by a later
  *     attn_sync_status().
  *   - Workspace: the library owns a per-device workspace (tile schedules,
- *     split-KV partials, error word).  It grows on demand with cudaMalloc and
- *     is released by attn_shutdown().  A call that must grow it synchronises
- *     the device.
+ *     split-KV partials, backward and key-statistics scratch, error word).
+ *     It grows on demand with cudaMalloc and is released by attn_shutdown().
+ *     A call that must grow it synchronises the device.  Calls that use the
+ *     same scratch (decode, backward; key statistics) must not run
+ *     concurrently on different streams: order them.
  *   - Masks.  NONE: every key allowed.  CAUSAL: key j allowed for query i iff
  *     j <= i + (Nkv - Nq) (bottom-right alignment).  BLOCK: allowed iff
  *     block_map[i/16][j/16] != 0, a host uint8 array of
@@ -256,7 +258,7 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
  *   dk, dv      device, [B, Nkv, Hkv, d] bf16 (written)
  *   mask_kind   ATTN_MASK_NONE or ATTN_MASK_CAUSAL (as attn_fwd)
  * Limits: d == 64 or 128; all pointers 16-byte aligned.
- * Scratch: 2*B*Hq*Nq floats of library workspace.
+ * Scratch: 2*B*Hq*ceil(Nq/128)*128 floats of library workspace.
  * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED (other masks or d), CUDA, WORKSPACE;
  * a bounded wait that runs out latches ATTN_ERR_DEVICE_TIMEOUT.
  */
@@ -277,6 +279,46 @@ int attn_debug_fault(int kind);
 
 /* Library version string, e.g. "exact_io_aware_sm_b200 0.1". */
 const char* attn_version(void);
+
+/*
+ * attn_key_stats -- key statistics for the bound-based softmax.
+ *
+ * Passage: "TPU attention optimisation guide: collective overlap and mask
+ * removal, verified by trace", step 4: centring the keys on their mean leaves
+ * the softmax unchanged and tightens the Cauchy-Schwarz bound of the scores.
+ *
+ *   k       device, [B, Nkv, Hkv, d] bf16
+ *   kbar    device, fp32 [B, Hkv, d] (written): mean of the Nkv keys of each
+ *           (b, KV head)
+ *   radius  device, fp32 [B, Hkv] (written): max_j ||k_j - kbar||
+ * Limits: d == 64 or 128; B*Nkv*Hkv < 2^31; k and kbar 16-byte aligned,
+ * radius 4-byte aligned.
+ * Scratch: B*Hkv*ceil(Nkv/128)*d floats of library workspace.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, CUDA, WORKSPACE.
+ */
+int attn_key_stats(const void* k, float* kbar, float* radius, int B, int Nkv, int Hkv, int d, void* stream);
+
+/*
+ * attn_fwd_bound -- attn_fwd (bf16) with the bound-based softmax.
+ *
+ * Passage: the TPU guide, step 4: each row's running max is replaced by an
+ * upper bound of its scores, scale*(q.kbar + ||q||*radius) (Cauchy-Schwarz on
+ * the centred keys), so no row max is taken and nothing is rescaled; a row
+ * whose bound could push a probability below 2^-100 (2*scale*log2(e)*
+ * ||q||*radius > 100) falls back to the running max.  The guide checks this
+ * per head; here it is checked per row (a head qualifies iff all its rows do).
+ * O and LSE are those of attn_fwd up to rounding.
+ *
+ *   q, k, v, o, lse, sizes, scale, mask_kind, block_map: as attn_fwd
+ *   kbar, radius  device, from attn_key_stats on the same k
+ *   n_fallback    device int32 (may be NULL): the number of rows that kept
+ *                 the running max is added to it
+ * Limits: d == 64 or 128; as attn_fwd otherwise.
+ * Errors: as attn_fwd.
+ */
+int attn_fwd_bound(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                   int Nkv, int d, float scale, int mask_kind, const uint8_t* block_map, const float* kbar,
+                   const float* radius, int* n_fallback, void* stream);
 
 #ifdef __cplusplus
 }

@@ -461,3 +461,83 @@ def test_constant_v_rows():
     cf = synthetic.bf16_bits_to_f32(c).astype(np.float64)
     err = np.abs(host_f64(o) - cf).max()
     assert err <= 8e-3 * max(1.0, np.abs(cf).max())
+
+
+# ------------------------------------------------------- bound-based softmax
+BOUND_CASES = [
+    # B, Hq, Hkv, Nq, Nkv, d, kind
+    (2, 4, 2, 300, 300, 64, eio.MASK_CAUSAL),
+    (1, 8, 2, 257, 513, 128, eio.MASK_NONE),
+    (1, 4, 4, 200, 200, 64, eio.MASK_BLOCK),
+    (1, 2, 1, 130, 77, 128, eio.MASK_CAUSAL),  # rows that see no key
+]
+
+
+@pytest.mark.parametrize("case", BOUND_CASES)
+def test_key_stats_and_bound_forward(case):
+    B, Hq, Hkv, Nq, Nkv, d, kind = case
+    seed = 3300 + BOUND_CASES.index(case)
+    q, k, v = make_inputs(seed, B, Hq, Hkv, Nq, Nkv, d)
+    # an offset on the keys, so that the centring matters
+    kf = synthetic.bf16_bits_to_f32(k) + np.float32(0.75)
+    k = synthetic.f32_to_bf16_bits(kf)
+    bm = random_block_map(seed, Nq, Nkv) if kind == eio.MASK_BLOCK else None
+    scale = 1 / math.sqrt(d)
+    tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    kbar, radius = eio.key_stats(tk)
+    rk, rr = oracle.key_stats(k)
+    np.testing.assert_allclose(kbar.cpu().numpy(), rk, atol=2e-5, rtol=1e-5)
+    np.testing.assert_allclose(radius.cpu().numpy(), rr, rtol=1e-5)
+    nfb = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = eio.attn_fwd_bound(tq, tk, tv, kbar, radius, scale=scale, mask_kind=kind, block_map=bm, n_fallback=nfb)
+    eio.sync_status()
+    ro, rlse = oracle.attn_fwd(q, k, v, scale, kind, bm)
+    check(o, lse, ro, rlse, f"bound {case}")
+    _, _, flags = oracle.attn_fwd_bound(q, k, v, scale, kind, bm)
+    assert int(nfb.item()) == int((flags == 0).sum()) == 0
+
+
+def test_bound_forward_falls_back_on_long_queries():
+    """Every fifth query 40x longer: those rows' bounds exceed the limit and
+    keep the running max; the count matches the oracle's and O is exact."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 320, 64
+    q, k, v = make_inputs(3350, B, Hq, Hkv, N, N, d)
+    qf = synthetic.bf16_bits_to_f32(q)
+    qf[:, ::5] *= np.float32(40.0)
+    q = synthetic.f32_to_bf16_bits(qf)
+    scale = 1 / math.sqrt(d)
+    tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    kbar, radius = eio.key_stats(tk)
+    nfb = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = eio.attn_fwd_bound(tq, tk, tv, kbar, radius, scale=scale, mask_kind=eio.MASK_CAUSAL, n_fallback=nfb)
+    eio.sync_status()
+    ro, rlse, flags = oracle.attn_fwd_bound(q, k, v, scale, oracle.MASK_CAUSAL)
+    # the decision is far from the limit on both sides (about 32 and 1270 log2 units)
+    assert int(nfb.item()) == int((flags == 0).sum()) == B * Hq * (N // 5)
+    rq = oracle.attn_fwd(q, k, v, scale, oracle.MASK_CAUSAL)
+    np.testing.assert_allclose(ro, rq[0], atol=1e-10)
+    # long rows have sharp softmaxes: compare with the forward tolerance
+    check(o, lse, ro, rlse, "bound with fallback rows")
+
+
+def test_bound_forward_matches_online_forward_gpt2_shape():
+    """The similarity band between the bound-based and the online forward on
+    the GPT-2 workload shape: same result up to rounding."""
+    B, H, N, d = 8, 12, 1024, 64
+    q, k, v = make_inputs(1002, B, H, H, N, N, d)
+    tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    o0, l0 = eio.attn_fwd(tq, tk, tv, mask_kind=eio.MASK_CAUSAL)
+    kbar, radius = eio.key_stats(tk)
+    nfb = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o1, l1 = eio.attn_fwd_bound(tq, tk, tv, kbar, radius, mask_kind=eio.MASK_CAUSAL, n_fallback=nfb)
+    eio.sync_status()
+    assert int(nfb.item()) == 0
+    a, b = o0.float(), o1.float()
+    assert (a - b).abs().max().item() <= 2e-2
+    cos = torch.nn.functional.cosine_similarity(a.reshape(-1, d), b.reshape(-1, d), dim=1)
+    assert cos.min().item() > 0.9999
+    assert (l0 - l1).abs().max().item() <= 1e-3
+    rows = np.array([[0, 0, 0], [3, 7, 511], [7, 11, 1023], [5, 2, 1]], np.int32)
+    ro, rlse = oracle.attn_rows(q, k, v, 1 / math.sqrt(d), rows, oracle.MASK_CAUSAL)
+    got = np.stack([host_f64(o1[b_, i, h]) for b_, h, i in rows])
+    assert np.abs(got - ro).max() <= O_MAX
