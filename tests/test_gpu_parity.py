@@ -541,3 +541,15 @@ def test_bound_forward_matches_online_forward_gpt2_shape():
     ro, rlse = oracle.attn_rows(q, k, v, 1 / math.sqrt(d), rows, oracle.MASK_CAUSAL)
     got = np.stack([host_f64(o1[b_, i, h]) for b_, h, i in rows])
     assert np.abs(got - ro).max() <= O_MAX
+
+
+def test_ulysses_single_rank_uses_the_cuda_forward():
+    """Without a process group (one rank) the Ulysses entry is the CUDA
+    forward itself: bit-identical to attn_fwd."""
+    from exact_io_aware_sm_b200.ulysses import ulysses_attention
+    q, k, v = make_inputs(3400, 1, 4, 2, 200, 200, 64)
+    tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    o0, l0 = eio.attn_fwd(tq, tk, tv, mask_kind=eio.MASK_CAUSAL)
+    o1, l1 = ulysses_attention(tq, tk, tv, mask_kind=eio.MASK_CAUSAL)
+    eio.sync_status()
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)

@@ -1,0 +1,134 @@
+"""Ulysses sequence parallelism on CPU ranks (gloo).
+
+Each rank holds a slice of the sequence; the module swaps sequence shards for
+head shards with all-to-alls, runs attention on whole sequences for its heads
+and swaps back.  With the fp64 oracle as the attention (test infrastructure
+only), the result gathered over the ranks must equal the oracle on the whole,
+unsharded tensors: the exchange is pure data movement, so the comparison is
+exact up to the oracle's own rounding.
+"""
+import math
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _oracle_attention(q, k, v, mask_kind, scale):
+    import oracle
+    o, lse = oracle.attn_fwd(q.numpy(), k.numpy(), v.numpy(), scale, mask_kind)
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def _inputs(B, N, Hq, Hkv, d):
+    rng = np.random.default_rng(77)
+    q = rng.standard_normal((B, N, Hq, d))
+    k = rng.standard_normal((B, N, Hkv, d))
+    v = rng.standard_normal((B, N, Hkv, d))
+    return q, k, v
+
+
+def _rank_main(rank, world, port, shape, mask_kind, groups, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+
+    from exact_io_aware_sm_b200.ulysses import ulysses_attention
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, N, Hq, Hkv, d = shape
+        q, k, v = _inputs(B, N, Hq, Hkv, d)
+        Nl = N // world
+        sl = slice(rank * Nl, (rank + 1) * Nl)
+        tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x[:, sl])) for x in (q, k, v))
+        o, lse = ulysses_attention(tq, tk, tv, mask_kind=mask_kind, scale=1 / math.sqrt(d), head_groups=groups,
+                                   attention=_oracle_attention)
+        out_q.put((rank, o.numpy(), lse.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(world, shape, mask_kind, groups):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, shape, mask_kind, groups, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict()
+    for _ in range(world):
+        r, o, lse = q.get(timeout=180)
+        got[r] = (o, lse)
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    o = np.concatenate([got[r][0] for r in range(world)], axis=1)
+    lse = np.concatenate([got[r][1] for r in range(world)], axis=2)
+    return o, lse
+
+
+@pytest.mark.parametrize("world,shape,mask_kind,groups", [
+    (2, (1, 64, 4, 2, 8), 1, 1),   # causal, GQA (2 query heads per KV head)
+    (2, (2, 48, 8, 4, 16), 0, 2),  # two head groups, each with its own exchanges
+    (4, (1, 64, 8, 4, 8), 1, 1),   # four ranks
+])
+def test_ulysses_equals_unsharded_attention(world, shape, mask_kind, groups):
+    import oracle
+    B, N, Hq, Hkv, d = shape
+    o, lse = _run(world, shape, mask_kind, groups)
+    q, k, v = _inputs(B, N, Hq, Hkv, d)
+    ro, rlse = oracle.attn_fwd(q, k, v, 1 / math.sqrt(d), mask_kind)
+    np.testing.assert_allclose(o, ro, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(lse, rlse, atol=1e-13, rtol=0)
+
+
+def test_layout_helpers_round_trip():
+    """The send buffer of head group g for rank i holds exactly rank i's heads
+    of that group; reassembling the received chunks restores the rows."""
+    from exact_io_aware_sm_b200.ulysses import _from_seq, _to_heads
+    B, Nl, H, d, P, ng = 2, 3, 8, 4, 2, 2
+    x = torch.arange(B * Nl * H * d, dtype=torch.float64).view(B, Nl, H, d)
+    for g in range(ng):
+        buf = _to_heads(x, P, g, ng)
+        assert buf.shape == (P, B, Nl, H // P // ng, d)
+        for i in range(P):
+            h0 = i * (H // P) + g * (H // P // ng)
+            assert torch.equal(buf[i], x[:, :, h0:h0 + H // P // ng])
+    # as if every rank sent this same buffer: rows of rank j land at j*Nl
+    buf = _to_heads(x, P, 0, 1)
+    whole = _from_seq(buf)
+    assert whole.shape == (B, P * Nl, H // P, d)
+    assert torch.equal(whole[:, Nl:2 * Nl], x[:, :, H // P:2 * (H // P)])
+
+
+def test_argument_checks():
+    from exact_io_aware_sm_b200.ulysses import _check
+    with pytest.raises(ValueError):
+        _check(1, 8, 6, 3, 4, 1)   # heads not divisible by the world size
+    with pytest.raises(ValueError):
+        _check(1, 8, 8, 4, 2, 4)   # Hkv/P = 2 not a multiple of 4 head groups
+    _check(1, 8, 8, 4, 2, 2)
+
+
+def test_single_rank_is_the_plain_call():
+    from exact_io_aware_sm_b200.ulysses import ulysses_attention
+    q, k, v = (torch.from_numpy(x) for x in _inputs(1, 16, 2, 1, 4))
+    calls = []
+
+    def att(q_, k_, v_, mk, sc):
+        calls.append(q_.shape)
+        return _oracle_attention(q_, k_, v_, mk, sc)
+    o, lse = ulysses_attention(q, k, v, mask_kind=1, attention=att)
+    assert calls == [q.shape]
