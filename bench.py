@@ -457,15 +457,16 @@ def bench_backward(w, args, world, rank, peaks):
     q, k, v = host_prefill_inputs(w, seed)
     dout = synthetic.tensor(seed, 9, q.shape, w["dtype"])
     tq, tk, tv, tdo = (to_torch(x, "cuda") for x in (q, k, v, dout))
-    mk, _ = mask_of(w)
+    mk, bm = mask_of(w)
+    bm_ptr = None if bm is None else bm.ctypes.data
     scale = 1.0 / math.sqrt(w["d"])
-    o, lse = eio.attn_fwd(tq, tk, tv, scale=scale, mask_kind=mk)
+    o, lse = eio.attn_fwd(tq, tk, tv, scale=scale, mask_kind=mk, block_map=bm)
     dq, dk, dv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
 
     def step():
         eio.lib().attn_bwd(tq.data_ptr(), tk.data_ptr(), tv.data_ptr(), o.data_ptr(), lse.data_ptr(),
                            tdo.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), w["B"], w["Hq"], w["Hkv"],
-                           w["N"], w["N"], w["d"], scale, mk, torch.cuda.current_stream().cuda_stream)
+                           w["N"], w["N"], w["d"], scale, mk, bm_ptr, torch.cuda.current_stream().cuda_stream)
 
     flush = make_flush()
     time_steps(step, 3, args.warmup, world, flush)
@@ -769,8 +770,6 @@ def main():
     if args.backward_only or args.bound_only:
         if args.workload == "decode":
             raise SystemExit("--backward-only / --bound-only need a prefill workload")
-        if args.backward_only and w["mask"] not in ("none", "causal"):
-            raise SystemExit("--backward-only needs a workload without a block map")
         with sampler:
             d = (bench_backward if args.backward_only else bench_bound)(w, args, world, rank, peaks)
         if rank == 0:
@@ -802,8 +801,7 @@ def main():
         extra = {}
         if not args.no_extra:
             extra["decode"] = bench_decode(WORKLOADS["decode"], args, world, rank, peaks)
-            if w["mask"] in ("none", "causal"):
-                extra["backward"] = bench_backward(w, args, world, rank, peaks)
+            extra["backward"] = bench_backward(w, args, world, rank, peaks)
             extra["bound"] = bench_bound(w, args, world, rank, peaks)
             for name in ("long", "frame"):
                 if name == args.workload:

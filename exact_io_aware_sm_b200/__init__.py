@@ -54,7 +54,7 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, I, P]
         L.attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P]
         L.attn_decode_multi.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
-        L.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+        L.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, P]
         L.attn_frame_block_map.argtypes = [I, I, P]
         L.attn_classify.argtypes = [I, P, I, I, I, I, P]
         L.attn_plan.argtypes = [I, P, I, I, P, I, P, I, P, P]
@@ -209,9 +209,10 @@ def attn_decode_multi(q, k_cache, v_cache, seqlens, o=None, lse=None, scale=None
     return o, lse
 
 
-def attn_bwd(q, k, v, o, lse, dout, scale=None, mask_kind=MASK_NONE, stream=None):
+def attn_bwd(q, k, v, o, lse, dout, scale=None, mask_kind=MASK_NONE, block_map=None, stream=None):
     """Gradients of attn_fwd (bf16): q, o, dout [B,Nq,Hq,d]; k, v [B,Nkv,Hkv,d];
-    lse [B,Hq,Nq] fp32 from the forward.  Returns (dq, dk, dv) like q, k, v."""
+    lse [B,Hq,Nq] fp32 from the forward; the mask as for attn_fwd.
+    Returns (dq, dk, dv) like q, k, v."""
     import torch
     for t in (q, k, v, o, dout):
         if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
@@ -221,9 +222,10 @@ def attn_bwd(q, k, v, o, lse, dout, scale=None, mask_kind=MASK_NONE, stream=None
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bm = _bm(block_map)
     _check(lib().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nkv, d, float(scale),
-                          mask_kind, _stream_ptr(stream)))
+                          mask_kind, _np_ptr(bm), _stream_ptr(stream)))
     return dq, dk, dv
 
 

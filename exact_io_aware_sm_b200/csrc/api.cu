@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -57,6 +58,31 @@ struct DevPlan {
   int4* d_pkv = nullptr;
 };
 
+// Backward tile lists under a BLOCK mask: for every 128-row Q tile the live
+// 128-key tiles, and for every key tile the live Q tiles, each entry with the
+// 8 x 8 bitmap of its 16 x 16 blocks; visit orders longest list first.
+struct BwdPlan {
+  std::vector<uint8_t> map;
+  int Nq = 0, Nkv = 0;
+  int* d_qoff = nullptr;
+  int4* d_qlist = nullptr;
+  int* d_qord = nullptr;
+  int* d_koff = nullptr;
+  int4* d_klist = nullptr;
+  int* d_kord = nullptr;
+};
+
+void free_bwd_plan(BwdPlan& p) {
+  cudaFree(p.d_qoff);
+  cudaFree(p.d_qlist);
+  cudaFree(p.d_qord);
+  cudaFree(p.d_koff);
+  cudaFree(p.d_klist);
+  cudaFree(p.d_kord);
+  p.d_qoff = p.d_koff = p.d_qord = p.d_kord = nullptr;
+  p.d_qlist = p.d_klist = nullptr;
+}
+
 struct DevWs {
   int* d_err = nullptr;
   float* d_part = nullptr;
@@ -64,6 +90,7 @@ struct DevWs {
   float* d_stats = nullptr;  // key-statistics partial sums
   size_t stats_floats = 0;
   std::list<DevPlan> plans;  // most recent first
+  std::list<BwdPlan> bplans;  // most recent first
 };
 
 std::mutex g_mu;
@@ -185,6 +212,72 @@ int get_plan(DevWs& ws, int mask_kind, const uint8_t* block_map, int Nq, int Nkv
     ws.plans.pop_back();
   }
   *out = &ws.plans.front();
+  return ATTN_OK;
+}
+
+int get_bwd_plan(DevWs& ws, const uint8_t* block_map, int Nq, int Nkv, cudaStream_t s, BwdPlan** out) {
+  const int nbq = (Nq + kGrain - 1) / kGrain, nbk = (Nkv + kGrain - 1) / kGrain;
+  const size_t map_bytes = static_cast<size_t>(nbq) * nbk;
+  for (auto it = ws.bplans.begin(); it != ws.bplans.end(); ++it) {
+    if (it->Nq != Nq || it->Nkv != Nkv || it->map.size() != map_bytes ||
+        std::memcmp(it->map.data(), block_map, map_bytes) != 0)
+      continue;
+    ws.bplans.splice(ws.bplans.begin(), ws.bplans, it);
+    *out = &ws.bplans.front();
+    return ATTN_OK;
+  }
+  const int n_qt = (Nq + 127) / 128, n_kt = (Nkv + 127) / 128;
+  std::vector<std::vector<int4>> ql(n_qt), kl(n_kt);
+  for (int qt = 0; qt < n_qt; ++qt)
+    for (int kt = 0; kt < n_kt; ++kt) {
+      unsigned long long m = 0;
+      for (int i = 0; i < 8 && qt * 8 + i < nbq; ++i)
+        for (int j = 0; j < 8 && kt * 8 + j < nbk; ++j)
+          if (block_map[static_cast<size_t>(qt * 8 + i) * nbk + kt * 8 + j]) m |= 1ull << (i * 8 + j);
+      if (!m) continue;
+      const int lo = static_cast<int>(m & 0xffffffffull), hi = static_cast<int>(m >> 32);
+      ql[qt].push_back(make_int4(kt, lo, hi, 0));
+      kl[kt].push_back(make_int4(qt, lo, hi, 0));
+    }
+  auto flatten = [](const std::vector<std::vector<int4>>& l, std::vector<int>* off, std::vector<int4>* flat,
+                    std::vector<int>* ord) {
+    off->assign(1, 0);
+    for (const auto& v : l) {
+      flat->insert(flat->end(), v.begin(), v.end());
+      off->push_back(static_cast<int>(flat->size()));
+    }
+    ord->resize(l.size());
+    for (size_t i = 0; i < l.size(); ++i) (*ord)[i] = static_cast<int>(i);
+    std::stable_sort(ord->begin(), ord->end(), [&](int a, int b) { return l[a].size() > l[b].size(); });
+    if (flat->empty()) flat->push_back(make_int4(0, 0, 0, 0));  // never read: every list is empty
+  };
+  std::vector<int> qoff, qord, koff, kord;
+  std::vector<int4> qflat, kflat;
+  flatten(ql, &qoff, &qflat, &qord);
+  flatten(kl, &koff, &kflat, &kord);
+  BwdPlan bp;
+  bp.map.assign(block_map, block_map + map_bytes);
+  bp.Nq = Nq;
+  bp.Nkv = Nkv;
+  int rc;
+  if ((rc = upload(&bp.d_qoff, qoff.data(), qoff.size(), s)) || (rc = upload(&bp.d_qlist, qflat.data(), qflat.size(), s)) ||
+      (rc = upload(&bp.d_qord, qord.data(), qord.size(), s)) || (rc = upload(&bp.d_koff, koff.data(), koff.size(), s)) ||
+      (rc = upload(&bp.d_klist, kflat.data(), kflat.size(), s)) || (rc = upload(&bp.d_kord, kord.data(), kord.size(), s))) {
+    free_bwd_plan(bp);
+    return rc;
+  }
+  cudaError_t e = cudaStreamSynchronize(s);  // the host vectors die with this scope
+  if (e != cudaSuccess) {
+    free_bwd_plan(bp);
+    return cuda_err(e, "backward plan upload");
+  }
+  ws.bplans.push_front(std::move(bp));
+  while (ws.bplans.size() > kMaxPlans) {
+    cudaDeviceSynchronize();
+    free_bwd_plan(ws.bplans.back());
+    ws.bplans.pop_back();
+  }
+  *out = &ws.bplans.front();
   return ATTN_OK;
 }
 
@@ -490,14 +583,13 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
 
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
              void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nkv, int d, float scale,
-             int mask_kind, void* stream) {
+             int mask_kind, const uint8_t* block_map, void* stream) {
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv)
     return set_err(ATTN_ERR_NULL, "every tensor of attn_bwd must be non-NULL");
   if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nkv < 1) return set_err(ATTN_ERR_SHAPE, "sizes must be >= 1");
   if (Hq % Hkv != 0) return set_err(ATTN_ERR_SHAPE, "Hq (%d) is not a multiple of Hkv (%d)", Hq, Hkv);
   if (d != 64 && d != 128) return set_err(ATTN_ERR_UNSUPPORTED, "attn_bwd needs d in {64, 128}");
-  if (mask_kind != ATTN_MASK_NONE && mask_kind != ATTN_MASK_CAUSAL)
-    return set_err(ATTN_ERR_UNSUPPORTED, "attn_bwd supports ATTN_MASK_NONE and ATTN_MASK_CAUSAL");
+  if (int rc = check_mask_args(mask_kind, block_map)) return rc;
   if (!(scale > 0.f) || !std::isfinite(scale)) return set_err(ATTN_ERR_SHAPE, "scale must be positive and finite");
   if (B > 65535 || Hq > 65535 || static_cast<long long>(B) * Hq * Nq >= (1ll << 31) ||
       static_cast<long long>(B) * Hkv * Nkv >= (1ll << 31))
@@ -541,6 +633,16 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   a.Nkv = Nkv;
   a.causal = mask_kind == ATTN_MASK_CAUSAL;
   a.scale = scale;
+  if (mask_kind == ATTN_MASK_BLOCK) {
+    BwdPlan* bp = nullptr;
+    if (int rc = get_bwd_plan(*ws, block_map, Nq, Nkv, s, &bp)) return rc;
+    a.qoff = bp->d_qoff;
+    a.qlist = bp->d_qlist;
+    a.qord = bp->d_qord;
+    a.koff = bp->d_koff;
+    a.klist = bp->d_klist;
+    a.kord = bp->d_kord;
+  }
   cudaError_t e = launch_bwd(d, a, s);
   return e == cudaSuccess ? ATTN_OK : cuda_err(e, "backward launch");
 }
@@ -622,6 +724,7 @@ int attn_shutdown(void) {
     if (cudaSetDevice(kv.first) != cudaSuccess) continue;
     cudaDeviceSynchronize();
     for (auto& p : kv.second.plans) free_plan(p);
+    for (auto& p : kv.second.bplans) free_bwd_plan(p);
     cudaFree(kv.second.d_part);
     cudaFree(kv.second.d_stats);
     cudaFree(kv.second.d_err);

@@ -140,35 +140,69 @@ __device__ __forceinline__ long long bwd_item(long long k, long long n_items) {
 // most Q tiles).
 struct KvItem {
   int b, hkv, k0, first_qt, per_head, steps;
+  const int4* list;  // BLOCK masks: the key tile's live Q tiles; else null
 };
+template <bool BLK>
 __device__ __forceinline__ KvItem kv_item(const BwdArgs& a, long long w) {
   KvItem it;
   const int per_kt = a.Hkv * a.B;
   const int r = static_cast<int>(w % per_kt);
-  it.k0 = static_cast<int>(w / per_kt) * kT;
+  int kt = static_cast<int>(w / per_kt);
   it.hkv = r / a.B;
   it.b = r % a.B;
   const int n_qt = (a.Nq + kT - 1) / kT;
-  // causal: row i sees key k0 iff i >= k0 - off; earlier Q tiles see none of these keys
-  it.first_qt = a.causal ? min(n_qt, max(0, it.k0 - (a.Nkv - a.Nq)) / kT) : 0;
-  it.per_head = n_qt - it.first_qt;
+  it.list = nullptr;
+  if (BLK) {
+    kt = a.kord[kt];
+    it.list = a.klist + a.koff[kt];
+    it.first_qt = 0;
+    it.per_head = a.koff[kt + 1] - a.koff[kt];
+  } else {
+    // causal: row i sees key k0 iff i >= k0 - off; earlier Q tiles see none of these keys
+    it.first_qt = a.causal ? min(n_qt, max(0, kt * kT - (a.Nkv - a.Nq)) / kT) : 0;
+    it.per_head = n_qt - it.first_qt;
+  }
+  it.k0 = kt * kT;
   it.steps = (a.Hq / a.Hkv) * it.per_head;
   return it;
+}
+
+// The Q tile and live-block bitmap of step u of a dK/dV item.
+template <bool BLK>
+__device__ __forceinline__ int kv_step_qt(const KvItem& it, int u, unsigned long long* bits) {
+  const int idx = u % it.per_head;
+  if (!BLK) {
+    *bits = ~0ull;
+    return it.first_qt + idx;
+  }
+  const int4 e = it.list[idx];
+  *bits = static_cast<unsigned>(e.y) | (static_cast<unsigned long long>(static_cast<unsigned>(e.z)) << 32);
+  return e.x;
 }
 
 // dQ item: Q tile slowest, last tile first (under a causal mask the last
 // tiles visit the most K/V tiles).
 struct QItem {
   int b, hq, q0, n_kv;
+  const int4* list;  // BLOCK masks: the Q tile's live key tiles; else null
 };
+template <bool BLK>
 __device__ __forceinline__ QItem q_item(const BwdArgs& a, long long w) {
   QItem it;
   const int per_qt = a.Hq * a.B;
   const int n_qt = (a.Nq + kT - 1) / kT;
   const int r = static_cast<int>(w % per_qt);
-  it.q0 = (n_qt - 1 - static_cast<int>(w / per_qt)) * kT;
   it.hq = r / a.B;
   it.b = r % a.B;
+  it.list = nullptr;
+  if (BLK) {
+    const int qt = a.qord[w / per_qt];
+    it.q0 = qt * kT;
+    it.list = a.qlist + a.qoff[qt];
+    it.n_kv = a.qoff[qt + 1] - a.qoff[qt];
+    return it;
+  }
+  it.q0 = (n_qt - 1 - static_cast<int>(w / per_qt)) * kT;
   int n_kv = (a.Nkv + kT - 1) / kT;
   if (a.causal) {
     const int last = min(it.q0 + kT - 1, a.Nq - 1) + (a.Nkv - a.Nq);  // largest key any row may see
@@ -176,6 +210,18 @@ __device__ __forceinline__ QItem q_item(const BwdArgs& a, long long w) {
   }
   it.n_kv = n_kv;
   return it;
+}
+
+// The key tile and live-block bitmap of step j of a dQ item.
+template <bool BLK>
+__device__ __forceinline__ int q_step_kt(const QItem& it, int j, unsigned long long* bits) {
+  if (!BLK) {
+    *bits = ~0ull;
+    return j;
+  }
+  const int4 e = it.list[j];
+  *bits = static_cast<unsigned>(e.y) | (static_cast<unsigned long long>(static_cast<unsigned>(e.z)) << 32);
+  return e.x;
 }
 
 __device__ __forceinline__ uint8_t* align1k(uint8_t* p) {
@@ -237,16 +283,19 @@ __device__ __forceinline__ void store_cols(uint32_t t, __nv_bfloat16* dst, float
 
 // p = 2^(s * sl2 - lse2) for one thread's 64 columns (sr: the S values as
 // loaded from TMEM); nl(c) gives -lse2 for the columns c, c + 1.  MASK:
-// columns outside [lo, hi) are 0.
+// columns outside [lo, hi), and columns of a 16-column group whose bit in
+// `groups` is clear, are 0.
 template <int NP, bool MASK, typename NLFn>
-__device__ __forceinline__ void p_row(float* p, const uint32_t* sr, float sl2, NLFn nl, int lo, int hi) {
+__device__ __forceinline__ void p_row(float* p, const uint32_t* sr, float sl2, NLFn nl, int lo, int hi,
+                                      unsigned groups = 0xFu) {
   const float2 sl = make_float2(sl2, sl2);
 #pragma unroll
   for (int c = 0; c < 64; c += 2) {
     float2 e = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl, nl(c));
     if (MASK) {
-      if (c < lo || c >= hi) e.x = -INFINITY;
-      if (c + 1 < lo || c + 1 >= hi) e.y = -INFINITY;
+      const bool live = (groups >> (c >> 4)) & 1u;  // c and c + 1 share their group
+      if (!live || c < lo || c >= hi) e.x = -INFINITY;
+      if (!live || c + 1 < lo || c + 1 >= hi) e.y = -INFINITY;
     }
     const float2 v = ((c >> 1) & 7) < NP ? exp2_poly2(e) : make_float2(wm_ex2(e.x), wm_ex2(e.y));
     p[c] = v.x;
@@ -273,7 +322,9 @@ __device__ __forceinline__ void write_ds(uint32_t t_dp, uint32_t t_ds, const flo
 }
 
 // ----------------------------------------------------------------- dK, dV
-template <int D>
+// BLK: block-sparse mask (tile lists with block bitmaps); otherwise no mask
+// or causal.
+template <int D, bool BLK>
 __global__ void __launch_bounds__(kBThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -349,7 +400,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (long long k = 0; ok; ++k) {
       const long long w = bwd_item(k, n_items);
       if (w < 0) break;
-      const KvItem it = kv_item(a, w);
+      const KvItem it = kv_item<BLK>(a, w);
       // K and V of the previous item are free once its last S and dP have run
       if (k > 0 && !wwait(br.fixed_empty, (k - 1) & 1)) {
         ok = false;
@@ -368,7 +419,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
           ok = false;
           break;
         }
-        const int hq = it.hkv * G + u / it.per_head, qt = it.first_qt + u % it.per_head;
+        unsigned long long bits;
+        const int hq = it.hkv * G + u / it.per_head, qt = kv_step_qt<BLK>(it, u, &bits);
         uint8_t* st = stage(g);
         mbar_arrive_expect_tx_elect(&br.full[s], 2 * C::kTile + C::kVecBytes);
 #pragma unroll
@@ -396,7 +448,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (long long k = 0; ok; ++k) {
       const long long w = bwd_item(k, n_items);
       if (w < 0) break;
-      const KvItem it = kv_item(a, w);
+      const KvItem it = kv_item<BLK>(a, w);
       if (!wwait(br.fixed_full, k & 1)) {
         ok = false;
         break;
@@ -506,11 +558,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (long long k = 0; ok; ++k) {
       const long long w = bwd_item(k, n_items);
       if (w < 0) break;
-      const KvItem it = kv_item(a, w);
+      const KvItem it = kv_item<BLK>(a, w);
       const int key = it.k0 + quarter * 32 + lane;  // this thread's key (TMEM lane)
       for (int u = 0; u < it.steps; ++u, ++g) {
         const int s = g % R, x = g % NB;
-        const int q0 = (it.first_qt + u % it.per_head) * kT + 64 * h;  // query of this thread's first column
+        unsigned long long bits;
+        const int q0 = kv_step_qt<BLK>(it, u, &bits) * kT + 64 * h;  // query of this thread's first column
         if (!wwait(&br.full[s], (g / R) & 1) || !wwait(&br.s_full[x], (g / NB) & 1)) {
           ok = false;
           break;
@@ -526,8 +579,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
           tmem_wait_ld();
           // causal: query q0 + c sees this key iff c >= key - off - q0
           auto nl = [&](int c) { return *reinterpret_cast<const float2*>(vs + c); };
+          // block masks: this key's 16-key block j against the four 16-query
+          // groups of the thread's columns
+          const int kb = (quarter * 32 + lane) >> 4;
+          unsigned groups = 0xFu;
+          if (BLK) {
+            groups = 0u;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) groups |= static_cast<unsigned>((bits >> ((4 * h + q4) * 8 + kb)) & 1ull) << q4;
+          }
           if (a.causal && it.k0 + kT - 1 > q0 + off)
             p_row<kPolyPairsB<D>, true>(p, sr, sl2, nl, key - off - q0, 64);
+          else if (BLK && __any_sync(0xffffffffu, groups != 0xFu))
+            p_row<kPolyPairsB<D>, true>(p, sr, sl2, nl, 0, 64, groups);
           else
             p_row<kPolyPairsB<D>, false>(p, sr, sl2, nl, 0, 64);
         }
@@ -612,7 +676,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
 }
 
 // -------------------------------------------------------------------- dQ
-template <int D>
+template <int D, bool BLK>
 __global__ void __launch_bounds__(kBThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -687,7 +751,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (long long k = 0; ok; ++k) {
       const long long w = bwd_item(k, n_items);
       if (w < 0) break;
-      const QItem it = q_item(a, w);
+      const QItem it = q_item<BLK>(a, w);
       // Q, dO and O of the previous item are free once its last S and dP
       // have run and D has been computed
       if (k > 0 && !wwait(br.fixed_empty, (k - 1) & 1)) {
@@ -710,11 +774,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
           break;
         }
         uint8_t* st = stage(g);
+        unsigned long long bits;
+        const int kt = q_step_kt<BLK>(it, j, &bits);
         mbar_arrive_expect_tx_elect(&br.full[s], 2 * C::kTile);
 #pragma unroll
         for (int ch = 0; ch < C::NCH; ++ch) {
-          tma_load_4d_elect(st + ch * C::kChunk, &tmK, &br.full[s], 64 * ch, hkv, j * kT, it.b);
-          tma_load_4d_elect(st + C::kTile + ch * C::kChunk, &tmV, &br.full[s], 64 * ch, hkv, j * kT, it.b);
+          tma_load_4d_elect(st + ch * C::kChunk, &tmK, &br.full[s], 64 * ch, hkv, kt * kT, it.b);
+          tma_load_4d_elect(st + C::kTile + ch * C::kChunk, &tmV, &br.full[s], 64 * ch, hkv, kt * kT, it.b);
         }
       }
     }
@@ -731,7 +797,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (long long k = 0; ok; ++k) {
       const long long w = bwd_item(k, n_items);
       if (w < 0) break;
-      const QItem it = q_item(a, w);
+      const QItem it = q_item<BLK>(a, w);
       const int acc = static_cast<int>(k % NA);
       if (!wwait(br.fixed_full, k & 1)) {
         ok = false;
@@ -825,7 +891,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (long long k = 0; ok; ++k) {
       const long long w = bwd_item(k, n_items);
       if (w < 0) break;
-      const QItem it = q_item(a, w);
+      const QItem it = q_item<BLK>(a, w);
       const int acc = static_cast<int>(k % NA);
       const int row = it.q0 + r;
       // rows past Nq: lse2 = +inf makes their P exactly 0
@@ -869,10 +935,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         tc_fence_after();
         // keys at or past column lim are masked: past Nkv, and past the
-        // causal diagonal (rows with no visible key get lim <= 0)
-        const int c0 = j * kT + 64 * h;  // key of this thread's first column
+        // causal diagonal (rows with no visible key get lim <= 0); block
+        // masks: the four 16-key groups of the thread's columns against its
+        // 16-row block
+        unsigned long long bits;
+        const int c0 = q_step_kt<BLK>(it, j, &bits) * kT + 64 * h;  // key of this thread's first column
         int lim = min(64, a.Nkv - c0);
         if (a.causal) lim = min(lim, row + off + 1 - c0);
+        const unsigned groups = BLK ? static_cast<unsigned>((bits >> ((r >> 4) * 8 + 4 * h)) & 0xFull) : 0xFu;
         const uint32_t t_s = t_row + 128 * x + 64 * h;
         float p[64];
         {
@@ -881,8 +951,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
           tmem_ld32(t_s + 32, sr + 32);
           tmem_wait_ld();
           auto nl = [&](int) { return make_float2(-l2, -l2); };
-          if (__any_sync(0xffffffffu, lim < 64))
-            p_row<kPolyPairsB<D>, true>(p, sr, sl2, nl, 0, lim);
+          if (__any_sync(0xffffffffu, lim < 64 || groups != 0xFu))
+            p_row<kPolyPairsB<D>, true>(p, sr, sl2, nl, 0, lim, groups);
           else
             p_row<kPolyPairsB<D>, false>(p, sr, sl2, nl, 0, 64);
         }
@@ -952,16 +1022,17 @@ __global__ void __launch_bounds__(kBThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D>
+template <int D, bool BLK>
 cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   using C = BCfg<D>;
   static int attr_dev = -1, n_sm = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemQ);
+    cudaError_t e =
+        cudaFuncSetAttribute(bwd_dq_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemQ);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemKV);
+      e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemKV);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
@@ -975,11 +1046,11 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   const long long n_q = static_cast<long long>((a.Nq + kT - 1) / kT) * a.Hq * a.B;
   const long long n_kv = static_cast<long long>((a.Nkv + kT - 1) / kT) * a.Hkv * a.B;
   // The dQ kernel also writes D and lse2, which the dK/dV kernel reads.
-  bwd_dq_kernel<D><<<static_cast<unsigned>(n_q < n_sm ? n_q : n_sm), kBThreads, C::kSmemQ, s>>>(tq, tdo, tk, tv, to,
+  bwd_dq_kernel<D, BLK><<<static_cast<unsigned>(n_q < n_sm ? n_q : n_sm), kBThreads, C::kSmemQ, s>>>(tq, tdo, tk, tv, to,
                                                                                                  tdq, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dkdv_kernel<D><<<static_cast<unsigned>(n_kv < n_sm ? n_kv : n_sm), kBThreads, C::kSmemKV, s>>>(tq, tdo, tk, tv,
+  bwd_dkdv_kernel<D, BLK><<<static_cast<unsigned>(n_kv < n_sm ? n_kv : n_sm), kBThreads, C::kSmemKV, s>>>(tq, tdo, tk, tv,
                                                                                                      tdk, tdv, a);
   return cudaGetLastError();
 }
@@ -987,8 +1058,9 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_bwd(int d, const BwdArgs& a, cudaStream_t s) {
-  if (d == 64) return launch_bwd_d<64>(a, s);
-  return launch_bwd_d<128>(a, s);
+  const bool blk = a.qlist != nullptr;
+  if (d == 64) return blk ? launch_bwd_d<64, true>(a, s) : launch_bwd_d<64, false>(a, s);
+  return blk ? launch_bwd_d<128, true>(a, s) : launch_bwd_d<128, false>(a, s);
 }
 
 }  // namespace eio

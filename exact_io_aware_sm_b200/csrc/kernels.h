@@ -104,6 +104,17 @@ struct BwdArgs {
   int* err;
   int B, Hq, Hkv, Nq, Nkv, causal;
   float scale;
+  // BLOCK masks (all null otherwise): per 128-row Q tile qt, entries
+  // qlist[qoff[qt] .. qoff[qt+1]) = (key tile, bitmap low, bitmap high, 0),
+  // bit i*8+j set when the 16 x 16 block (query block i, key block j) of the
+  // tile pair is live; klist / koff the same per key tile with (Q tile, ...).
+  // qord / kord: the tiles in visit order (longest list first).
+  const int* qoff;
+  const int4* qlist;
+  const int* qord;
+  const int* koff;
+  const int4* klist;
+  const int* kord;
 };
 cudaError_t launch_bwd(int d, const BwdArgs& a, cudaStream_t s);
 

@@ -256,15 +256,18 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
  *   lse         device, [B, Hq, Nq] fp32, the forward LSE (natural log)
  *   dq          device, [B, Nq, Hq, d] bf16 (written)
  *   dk, dv      device, [B, Nkv, Hkv, d] bf16 (written)
- *   mask_kind   ATTN_MASK_NONE or ATTN_MASK_CAUSAL (as attn_fwd)
+ *   mask_kind, block_map  as attn_fwd (NONE, CAUSAL or BLOCK with its host map)
  * Limits: d == 64 or 128; all pointers 16-byte aligned.
  * Scratch: 2*B*Hq*ceil(Nq/128)*128 floats of library workspace.
- * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED (other masks or d), CUDA, WORKSPACE;
+ * Under a BLOCK mask the live 128 x 128 tile pairs are listed on the host
+ * (cached per map, like attn_fwd's schedules) with the bitmap of their 16 x 16
+ * blocks; only live pairs are computed.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED (d), MASK, CUDA, WORKSPACE;
  * a bounded wait that runs out latches ATTN_ERR_DEVICE_TIMEOUT.
  */
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
              void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nkv, int d, float scale,
-             int mask_kind, void* stream);
+             int mask_kind, const uint8_t* block_map, void* stream);
 
 /*
  * attn_debug_fault -- test hook for the device time-out path.

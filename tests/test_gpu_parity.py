@@ -241,6 +241,36 @@ def test_backward_small(case):
     check_grad(dv, rv, f"{case} dv")
 
 
+BWD_BLOCK_CASES = [
+    # B, Hq, Hkv, N, d, map
+    (1, 2, 2, 300, 64, "random"),
+    (2, 4, 2, 250, 128, "random"),
+    (1, 2, 2, 480, 64, "frames"),  # 6 frames x 80 tokens: own, previous and first frame
+]
+
+
+@pytest.mark.parametrize("case", BWD_BLOCK_CASES)
+def test_backward_block_mask(case):
+    B, Hq, Hkv, N, d, kind = case
+    seed = 3500 + BWD_BLOCK_CASES.index(case)
+    q, k, v = make_inputs(seed, B, Hq, Hkv, N, N, d)
+    dout = synthetic.tensor(seed, 9, (B, N, Hq, d))
+    if kind == "frames":
+        bm = eio.frame_block_map(6, 80)
+    else:
+        bm = random_block_map(seed, N, N, p=0.4)
+        bm[3] = 0  # a block row with no key: its gradients are zero
+    scale = 1 / math.sqrt(d)
+    tq, tk, tv, tdo = dev_bf16(q), dev_bf16(k), dev_bf16(v), dev_bf16(dout)
+    o, lse = eio.attn_fwd(tq, tk, tv, scale=scale, mask_kind=eio.MASK_BLOCK, block_map=bm)
+    dq, dk, dv = eio.attn_bwd(tq, tk, tv, o, lse, tdo, scale=scale, mask_kind=eio.MASK_BLOCK, block_map=bm)
+    eio.sync_status()
+    rq, rk, rv = oracle.attn_bwd(q, k, v, dout, scale, oracle.MASK_BLOCK, bm)
+    check_grad(dq, rq, f"{case} dq")
+    check_grad(dk, rk, f"{case} dk")
+    check_grad(dv, rv, f"{case} dv")
+
+
 def test_backward_gpt2_shape_first_batch_element():
     B, H, N, d = 8, 12, 1024, 64
     q, k, v = make_inputs(1002, B, H, H, N, N, d)
