@@ -199,3 +199,32 @@ def test_no_device_is_an_error_not_a_crash():
     # valid arguments, no GPU: reported as a CUDA error, nothing dereferenced
     assert _fwd() == 6
     assert eio.lib().attn_shutdown() == 0
+
+
+def test_backward_bound_and_stats_argument_errors():
+    """attn_bwd, attn_key_stats and attn_fwd_bound reject bad arguments on the
+    host, before any device work (their status codes as documented)."""
+    L = eio.lib()
+
+    def bwd(mask=0, bm=None, d=64, q=FAKE, Hq=2, Hkv=2):
+        return L.attn_bwd(q, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, Hq, Hkv, 16, 16, d, 0.125, mask,
+                          bm, None)
+    assert bwd(q=None) == 1
+    assert bwd(Hq=3) == 2
+    assert bwd(d=96) == 4
+    assert bwd(mask=2, bm=None) == 5  # BLOCK without its map
+    assert bwd(mask=9) == 5
+    assert L.attn_key_stats(None, FAKE, FAKE, 1, 16, 2, 64, None) == 1
+    assert L.attn_key_stats(FAKE, FAKE, FAKE, 1, 0, 2, 64, None) == 2
+    assert L.attn_key_stats(FAKE, FAKE, FAKE, 1, 16, 2, 96, None) == 4
+    assert L.attn_key_stats(FAKE + 8, FAKE, FAKE, 1, 16, 2, 64, None) == 3
+
+    def fb(kbar=FAKE, radius=FAKE, nfb=None, d=64, mask=0, bm=None, o=FAKE):
+        return L.attn_fwd_bound(FAKE, FAKE, FAKE, o, None, 1, 2, 2, 16, 16, d, 0.125, mask, bm, kbar, radius, nfb,
+                                None)
+    assert fb(kbar=None) == 1
+    assert fb(o=None) == 1
+    assert fb(d=32) == 4
+    assert fb(mask=2) == 5
+    assert fb(kbar=FAKE + 4) == 3
+    assert fb(nfb=FAKE + 2) == 3
