@@ -361,8 +361,10 @@ static int fwd_bf16(DevWs& wsr, const void* q, const void* k, const void* v, voi
   if (int rc = make_map(&tq, q, B, Nq, Hq, d)) return rc;
   if (int rc = make_map(&tk, k, B, Nkv, Hkv, d)) return rc;
   if (int rc = make_map(&tv, v, B, Nkv, Hkv, d)) return rc;
-  CUtensorMap to;
-  if (!encode_bf16_map(&to, o, B, Nq, Hq, d, 16)) return ATTN_ERR_CUDA;
+  CUtensorMap to, tk16, tv16;
+  if (!encode_bf16_map(&to, o, B, Nq, Hq, d, 16) || !encode_bf16_map(&tk16, k, B, Nkv, Hkv, d, 16) ||
+      !encode_bf16_map(&tv16, v, B, Nkv, Hkv, d, 16))
+    return ATTN_ERR_CUDA;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -393,7 +395,7 @@ static int fwd_bf16(DevWs& wsr, const void* q, const void* k, const void* v, voi
   a.kbar = kbar;
   a.radius = radius;
   a.n_fallback = n_fallback;
-  cudaError_t e = launch_prefill_bf16(d, tq, tk, tv, to, a, s);
+  cudaError_t e = launch_prefill_bf16(d, tq, tk, tv, to, tk16, tv16, a, s);
   return e == cudaSuccess ? ATTN_OK : cuda_err(e, "prefill launch");
 }
 

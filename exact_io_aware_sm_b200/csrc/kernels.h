@@ -49,10 +49,11 @@ int key_stats_splits(int Nkv);
 cudaError_t launch_key_stats(int d, const KeyStatsArgs& a, cudaStream_t s);
 
 // bf16 tensor-core prefill (tcgen05 / TMA).  d in {64, 128}.
-// to: O as {d, Hq, Nq, B} with a {64, 1, 16, 1} box (used by the d = 64 epilogue).
+// to: O as {d, Hq, Nq, B} with a {64, 1, 16, 1} box (used by the d = 64 epilogue);
+// tk16, tv16: K and V with 16-row boxes (two-segment KV tiles).
 cudaError_t launch_prefill_bf16(int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                                const CUtensorMap& tv, const CUtensorMap& to, const PrefillArgs& a,
-                                cudaStream_t s);
+                                const CUtensorMap& tv, const CUtensorMap& to, const CUtensorMap& tk16,
+                                const CUtensorMap& tv16, const PrefillArgs& a, cudaStream_t s);
 int prefill_bf16_smem_bytes(int d);
 
 struct PrefillF32Args {

@@ -2,6 +2,7 @@
 #include "plan.h"
 
 #include <algorithm>
+#include <utility>
 #include <cstring>
 
 namespace eio {
@@ -81,12 +82,79 @@ void build_plan(int mask_kind, const uint8_t* block_map, int Nq, int Nkv, Plan* 
   });
 }
 
+// A Q tile's KV list re-cut into tiles of up to 128 keys made of at most two
+// contiguous segments: the list's spans of consecutive keys are laid end to
+// end and cut every 128 keys, a tile taking the head of the next span when its
+// own span ends early.  Returns false (out untouched) for a list with a
+// partial tile, which keeps its own tiles.
+static bool recut(const Plan& plan, const QTile& q, std::vector<PairKV>* out) {
+  std::vector<std::pair<int, int>> spans;  // (first key, keys)
+  for (int k = 0; k < q.n_kv; ++k) {
+    const KVTile& t = plan.kv[q.first_kv + k];
+    if (t.partial) return false;
+    if (!spans.empty() && spans.back().first + spans.back().second == t.col0)
+      spans.back().second += t.ncols;
+    else
+      spans.push_back({t.col0, t.ncols});
+  }
+  size_t si = 0;
+  int off = 0;  // keys of spans[si] already placed
+  while (si < spans.size()) {
+    PairKV v{};
+    const int n0 = std::min(kTileKV, spans[si].second - off);
+    v.col0 = spans[si].first + off;
+    v.ncols = n0;
+    off += n0;
+    if (off == spans[si].second) {
+      ++si;
+      off = 0;
+    }
+    if (v.ncols < kTileKV && si < spans.size()) {
+      const int n1 = std::min(kTileKV - v.ncols, spans[si].second);
+      v.col1 = spans[si].first;
+      v.ncols += n1;
+      v.flags = n0 << 8;
+      off = n1;
+      if (off == spans[si].second) {
+        ++si;
+        off = 0;
+      }
+    }
+    out->push_back(v);
+  }
+  return true;
+}
+
 void build_pairs(const Plan& plan, bool rows_mode, PairPlan* out) {
   out->rows_mode = rows_mode;
   out->pairs.clear();
   out->kv.clear();
   out->order.clear();
+  auto same = [](const PairKV& x, const PairKV& y) {
+    return x.col0 == y.col0 && x.ncols == y.ncols && x.flags == y.flags && x.col1 == y.col1;
+  };
   auto push_pair = [&](const QTile* a, const QTile& b) {
+    // Two-segment tiles where both lists allow them and A's stays a prefix of B's.
+    std::vector<PairKV> vb, va;
+    if (recut(plan, b, &vb) && (!a || recut(plan, *a, &va))) {
+      bool ok = va.size() <= vb.size();
+      for (size_t k = 0; ok && k < va.size(); ++k) ok = same(va[k], vb[k]);
+      if (ok) {
+        PairTile pt{};
+        pt.rowB = b.row0;
+        pt.nrowsB = b.nrows;
+        pt.nB = static_cast<int32_t>(vb.size());
+        pt.kv_first = static_cast<int32_t>(out->kv.size());
+        if (a) {
+          pt.rowA = a->row0;
+          pt.nrowsA = a->nrows;
+          pt.nA = static_cast<int32_t>(va.size());
+        }
+        out->kv.insert(out->kv.end(), vb.begin(), vb.end());
+        out->pairs.push_back(pt);
+        return;
+      }
+    }
     PairTile pt{};
     pt.rowB = b.row0;
     pt.nrowsB = b.nrows;

@@ -44,8 +44,12 @@ struct PairTile {
   int32_t rowA, nrowsA, rowB, nrowsB;  // nrowsA == 0: slot A unused
   int32_t kv_first, nA, nB, pad;       // KV tiles [kv_first, kv_first + nB); A uses the first nA
 };
+// A KV tile of up to 128 keys in one or two contiguous segments:
+// [col0, col0 + n0) then [col1, col1 + ncols - n0), n0 = flags >> 8 (0: one
+// segment of ncols keys from col0).  Two segments join the short tails of
+// separate key spans of a block-sparse list (never on partial tiles).
 struct PairKV {
-  int32_t col0, ncols, flags, pad;  // flags bit 0: partial for A, bit 1: partial for B
+  int32_t col0, ncols, flags, col1;  // flags bit 0: partial for A, bit 1: partial for B; bits 8..15: n0
 };
 struct PairPlan {
   bool rows_mode = false;

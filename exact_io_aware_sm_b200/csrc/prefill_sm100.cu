@@ -199,7 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
-                        const __grid_constant__ CUtensorMap tmO, const PrefillArgs a) {
+                        const __grid_constant__ CUtensorMap tmO,
+                        const __grid_constant__ CUtensorMap tmK16,
+                        const __grid_constant__ CUtensorMap tmV16, const PrefillArgs a) {
   using C = Cfg<D>;
   constexpr int R = C::kRing;
   constexpr int NCH = D / 64;  // 64-element swizzle chunks per row
@@ -319,12 +321,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++seq;
             continue;
           }
-          mbar_arrive_expect_tx_elect(&ring_full[slot], C::kTileBytes);
-          const CUtensorMap* map = t == 0 ? &tmK : &tmV;
+          const int n0 = (kt.z >> 8) & 0xFF;  // two-segment tile: keys in the first segment
+          uint8_t* dst = smem + C::kOffRing + slot * C::kTileBytes;
+          if (n0 == 0) {
+            mbar_arrive_expect_tx_elect(&ring_full[slot], C::kTileBytes);
+            const CUtensorMap* map = t == 0 ? &tmK : &tmV;
 #pragma unroll
-          for (int ch = 0; ch < NCH; ++ch)
-            tma_load_4d_elect(smem + C::kOffRing + slot * C::kTileBytes + ch * C::kChunkBytes, map,
-                              &ring_full[slot], ch * 64, it.hkv, kt.x, it.b);
+            for (int ch = 0; ch < NCH; ++ch)
+              tma_load_4d_elect(dst + ch * C::kChunkBytes, map, &ring_full[slot], ch * 64, it.hkv, kt.x, it.b);
+          } else {
+            // [kt.x, kt.x + n0) then [kt.w, ...) into consecutive rows, 16 rows per copy
+            mbar_arrive_expect_tx_elect(&ring_full[slot], static_cast<uint32_t>(kt.y) * 128 * NCH);
+            const CUtensorMap* map = t == 0 ? &tmK16 : &tmV16;
+            for (int r = 0; r < kt.y; r += 16) {
+              const int src = r < n0 ? kt.x + r : kt.w + (r - n0);
+#pragma unroll
+              for (int ch = 0; ch < NCH; ++ch)
+                tma_load_4d_elect(dst + ch * C::kChunkBytes + r * 128, map, &ring_full[slot], ch * 64, it.hkv, src,
+                                  it.b);
+            }
+          }
           ++seq;
           // At start-up every CTA fills its whole ring at once; let the first
           // K tile (and the Q tiles issued before it) land before queueing the
@@ -698,7 +714,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool STAGGER, bool BOUND>
 cudaError_t launch_ds(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                      const CUtensorMap& to, const PrefillArgs& a, cudaStream_t s) {
+                      const CUtensorMap& to, const CUtensorMap& tk16, const CUtensorMap& tv16,
+                      const PrefillArgs& a, cudaStream_t s) {
   static int attr_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -717,16 +734,19 @@ cudaError_t launch_ds(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
   if (a.n_items == 0) return cudaSuccess;
   const long long grid = a.n_items < a.num_ctas ? a.n_items : a.num_ctas;
   prefill_bf16_kernel<D, STAGGER, BOUND>
-      <<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmem, s>>>(tq, tk, tv, to, a);
+      <<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmem, s>>>(tq, tk, tv, to, tk16, tv16, a);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                     const CUtensorMap& to, const PrefillArgs& a, cudaStream_t s) {
+                     const CUtensorMap& to, const CUtensorMap& tk16, const CUtensorMap& tv16,
+                     const PrefillArgs& a, cudaStream_t s) {
   if (a.bound)
-    return a.stagger ? launch_ds<D, true, true>(tq, tk, tv, to, a, s) : launch_ds<D, false, true>(tq, tk, tv, to, a, s);
-  return a.stagger ? launch_ds<D, true, false>(tq, tk, tv, to, a, s) : launch_ds<D, false, false>(tq, tk, tv, to, a, s);
+    return a.stagger ? launch_ds<D, true, true>(tq, tk, tv, to, tk16, tv16, a, s)
+                     : launch_ds<D, false, true>(tq, tk, tv, to, tk16, tv16, a, s);
+  return a.stagger ? launch_ds<D, true, false>(tq, tk, tv, to, tk16, tv16, a, s)
+                   : launch_ds<D, false, false>(tq, tk, tv, to, tk16, tv16, a, s);
 }
 
 }  // namespace
@@ -734,10 +754,10 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 int prefill_bf16_smem_bytes(int d) { return d == 64 ? Cfg<64>::kSmem : Cfg<128>::kSmem; }
 
 cudaError_t launch_prefill_bf16(int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                                const CUtensorMap& tv, const CUtensorMap& to, const PrefillArgs& a,
-                                cudaStream_t s) {
-  if (d == 64) return launch_d<64>(tq, tk, tv, to, a, s);
-  return launch_d<128>(tq, tk, tv, to, a, s);
+                                const CUtensorMap& tv, const CUtensorMap& to, const CUtensorMap& tk16,
+                                const CUtensorMap& tv16, const PrefillArgs& a, cudaStream_t s) {
+  if (d == 64) return launch_d<64>(tq, tk, tv, to, tk16, tv16, a, s);
+  return launch_d<128>(tq, tk, tv, to, tk16, tv16, a, s);
 }
 
 }  // namespace eio
