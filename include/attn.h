@@ -172,7 +172,7 @@ int attn_frame_block_map(int n_frames, int frame_len, uint8_t* out);
  * among live blocks; find a tile size that splits the mask into tiles fully
  * inside or outside it).
  *   out  host, uint8 [ceil(Nq/tq)][ceil(Nkv/tk)]: 0 empty, 1 full, 2 partial.
- *        Edge tiles are judged on their elements inside [0,Nq) x [0,Nkv).
+ *        Edge tiles are classified by their elements inside [0,Nq) x [0,Nkv).
  */
 int attn_classify(int mask_kind, const uint8_t* block_map, int Nq, int Nkv, int tq, int tk,
                   uint8_t* out);
