@@ -628,8 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = row < nrows;
       if constexpr (C::kStageO) {
         // Row -> shared staging (16-byte units XOR-swizzled by row), then
-        // each warp stores its 32 rows as whole lines: 8 lanes per row.
-        constexpr int UPR = D / 8;  // 16-byte units per row
+        // each warp stores its 32 rows as whole lines.
         uint8_t* stg = smem + C::kOffStage + x * (128 * D * 2);
         // The previous item's stores from this buffer must have read it.
         if (lane == 0) bulk_wait_read_all();
