@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
         L.ora_check_schedule.argtypes = [I, P, I, I, P, I, P, I]
         L.ora_allowed.argtypes = [I, P, I, I, I, I]
         L.ora_key_stats.argtypes = [P, I, I, I, I, I, P, P]
+        L.ora_attn_bwd_dq_rows.argtypes = [P, P, P, P, I, I, I, I, I, I, I, D, I, P, P, I, P]
         L.ora_attn_fwd_bound.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, P, P, P, D, P, P, P]
         _lib = L
     return _lib
@@ -255,3 +256,20 @@ def attn_fwd_bound(q, k, v, scale, mask_kind=MASK_NONE, block_map=None, kbar=Non
     if rc != 0:
         raise ValueError("ora_attn_fwd_bound rejected its arguments")
     return o, lse, flags
+
+
+def attn_bwd_dq_rows(q, k, v, dout, scale, rows, mask_kind=MASK_NONE, block_map=None):
+    """dQ of selected query rows (b, hq, i), as attn_bwd defines it, at O(N d)
+    per row: for gradient checks at sizes where the whole gradient is too
+    slow.  Returns [n, d] fp64."""
+    q, k, v, dout = (np.ascontiguousarray(x) for x in (q, k, v, dout))
+    B, Nq, Hq, d = q.shape
+    Nkv, Hkv = k.shape[1], k.shape[2]
+    rows = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 3)
+    out = np.zeros((rows.shape[0], d), np.float64)
+    bm = _bm(block_map)
+    rc = lib().ora_attn_bwd_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _dtype_code(q), B, Hq, Hkv, Nq, Nkv, d,
+                                    float(scale), mask_kind, _ptr(bm), _ptr(rows), rows.shape[0], _ptr(out))
+    if rc != 0:
+        raise ValueError("ora_attn_bwd_dq_rows rejected its arguments")
+    return out

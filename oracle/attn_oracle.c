@@ -602,3 +602,69 @@ int ora_attn_fwd_bound(const void *q, const void *k, const void *v, int dtype, i
   }
   return 0;
 }
+
+/*
+ * dQ for selected query rows only (the same definition as ora_attn_bwd,
+ * restricted to one row: its whole S and P rows, dP_i = dO_i V^T,
+ * D_i = sum_j P_ij dP_ij, dS_i = P_i * (dP_i - D_i), dQ_i = scale dS_i K).
+ * rows: nrows triples (b, hq, i); dq: [nrows][d] fp64.
+ */
+int ora_attn_bwd_dq_rows(const void *q, const void *k, const void *v, const void *dout, int dtype, int B,
+                         int Hq, int Hkv, int Nq, int Nkv, int d, double scale, int mask_kind,
+                         const uint8_t *block_map, const int32_t *rows, int nrows, double *dq) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || Nq <= 0 || Nkv <= 0) return -1;
+  if (mask_kind == ORA_MASK_BLOCK && !block_map) return -1;
+  int G = Hq / Hkv, bad = 0;
+#pragma omp parallel
+  {
+    double *S = (double *)malloc(sizeof(double) * (size_t)Nkv);
+    double *dP = (double *)malloc(sizeof(double) * (size_t)Nkv);
+#pragma omp for schedule(dynamic, 1)
+    for (int r = 0; r < nrows; ++r) {
+      int b = rows[3 * r], hq = rows[3 * r + 1], i = rows[3 * r + 2];
+      double *out = dq + (size_t)r * d;
+      for (int t = 0; t < d; ++t) out[t] = 0.0;
+      if (b < 0 || b >= B || hq < 0 || hq >= Hq || i < 0 || i >= Nq) {
+        bad = 1;
+        continue;
+      }
+      int hkv = hq / G;
+      size_t q_off = (((size_t)b * Nq + i) * Hq + hq) * d;
+      size_t kv_base = ((size_t)b * Nkv * Hkv + hkv) * d, kv_stride = (size_t)Hkv * d;
+      double m = -INFINITY;
+      for (int j = 0; j < Nkv; ++j) {
+        if (!ora_allowed(mask_kind, block_map, Nq, Nkv, i, j)) {
+          S[j] = -INFINITY;
+          continue;
+        }
+        double acc = 0.0;
+        for (int t = 0; t < d; ++t) acc += ld(q, dtype, q_off + t) * ld(k, dtype, kv_base + (size_t)j * kv_stride + t);
+        S[j] = acc * scale;
+        if (S[j] > m) m = S[j];
+      }
+      if (m == -INFINITY) continue; /* no allowed key: zero gradient */
+      double l = 0.0;
+      for (int j = 0; j < Nkv; ++j) {
+        S[j] = S[j] == -INFINITY ? 0.0 : exp(S[j] - m); /* P, unnormalised */
+        l += S[j];
+      }
+      double D = 0.0;
+      for (int j = 0; j < Nkv; ++j) {
+        S[j] /= l;
+        dP[j] = 0.0;
+        if (S[j] == 0.0) continue;
+        for (int t = 0; t < d; ++t)
+          dP[j] += ld(dout, dtype, q_off + t) * ld(v, dtype, kv_base + (size_t)j * kv_stride + t);
+        D += S[j] * dP[j];
+      }
+      for (int j = 0; j < Nkv; ++j) {
+        if (S[j] == 0.0) continue;
+        double ds = S[j] * (dP[j] - D);
+        for (int t = 0; t < d; ++t) out[t] += scale * ds * ld(k, dtype, kv_base + (size_t)j * kv_stride + t);
+      }
+    }
+    free(S);
+    free(dP);
+  }
+  return bad ? -1 : 0;
+}

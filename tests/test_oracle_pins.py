@@ -483,3 +483,25 @@ def test_oracle_gradient_invariants():
     assert not dk[:, 32:48].any() and not dv[:, 32:48].any()
     assert not dq[:, 16:32].any()
     assert dk[:, :32].any() and dq[:, :16].any()
+
+
+@pytest.mark.parametrize("case", [CASES[1], CASES[3], CASES[5]])
+def test_oracle_dq_rows_match_torch_autograd(case):
+    """The per-row dQ (for gradient checks at full size) against torch
+    autograd of SDPA on sampled rows, masks and GQA included."""
+    B, Hq, Hkv, Nq, Nkv, d, kind = case
+    seed = (hash(case) & 0xFFFF) + 29
+    q, k, v = rnd((B, Nq, Hq, d), seed), rnd((B, Nkv, Hkv, d), seed + 1), rnd((B, Nkv, Hkv, d), seed + 2)
+    dout = rnd((B, Nq, Hq, d), seed + 3)
+    bm = None
+    if kind == oracle.MASK_BLOCK:
+        rng = np.random.default_rng(seed)
+        bm = (rng.random(((Nq + 15) // 16, (Nkv + 15) // 16)) < 0.6).astype(np.uint8)
+        bm[:, 0] = 1
+    scale = 1.0 / math.sqrt(d)
+    rq, _, _ = _sdpa_grads(q, k, v, dout, scale, _allowed_matrix(kind, bm, Nq, Nkv))
+    rng = np.random.default_rng(seed)
+    rows = np.stack([rng.integers(0, B, 12), rng.integers(0, Hq, 12), rng.integers(0, Nq, 12)], axis=1).astype(np.int32)
+    got = oracle.attn_bwd_dq_rows(q, k, v, dout, scale, rows, kind, bm)
+    ref = np.stack([rq[b, i, h] for b, h, i in rows])
+    np.testing.assert_allclose(got, ref, atol=1e-11, rtol=1e-10)
