@@ -583,3 +583,44 @@ def test_ulysses_single_rank_uses_the_cuda_forward():
     o1, l1 = ulysses_attention(tq, tk, tv, mask_kind=eio.MASK_CAUSAL)
     eio.sync_status()
     assert torch.equal(o0, o1) and torch.equal(l0, l1)
+
+
+BWD_FULL = [
+    # B, Hq, Hkv, N, d, mask: the GQA causal backward shape and the frame workload at full size
+    (1, 32, 8, 4096, 128, "causal"),
+    (1, 24, 24, 24960, 128, "frames"),
+]
+
+
+@pytest.mark.parametrize("case", BWD_FULL)
+def test_backward_full_size_sampled_rows_and_identities(case):
+    """At full size: dQ on sampled query rows against the oracle's per-row
+    dQ, and two identities over all keys that hold at any size: every row's
+    probabilities sum to one, so sum_j dV_j equals the sum of dO over the
+    rows and query heads of the group; every row's dS sums to zero, so
+    sum_j dK_j = 0 (both per batch element, KV head and column)."""
+    B, Hq, Hkv, N, d, kind = case
+    seed = 3600 + BWD_FULL.index(case)
+    q, k, v = make_inputs(seed, B, Hq, Hkv, N, N, d)
+    dout = synthetic.tensor(seed, 9, (B, N, Hq, d))
+    mk, bm = (eio.MASK_CAUSAL, None) if kind == "causal" else (eio.MASK_BLOCK, eio.frame_block_map(24, 1040))
+    scale = 1 / math.sqrt(d)
+    tq, tk, tv, tdo = dev_bf16(q), dev_bf16(k), dev_bf16(v), dev_bf16(dout)
+    o, lse = eio.attn_fwd(tq, tk, tv, scale=scale, mask_kind=mk, block_map=bm)
+    dq, dk, dv = eio.attn_bwd(tq, tk, tv, o, lse, tdo, scale=scale, mask_kind=mk, block_map=bm)
+    eio.sync_status()
+    rng = np.random.default_rng(seed)
+    rows = np.stack([rng.integers(0, B, 16), rng.integers(0, Hq, 16), rng.integers(0, N, 16)], axis=1).astype(np.int32)
+    rows[0] = (0, 0, 0)
+    rows[1] = (B - 1, Hq - 1, N - 1)
+    ref = oracle.attn_bwd_dq_rows(q, k, v, dout, scale, rows, mk, bm)
+    got = np.stack([host_f64(dq[b, i, h]) for b, h, i in rows])
+    check_grad(torch.from_numpy(got), ref, f"{case} dq rows")
+    G = Hq // Hkv
+    do64 = synthetic.bf16_bits_to_f32(dout).astype(np.float64).reshape(B, N, Hkv, G, d)
+    want_dv = do64.sum(axis=(1, 3))                      # [B, Hkv, d]
+    dv64, dk64 = host_f64(dv), host_f64(dk)
+    err_v = np.abs(dv64.sum(axis=1) - want_dv)
+    assert (err_v <= 4e-3 * np.abs(dv64).sum(axis=1) + 1e-3).all(), err_v.max()
+    err_k = np.abs(dk64.sum(axis=1))
+    assert (err_k <= 4e-3 * np.abs(dk64).sum(axis=1) + 1e-3).all(), err_k.max()
