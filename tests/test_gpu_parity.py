@@ -624,3 +624,29 @@ def test_backward_full_size_sampled_rows_and_identities(case):
     assert (err_v <= 4e-3 * np.abs(dv64).sum(axis=1) + 1e-3).all(), err_v.max()
     err_k = np.abs(dk64.sum(axis=1))
     assert (err_k <= 4e-3 * np.abs(dk64).sum(axis=1) + 1e-3).all(), err_k.max()
+
+
+@pytest.mark.parametrize("which", ["long", "frame"])
+def test_bound_forward_full_size_d128(which):
+    """The bound-based forward (key statistics + attn_fwd_bound) on the two
+    d = 128 workloads at full size, sampled rows against the oracle; no row
+    needs the fallback on these inputs (the oracle's rule agrees)."""
+    if which == "long":
+        B, Hq, Hkv, N, mk, bm, obm = 1, 32, 8, 16384, eio.MASK_CAUSAL, None, None
+    else:
+        B, Hq, Hkv, N, mk = 1, 24, 24, 24 * 1040, eio.MASK_BLOCK
+        bm, obm = eio.frame_block_map(24, 1040), oracle.frame_block_map(24, 1040)
+    d = 128
+    q, k, v = make_inputs(1003 if which == "long" else 1004, B, Hq, Hkv, N, N, d)
+    tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    kbar, radius = eio.key_stats(tk)
+    nfb = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = eio.attn_fwd_bound(tq, tk, tv, kbar, radius, mask_kind=mk, block_map=bm, n_fallback=nfb)
+    eio.sync_status()
+    assert int(nfb.item()) == 0
+    rk, rr = oracle.key_stats(k)
+    np.testing.assert_allclose(kbar.cpu().numpy(), rk, atol=2e-5, rtol=1e-5)
+    np.testing.assert_allclose(radius.cpu().numpy(), rr, rtol=1e-5)
+    rows = sampled_rows(np.random.default_rng(7), B, Hq, N, [0, 127, 128, N - 1], 80)
+    ro, rl = oracle.attn_rows(q, k, v, 1 / math.sqrt(d), rows, mk, obm)
+    check_rows(o, lse, ro, rl, rows, f"bound {which}")
