@@ -6,7 +6,8 @@ seed, so every run checks the same shapes) over the whole supported range:
 batch, query heads per KV head (including odd groups), ragged lengths with
 Nq != Nkv in both directions, d in {64, 128}, every mask kind, block maps of
 varying density with empty block rows, decode lengths of zero, and
-multi-token decode.  The tolerances are those of the other parity tests.
+multi-token decode.  Two sets: a quick one (sequences up to 700) and a
+larger one (up to 1500).  The tolerances are those of the other parity tests.
 """
 import math
 
@@ -22,7 +23,8 @@ from tests.test_gpu_parity import (check, check_grad, dev_bf16, make_inputs, ora
 
 pytestmark = pytest.mark.gpu
 
-SEED = 20240611
+SEED = 20240611      # the quick set
+SEED_LARGE = 777001  # the larger set
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -44,7 +46,7 @@ def _block_map(rng, Nq, Nkv):
     return bm
 
 
-def _fwd_cases(n, seed, nmax, groups, kinds):
+def _fwd_cases(n, seed, nmax, groups, kinds, base):
     rng = np.random.default_rng(seed)
     out = []
     for i in range(n):
@@ -54,12 +56,12 @@ def _fwd_cases(n, seed, nmax, groups, kinds):
         B = int(rng.integers(1, 4))
         Nq, Nkv = (int(x) for x in rng.integers(1, nmax, size=2))
         kind = str(rng.choice(kinds))
-        out.append((i, B, G * Hkv, Hkv, Nq, Nkv, d, kind))
+        out.append((base, i, B, G * Hkv, Hkv, Nq, Nkv, d, kind))
     return out
 
 
 def _ids(cases):
-    return [f"{c[-1]}-b{c[1]}h{c[2]}g{c[2] // c[3]}-{c[4]}x{c[5]}-d{c[6]}" for c in cases]
+    return [f"{c[0]}-{c[-1]}-b{c[2]}h{c[3]}g{c[3] // c[4]}-{c[5]}x{c[6]}-d{c[7]}" for c in cases]
 
 
 def _mask(kind, rng, Nq, Nkv):
@@ -70,14 +72,15 @@ def _mask(kind, rng, Nq, Nkv):
     return eio.MASK_BLOCK, _block_map(rng, Nq, Nkv)
 
 
-FWD = _fwd_cases(24, SEED, 700, [1, 2, 3, 4, 8], ["none", "causal", "block"])
+FWD = (_fwd_cases(24, SEED, 700, [1, 2, 3, 4, 8], ["none", "causal", "block"], SEED) +
+       _fwd_cases(120, SEED_LARGE, 1500, [1, 2, 3, 4, 8], ["none", "causal", "block"], SEED_LARGE))
 
 
 @pytest.mark.parametrize("case", FWD, ids=_ids(FWD))
 def test_fuzz_forward_bf16(case):
-    i, B, Hq, Hkv, Nq, Nkv, d, kind = case
-    rng = np.random.default_rng(SEED + 1000 + i)
-    q, k, v = make_inputs(SEED + i, B, Hq, Hkv, Nq, Nkv, d)
+    base, i, B, Hq, Hkv, Nq, Nkv, d, kind = case
+    rng = np.random.default_rng(base + 1000 + i)
+    q, k, v = make_inputs(base + i, B, Hq, Hkv, Nq, Nkv, d)
     mk, bm = _mask(kind, rng, Nq, Nkv)
     scale = float(rng.uniform(0.5, 1.5)) / math.sqrt(d)
     o, lse = run_fwd(q, k, v, scale, mk, bm)
@@ -85,15 +88,15 @@ def test_fuzz_forward_bf16(case):
     check(o, lse, ro, rl, f"fwd {case}")
 
 
-FWD32 = [(i, *c[1:4], c[4], c[5], int(np.random.default_rng(SEED + 50 + i).choice([32, 64, 128])), c[7])
-         for i, c in enumerate(_fwd_cases(6, SEED + 50, 300, [1, 2, 4], ["none", "causal", "block"]))]
+FWD32 = [(*c[:7], int(np.random.default_rng(SEED + 50 + c[1]).choice([32, 64, 128])), c[8])
+         for c in _fwd_cases(6, SEED + 50, 300, [1, 2, 4], ["none", "causal", "block"], SEED)]
 
 
 @pytest.mark.parametrize("case", FWD32, ids=_ids(FWD32))
 def test_fuzz_forward_fp32(case):
-    i, B, Hq, Hkv, Nq, Nkv, d, kind = case
-    rng = np.random.default_rng(SEED + 2000 + i)
-    q, k, v = make_inputs(SEED + 100 + i, B, Hq, Hkv, Nq, Nkv, d, "f32")
+    base, i, B, Hq, Hkv, Nq, Nkv, d, kind = case
+    rng = np.random.default_rng(base + 2000 + i)
+    q, k, v = make_inputs(base + 100 + i, B, Hq, Hkv, Nq, Nkv, d, "f32")
     mk, bm = _mask(kind, rng, Nq, Nkv)
     scale = 1 / math.sqrt(d)
     o, lse = run_fwd(q, k, v, scale, mk, bm)
@@ -101,7 +104,7 @@ def test_fuzz_forward_fp32(case):
     check(o, lse, ro, rl, f"fwd32 {case}")
 
 
-def _decode_cases(n, seed):
+def _decode_cases(n, seed, base):
     rng = np.random.default_rng(seed)
     out = []
     for i in range(n):
@@ -116,18 +119,19 @@ def _decode_cases(n, seed):
             lens[int(rng.integers(0, B))] = 0
         if rng.random() < 0.3:
             lens[int(rng.integers(0, B))] = Lmax
-        out.append((i, B, Sq, G * Hkv, Hkv, Lmax, d, tuple(int(x) for x in lens)))
+        out.append((base, i, B, Sq, G * Hkv, Hkv, Lmax, d, tuple(int(x) for x in lens)))
     return out
 
 
-DEC = _decode_cases(14, SEED + 7)
+DEC = _decode_cases(14, SEED + 7, SEED) + _decode_cases(50, SEED_LARGE + 1, SEED_LARGE)
 
 
-@pytest.mark.parametrize("case", DEC, ids=[f"b{c[1]}s{c[2]}h{c[3]}g{c[3] // c[4]}-L{c[5]}-d{c[6]}" for c in DEC])
+@pytest.mark.parametrize("case", DEC,
+                         ids=[f"{c[0]}-b{c[2]}s{c[3]}h{c[4]}g{c[4] // c[5]}-L{c[6]}-d{c[7]}" for c in DEC])
 def test_fuzz_decode(case):
-    i, B, Sq, Hq, Hkv, Lmax, d, lens = case
+    base, i, B, Sq, Hq, Hkv, Lmax, d, lens = case
     lens = np.array(lens, np.int32)
-    seed = SEED + 300 + i
+    seed = base + 300 + i
     scale = 1 / math.sqrt(d)
     kc = synthetic.kv_cache(seed, synthetic.TID_K, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)  # NaN past len
     vc = synthetic.kv_cache(seed, synthetic.TID_V, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
@@ -144,16 +148,17 @@ def test_fuzz_decode(case):
     check(o, lse, ro, rl, f"decode {case}")
 
 
-BWD = _fwd_cases(10, SEED + 11, 400, [1, 2, 3, 4], ["none", "causal", "block"])
+BWD = (_fwd_cases(10, SEED + 11, 400, [1, 2, 3, 4], ["none", "causal", "block"], SEED) +
+       _fwd_cases(30, SEED_LARGE + 2, 700, [1, 2, 3, 4], ["none", "causal", "block"], SEED_LARGE))
 
 
 @pytest.mark.parametrize("case", BWD, ids=_ids(BWD))
 def test_fuzz_backward(case):
-    i, B, Hq, Hkv, Nq, Nkv, d, kind = case
+    base, i, B, Hq, Hkv, Nq, Nkv, d, kind = case
     B = min(B, 2)
-    rng = np.random.default_rng(SEED + 3000 + i)
-    q, k, v = make_inputs(SEED + 400 + i, B, Hq, Hkv, Nq, Nkv, d)
-    dout = synthetic.tensor(SEED + 400 + i, 9, (B, Nq, Hq, d))
+    rng = np.random.default_rng(base + 3000 + i)
+    q, k, v = make_inputs(base + 400 + i, B, Hq, Hkv, Nq, Nkv, d)
+    dout = synthetic.tensor(base + 400 + i, 9, (B, Nq, Hq, d))
     mk, bm = _mask(kind, rng, Nq, Nkv)
     scale = 1 / math.sqrt(d)
     tq, tk, tv, tdo = dev_bf16(q), dev_bf16(k), dev_bf16(v), dev_bf16(dout)
@@ -166,14 +171,15 @@ def test_fuzz_backward(case):
     check_grad(dv, rv, f"{case} dv")
 
 
-BOUND = _fwd_cases(8, SEED + 13, 600, [1, 2, 4, 8], ["none", "causal", "block"])
+BOUND = (_fwd_cases(8, SEED + 13, 600, [1, 2, 4, 8], ["none", "causal", "block"], SEED) +
+         _fwd_cases(25, SEED_LARGE + 3, 1000, [1, 2, 4, 8], ["none", "causal", "block"], SEED_LARGE))
 
 
 @pytest.mark.parametrize("case", BOUND, ids=_ids(BOUND))
 def test_fuzz_bound_forward(case):
-    i, B, Hq, Hkv, Nq, Nkv, d, kind = case
-    rng = np.random.default_rng(SEED + 4000 + i)
-    q, k, v = make_inputs(SEED + 500 + i, B, Hq, Hkv, Nq, Nkv, d)
+    base, i, B, Hq, Hkv, Nq, Nkv, d, kind = case
+    rng = np.random.default_rng(base + 4000 + i)
+    q, k, v = make_inputs(base + 500 + i, B, Hq, Hkv, Nq, Nkv, d)
     # keys offset by a random vector, so that the centring matters
     shift = rng.standard_normal(d).astype(np.float32)
     k = synthetic.f32_to_bf16_bits(synthetic.bf16_bits_to_f32(k) + shift)
