@@ -228,3 +228,32 @@ def test_backward_bound_and_stats_argument_errors():
     assert fb(mask=2) == 5
     assert fb(kbar=FAKE + 4) == 3
     assert fb(nfb=FAKE + 2) == 3
+
+
+# ------------------------------------------------------- binding checks
+def test_binding_rejects_block_maps_of_the_wrong_size():
+    """The library reads ceil(Nq/16) x ceil(Nkv/16) bytes of the map: the
+    binding refuses any other shape instead of letting it read past the end."""
+    bm = np.ones((3, 4), np.uint8)
+    qt, _ = eio.plan(oracle.MASK_BLOCK, bm, 48, 64)  # 3 x 4 blocks: accepted
+    assert len(qt) == 1
+    for Nq, Nkv in [(49, 64), (48, 65), (32, 64), (48, 48)]:
+        with pytest.raises(ValueError, match="block_map"):
+            eio.plan(oracle.MASK_BLOCK, bm, Nq, Nkv)
+        with pytest.raises(ValueError, match="block_map"):
+            eio.classify(oracle.MASK_BLOCK, bm, Nq, Nkv, 16, 16)
+
+
+def test_binding_rejects_host_tensors():
+    """Device entry points take CUDA tensors only; a host tensor is refused
+    before any pointer reaches the library."""
+    import torch
+    x = torch.zeros(1, 16, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        eio.attn_fwd(x, x, x)
+    with pytest.raises(ValueError, match="CUDA"):
+        eio.attn_bwd(x, x, x, x, torch.zeros(1, 2, 16), x)
+    with pytest.raises(ValueError, match="CUDA"):
+        eio.key_stats(x)
+    with pytest.raises(ValueError, match="CUDA"):
+        eio.attn_decode(x[0], x, x, torch.zeros(1, dtype=torch.int32))

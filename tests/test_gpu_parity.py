@@ -357,6 +357,32 @@ def test_decode_multi_token(case):
     check(o, lse, ro, rl, str(case))
 
 
+def test_binding_rejects_mis_shaped_tensors():
+    """Outputs, statistics and lengths of the wrong shape, dtype or layout
+    raise ValueError before any launch (the C ABI cannot see their sizes)."""
+    B, N, H, d = 1, 64, 2, 64
+    q = dev_bf16(synthetic.tensor(1, 1, (B, N, H, d)))
+    with pytest.raises(ValueError, match="lse"):
+        eio.attn_fwd(q, q, q, lse=torch.empty(B, H, N - 1, device="cuda"))
+    with pytest.raises(ValueError, match="o has dtype"):
+        eio.attn_fwd(q, q, q, o=torch.empty(B, N, H, d, device="cuda"))
+    with pytest.raises(ValueError, match="contiguous"):
+        eio.attn_fwd(q, q.transpose(1, 2).contiguous().transpose(1, 2), q)
+    with pytest.raises(ValueError, match="k has shape"):
+        eio.attn_fwd(q, q[..., :32].contiguous(), q)
+    with pytest.raises(ValueError, match="kbar"):
+        eio.key_stats(q, kbar=torch.empty(B, H, d + 1, device="cuda"))
+    kbar, radius = eio.key_stats(q)
+    with pytest.raises(ValueError, match="radius"):
+        eio.attn_fwd_bound(q, q, q, kbar, radius.double())
+    qd = q[:, 0].contiguous()
+    with pytest.raises(ValueError, match="seqlens"):
+        eio.attn_decode(qd, q, q, torch.full((B,), N, dtype=torch.int64, device="cuda"))
+    with pytest.raises(ValueError, match="lse"):
+        eio.attn_bwd(q, q, q, q, torch.empty(B, H, N, dtype=torch.float16, device="cuda"), q)
+    eio.sync_status()
+
+
 def test_decode_multi_equals_single_at_sq1():
     B, Hq, Hkv, Lmax, d = 4, 8, 2, 900, 128
     lens = np.array([900, 1, 511, 512], np.int32)
