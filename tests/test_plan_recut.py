@@ -21,3 +21,17 @@ def test_two_segment_recut_covers_the_plan(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "bad 0" in r.stdout
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+def test_pair_plans_keep_the_kernel_invariants(tmp_path):
+    """tests/plan_pairs_check.cpp: over random shapes of every mask kind and
+    both pairing modes, each Q tile runs exactly once, each slot visits
+    exactly its own keys (slot A a prefix of the shared list), partial flags
+    are per slot, and the visit order is longest first."""
+    exe = tmp_path / "pairs_check"
+    subprocess.run(["g++", "-O2", "-std=c++17", "-I", CSRC, os.path.join(ROOT, "tests", "plan_pairs_check.cpp"),
+                    os.path.join(CSRC, "plan.cpp"), "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.startswith("bad 0")
