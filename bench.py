@@ -106,9 +106,35 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def _code_only(src: str) -> str:
+    """C/C++ source with comments removed and whitespace runs collapsed, so
+    that an edit to comments or layout alone does not count as a change."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":  # string or character literal: kept whole
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def kernel_source_sha(fn):
-    """Hash of a kernel source together with the local headers it includes
-    (recursively), so that a change to a shared device helper also counts."""
+    """Hash of a kernel's code together with the local headers it includes
+    (recursively), so that a change to a shared device helper also counts;
+    comments and whitespace are excluded (see _code_only)."""
     csrc = os.path.join(ROOT, "exact_io_aware_sm_b200", "csrc")
     h, seen, todo = hashlib.sha256(), set(), [fn]
     while todo:
@@ -118,9 +144,9 @@ def kernel_source_sha(fn):
             continue
         seen.add(name)
         with open(path, "rb") as f:
-            data = f.read()
-        h.update(name.encode() + b"\0" + data)
-        todo += re.findall(r'^#include "([^"/]+)"', data.decode(), flags=re.M)
+            data = f.read().decode()
+        h.update(name.encode() + b"\0" + _code_only(data).encode())
+        todo += re.findall(r'^#include "([^"/]+)"', data, flags=re.M)
     return h.hexdigest()[:16]
 
 
