@@ -26,8 +26,8 @@
 //   warps 8..11   softmax for slot B.
 // Each softmax thread loads its whole S row from TMEM (one wait), takes the
 // row max, keeps the running max m and sum l (online softmax: FlashAttention
-// page section 2, inference page "Online-Softmax"), packs P to bf16 in place
-// and writes it back over the first 64 columns of its own S row, where the PV
+// page section 2, inference page "Online-Softmax"), packs P to bf16 in
+// registers and writes it to TMEM (64 columns of bf16 pairs), where the PV
 // MMA reads it.  At the end of an item it writes O / l (bf16) and LSE.
 //
 // The exponent base moves only when a tile's row max exceeds it by more than
@@ -35,8 +35,11 @@
 // base, so the result is exactly softmax(S) V while most rescales vanish.
 //
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+d), O_B after O_A.
-// P_X is stored as bf16 pairs in S_X's first 64 columns; the MMA issuer
-// orders S_X(j+1) after PV_X(j) has completed, since they share columns.
+// d = 128: P_X overwrites the first 64 columns of S_X, so the MMA issuer
+// orders S_X(j+1) after PV_X(j) has completed.  d = 64 leaves 128 columns
+// free: P_A [384,448) and P_B [448,512) have their own, and S_X(j+1) is
+// issued as soon as the softmax threads have loaded S_X(j) into registers,
+// so it overlaps their exponentials.
 #include <cuda_bf16.h>
 
 #include "fastmath.cuh"
