@@ -30,6 +30,13 @@
 // S and dP are recomputed by both kernels (seven products instead of five)
 // so that neither needs atomics or a second pass over an fp32 dQ.
 //
+// Masks: none; causal (bottom-right aligned, diagonal tiles masked by index);
+// and 16 x 16 block maps, for which the host lists, per Q tile and per key
+// tile, the tiles of the other kind that hold an allowed block, each with the
+// 64-bit bitmap of its 8 x 8 allowed blocks: tiles without one are never
+// visited, and the bitmap masks the blocks of a visited tile that are not
+// allowed.
+//
 // Across items: the producer loads the next item's resident tiles as soon as
 // the current item's last S / dP MMAs have read them, its first stream tiles
 // queue in the ring behind the current ones, and the next item's first S and

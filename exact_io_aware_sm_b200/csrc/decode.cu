@@ -1,8 +1,11 @@
-// decode.cu -- single-token GQA decode over a KV cache, split along the keys.
+// decode.cu -- GQA decode of the newest token (or the Sq newest tokens) of
+// each sequence over a KV cache, split along the keys.
 //
-// Decode reads the whole cache once per step and does about 2 FLOPs per byte
-// (inference page, "Why Decode is Memory-bound"), so this path is built to
-// keep HBM streaming and to spend as few instructions per byte as possible:
+// Decode reads the whole cache once per step and does little arithmetic per
+// byte (inference page, "Why Decode is Memory-bound"): 4d FLOPs per query
+// head per cached key against 4d bytes of K and V, i.e. G FLOPs per byte for
+// G query heads per KV head (times Sq for Sq tokens).  So this path is built
+// to keep HBM streaming and to spend as few instructions per byte as possible:
 //
 //   decode_split_kernel   persistent, one CTA per SM, four warps.  A work
 //     item is (sequence b, KV head, split of 512 keys), for the Sq newest
@@ -21,7 +24,7 @@
 //       O^T (d x 8 columns) += V^T (d x 16) P^T       V by ldmatrix.trans, P^T by movmatrix
 //     Columns past G * Sq are zero.  The output is a normalised partial O
 //     and its log2-sum-exp per (sequence, query head, split).
-//   decode_combine_kernel  one CTA per (sequence, query head): merges the
+//   decode_combine_kernel  one CTA per (sequence, token, query head): merges the
 //     splits with the block rule of the FlashAttention page, section 2
 //     (rescale each part by 2^(lse_s - lse)), writes O (bf16) and LSE
 //     (natural log).
