@@ -13,11 +13,15 @@ NVLink / NVSwitch on GPUs, gloo on CPU) issued asynchronously; the attention
 is `attn_fwd` of this package unless another callable is given.  Nothing here
 reads a peer's memory directly.
 
-Layouts (per rank r of P): q [B, N/P, Hq, d], k and v [B, N/P, Hkv, d], rank r
-holding sequence rows [r N/P, (r+1) N/P); the result o [B, N/P, Hq, d] and
-lse [B, Hq, N/P] for the same rows.  Query head h lives on rank h // (Hq/P)
-during attention, KV head g on rank g // (Hkv/P), so GQA groups stay whole
-when Hkv % P == 0.
+Layouts (per rank r of P): q [B, N_r, Hq, d], k and v [B, N_r, Hkv, d], rank r
+holding the contiguous sequence rows that follow those of ranks 0..r-1; the
+result o [B, N_r, Hq, d] and lse [B, Hq, N_r] for the same rows.  The shards
+may differ in length (N = sum of N_r): each is padded to the longest for the
+exchange, the padding is dropped before attention (which sees exactly the N
+rows, so masks and the LSE are those of the unsharded sequence) and restored
+for the return exchange.  Query head h lives on rank h // (Hq/P) during
+attention, KV head g on rank g // (Hkv/P), so GQA groups stay whole when
+Hkv % P == 0.
 """
 from __future__ import annotations
 
@@ -53,14 +57,36 @@ def default_attention(q, k, v, mask_kind, scale):
     return attn_fwd(q.contiguous(), k.contiguous(), v.contiguous(), scale=scale, mask_kind=mask_kind)
 
 
-def ulysses_attention(q, k, v, group=None, mask_kind=0, scale=None, head_groups=1, attention=None):
+def _shard_lens(Nl, P, group, device):
+    """Every rank's shard length (one small all-gather)."""
+    import torch
+    import torch.distributed as dist
+    mine = torch.tensor([Nl], dtype=torch.int64, device=device)
+    allv = [torch.zeros_like(mine) for _ in range(P)]
+    dist.all_gather(allv, mine, group=group)
+    return [int(t.item()) for t in allv]
+
+
+def _pad_rows(x, n):
+    """[B, Nl, ...] -> [B, n, ...] with zero rows appended (x itself if Nl == n)."""
+    import torch
+    if x.shape[1] == n:
+        return x
+    pad = torch.zeros((x.shape[0], n - x.shape[1]) + tuple(x.shape[2:]), dtype=x.dtype, device=x.device)
+    return torch.cat([x, pad], dim=1)
+
+
+def ulysses_attention(q, k, v, group=None, mask_kind=0, scale=None, head_groups=1, attention=None,
+                      shard_lens=None):
     """Sequence-parallel attention over the ranks of `group` (the default
     process group if None).  Returns (o, lse) for this rank's rows.
 
     attention(q, k, v, mask_kind, scale) -> (o [B,N,H,d], lse [B,H,N]) runs on
     whole sequences; the default is this package's attn_fwd (bf16 CUDA
     tensors).  mask_kind is NONE or CAUSAL: the whole sequence is present on
-    every rank, so a causal mask needs no change."""
+    every rank, so a causal mask needs no change.  shard_lens: every rank's
+    number of rows, in rank order, if the caller knows them (else they are
+    gathered; shards of equal length need no padding)."""
     import torch
     import torch.distributed as dist
 
@@ -73,6 +99,17 @@ def ulysses_attention(q, k, v, group=None, mask_kind=0, scale=None, head_groups=
     _check(B, Nl, Hq, Hkv, P, head_groups)
     if P == 1:
         return attention(q, k, v, mask_kind, scale)
+    lens = list(shard_lens) if shard_lens is not None else _shard_lens(Nl, P, group, q.device)
+    me = dist.get_rank(group)
+    if len(lens) != P or lens[me] != Nl:
+        raise ValueError(f"shard_lens {lens} does not match this rank's {Nl} rows")
+    Np = max(lens)  # every shard padded to this many rows for the exchanges
+    ragged = any(n != Np for n in lens)
+    # rows of the padded, gathered sequence that hold real rows, in sequence order
+    keep = None
+    if ragged:
+        keep = torch.cat([torch.arange(j * Np, j * Np + n, device=q.device) for j, n in enumerate(lens)])
+        q, k, v = (_pad_rows(t, Np) for t in (q, k, v))
     ng = head_groups
     Hqg, Hkg = Hq // P // ng, Hkv // P // ng
 
@@ -90,17 +127,25 @@ def ulysses_attention(q, k, v, group=None, mask_kind=0, scale=None, head_groups=
         for w in works[g]:
             w.wait()
         qg, kg, vg = (_from_seq(r_) for r_ in recvs[g])
+        if ragged:  # drop the padding: attention sees exactly the N rows
+            qg, kg, vg = (t.index_select(1, keep).contiguous() for t in (qg, kg, vg))
         o_g, lse_g = attention(qg, kg, vg, mask_kind, scale)  # [B, N, Hqg, d], [B, Hqg, N]
-        o_send = o_g.view(B, P, Nl, Hqg, d).permute(1, 0, 2, 3, 4).contiguous()
-        l_send = lse_g.view(B, Hqg, P, Nl).permute(2, 0, 1, 3).contiguous()
+        if ragged:  # back to the padded layout for the return exchange
+            o_p = torch.zeros((B, P * Np, Hqg, d), dtype=o_g.dtype, device=o_g.device)
+            o_p[:, keep] = o_g
+            l_p = torch.zeros((B, Hqg, P * Np), dtype=lse_g.dtype, device=lse_g.device)
+            l_p[:, :, keep] = lse_g
+            o_g, lse_g = o_p, l_p
+        o_send = o_g.view(B, P, Np, Hqg, d).permute(1, 0, 2, 3, 4).contiguous()
+        l_send = lse_g.view(B, Hqg, P, Np).permute(2, 0, 1, 3).contiguous()
         o_recv, l_recv = torch.empty_like(o_send), torch.empty_like(l_send)
         out_works.append((dist.all_to_all_single(o_recv, o_send, group=group, async_op=True),
                           dist.all_to_all_single(l_recv, l_send, group=group, async_op=True)))
         out_bufs.append((o_send, l_send, o_recv, l_recv))
     # 3. reassemble this rank's rows: chunk i of group g holds query heads
     #    i*Hq/P + g*Hqg .. of every row here
-    o = torch.empty((B, Nl, P, ng, Hqg, d), dtype=q.dtype, device=q.device)
-    lse = torch.empty((B, P, ng, Hqg, Nl), dtype=torch.float32 if q.is_cuda else out_bufs[0][3].dtype,
+    o = torch.empty((B, Np, P, ng, Hqg, d), dtype=q.dtype, device=q.device)
+    lse = torch.empty((B, P, ng, Hqg, Np), dtype=torch.float32 if q.is_cuda else out_bufs[0][3].dtype,
                       device=q.device)
     for g in range(ng):
         for w in out_works[g]:
@@ -108,4 +153,7 @@ def ulysses_attention(q, k, v, group=None, mask_kind=0, scale=None, head_groups=
         o_recv, l_recv = out_bufs[g][2], out_bufs[g][3]
         o[:, :, :, g] = o_recv.permute(1, 2, 0, 3, 4)
         lse[:, :, g] = l_recv.permute(1, 0, 2, 3).to(lse.dtype)
-    return o.view(B, Nl, Hq, d), lse.view(B, Hq, Nl)
+    o, lse = o.view(B, Np, Hq, d), lse.view(B, Hq, Np)
+    if ragged:
+        o, lse = o[:, :Nl].contiguous(), lse[:, :, :Nl].contiguous()
+    return o, lse

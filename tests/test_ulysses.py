@@ -41,7 +41,7 @@ def _inputs(B, N, Hq, Hkv, d):
     return q, k, v
 
 
-def _rank_main(rank, world, port, shape, mask_kind, groups, out_q):
+def _rank_main(rank, world, port, shape, mask_kind, groups, out_q, lens=None, pass_lens=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import torch.distributed as dist
 
@@ -50,21 +50,23 @@ def _rank_main(rank, world, port, shape, mask_kind, groups, out_q):
     try:
         B, N, Hq, Hkv, d = shape
         q, k, v = _inputs(B, N, Hq, Hkv, d)
-        Nl = N // world
-        sl = slice(rank * Nl, (rank + 1) * Nl)
+        lens = lens or [N // world] * world
+        r0 = sum(lens[:rank])
+        sl = slice(r0, r0 + lens[rank])
         tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x[:, sl])) for x in (q, k, v))
         o, lse = ulysses_attention(tq, tk, tv, mask_kind=mask_kind, scale=1 / math.sqrt(d), head_groups=groups,
-                                   attention=_oracle_attention)
+                                   attention=_oracle_attention, shard_lens=lens if pass_lens else None)
         out_q.put((rank, o.numpy(), lse.numpy()))
     finally:
         dist.destroy_process_group()
 
 
-def _run(world, shape, mask_kind, groups):
+def _run(world, shape, mask_kind, groups, lens=None, pass_lens=False):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, shape, mask_kind, groups, q)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, shape, mask_kind, groups, q, lens, pass_lens))
+             for r in range(world)]
     for p in procs:
         p.start()
     got = dict()
@@ -90,6 +92,26 @@ def test_ulysses_equals_unsharded_attention(world, shape, mask_kind, groups):
     o, lse = _run(world, shape, mask_kind, groups)
     q, k, v = _inputs(B, N, Hq, Hkv, d)
     ro, rlse = oracle.attn_fwd(q, k, v, 1 / math.sqrt(d), mask_kind)
+    np.testing.assert_allclose(o, ro, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(lse, rlse, atol=1e-13, rtol=0)
+
+
+@pytest.mark.parametrize("world,shape,mask_kind,groups,lens,pass_lens", [
+    (2, (1, 61, 4, 2, 8), 1, 1, [33, 28], False),     # causal, last shard shorter, lengths gathered
+    (2, (2, 40, 4, 4, 8), 0, 2, [9, 31], True),       # first shard shorter, lengths given, two groups
+    (3, (1, 50, 6, 3, 8), 1, 1, [20, 1, 29], False),  # three ranks, one holding a single row
+])
+def test_ulysses_uneven_shards(world, shape, mask_kind, groups, lens, pass_lens):
+    """Shards of different lengths: padded for the exchanges, the padding is
+    never attended (keys) nor returned (rows), so the gathered result equals
+    attention on the unsharded sequence."""
+    import oracle
+    B, N, Hq, Hkv, d = shape
+    assert sum(lens) == N
+    o, lse = _run(world, shape, mask_kind, groups, lens, pass_lens)
+    q, k, v = _inputs(B, N, Hq, Hkv, d)
+    ro, rlse = oracle.attn_fwd(q, k, v, 1 / math.sqrt(d), mask_kind)
+    assert o.shape == ro.shape and lse.shape == rlse.shape
     np.testing.assert_allclose(o, ro, atol=1e-13, rtol=0)
     np.testing.assert_allclose(lse, rlse, atol=1e-13, rtol=0)
 
