@@ -157,3 +157,107 @@ def ulysses_attention(q, k, v, group=None, mask_kind=0, scale=None, head_groups=
     if ragged:
         o, lse = o[:, :Nl].contiguous(), lse[:, :, :Nl].contiguous()
     return o, lse
+
+
+def _lse_to_heads(lse, P, g, ng):
+    """[B, H, Nl] -> send buffer [P, B, Hg, Nl]: chunk i holds head group g of
+    the heads rank i will own."""
+    B, H, Nl = lse.shape
+    Hp = H // P
+    Hg = Hp // ng
+    return lse.view(B, P, Hp, Nl)[:, :, g * Hg:(g + 1) * Hg, :].permute(1, 0, 2, 3).contiguous()
+
+
+def _lse_from_seq(buf):
+    """receive buffer [P, B, Hg, Nl] (chunk j = rank j's rows) -> [B, Hg, P*Nl]."""
+    P, B, Hg, Nl = buf.shape
+    return buf.permute(1, 2, 0, 3).reshape(B, Hg, P * Nl)
+
+
+def default_backward(q, k, v, o, lse, dout, mask_kind, scale):
+    from . import attn_bwd
+    c = [t.contiguous() for t in (q, k, v, o, lse, dout)]
+    return attn_bwd(*c, scale=scale, mask_kind=mask_kind)
+
+
+def ulysses_attention_bwd(q, k, v, o, lse, dout, group=None, mask_kind=0, scale=None, head_groups=1,
+                          backward=None, shard_lens=None):
+    """Gradients of ulysses_attention for this rank's rows: q, o, dout
+    [B, N_r, Hq, d], k, v [B, N_r, Hkv, d], lse [B, Hq, N_r] as the forward
+    returned them.  Returns (dq, dk, dv) shaped like q, k, v.
+
+    The same exchanges as the forward: every input goes from sequence shards
+    to head shards, backward(q, k, v, o, lse, dout, mask_kind, scale) ->
+    (dq, dk, dv) runs on whole sequences (default: this package's attn_bwd,
+    which recomputes P from the LSE), and the gradients return to the rows'
+    owners; head groups overlap one group's exchanges with another's
+    backward, and uneven shards are padded as in the forward."""
+    import torch
+    import torch.distributed as dist
+
+    P = dist.get_world_size(group) if dist.is_initialized() else 1
+    B, Nl, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    backward = backward or default_backward
+    _check(B, Nl, Hq, Hkv, P, head_groups)
+    if P == 1:
+        return backward(q, k, v, o, lse, dout, mask_kind, scale)
+    lens = list(shard_lens) if shard_lens is not None else _shard_lens(Nl, P, group, q.device)
+    me = dist.get_rank(group)
+    if len(lens) != P or lens[me] != Nl:
+        raise ValueError(f"shard_lens {lens} does not match this rank's {Nl} rows")
+    Np = max(lens)
+    ragged = any(n != Np for n in lens)
+    keep = None
+    if ragged:
+        keep = torch.cat([torch.arange(j * Np, j * Np + n, device=q.device) for j, n in enumerate(lens)])
+        q, k, v, o, dout = (_pad_rows(t, Np) for t in (q, k, v, o, dout))
+        lse = _pad_rows(lse.transpose(1, 2), Np).transpose(1, 2).contiguous()
+    ng = head_groups
+    Hqg, Hkg = Hq // P // ng, Hkv // P // ng
+
+    # 1. post every group's input exchanges
+    recvs, works = [], []
+    for g in range(ng):
+        xs = [_to_heads(t, P, g, ng) for t in (q, k, v, o, dout)] + [_lse_to_heads(lse, P, g, ng)]
+        rs = [torch.empty_like(x) for x in xs]
+        works.append([dist.all_to_all_single(r_, x_, group=group, async_op=True) for r_, x_ in zip(rs, xs)])
+        recvs.append((xs, rs))
+    # 2. per group: wait, run the backward on whole sequences, post the return exchanges
+    out = []
+    for g in range(ng):
+        for w in works[g]:
+            w.wait()
+        rs = recvs[g][1]
+        qg, kg, vg, og, dog = (_from_seq(r_) for r_ in rs[:5])
+        lg = _lse_from_seq(rs[5])
+        if ragged:
+            qg, kg, vg, og, dog = (t.index_select(1, keep).contiguous() for t in (qg, kg, vg, og, dog))
+            lg = lg.index_select(2, keep).contiguous()
+        dqg, dkg, dvg = backward(qg, kg, vg, og, lg, dog, mask_kind, scale)
+        sends = []
+        for t, H_ in ((dqg, Hqg), (dkg, Hkg), (dvg, Hkg)):
+            if ragged:
+                tp = torch.zeros((B, P * Np, H_, d), dtype=t.dtype, device=t.device)
+                tp[:, keep] = t
+                t = tp
+            sends.append(t.view(B, P, Np, H_, d).permute(1, 0, 2, 3, 4).contiguous())
+        rbufs = [torch.empty_like(x) for x in sends]
+        ws = [dist.all_to_all_single(r_, x_, group=group, async_op=True) for r_, x_ in zip(rbufs, sends)]
+        out.append((sends, rbufs, ws))
+    # 3. reassemble this rank's rows
+    dq = torch.empty((B, Np, P, ng, Hqg, d), dtype=q.dtype, device=q.device)
+    dk = torch.empty((B, Np, P, ng, Hkg, d), dtype=k.dtype, device=k.device)
+    dv = torch.empty((B, Np, P, ng, Hkg, d), dtype=v.dtype, device=v.device)
+    for g in range(ng):
+        sends, rbufs, ws = out[g]
+        for w in ws:
+            w.wait()
+        for dst, r_ in zip((dq, dk, dv), rbufs):
+            dst[:, :, :, g] = r_.permute(1, 2, 0, 3, 4).to(dst.dtype)
+    dq, dk, dv = dq.view(B, Np, Hq, d), dk.view(B, Np, Hkv, d), dv.view(B, Np, Hkv, d)
+    if ragged:
+        dq, dk, dv = (t[:, :Nl].contiguous() for t in (dq, dk, dv))
+    return dq, dk, dv

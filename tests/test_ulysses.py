@@ -154,3 +154,69 @@ def test_single_rank_is_the_plain_call():
         return _oracle_attention(q_, k_, v_, mk, sc)
     o, lse = ulysses_attention(q, k, v, mask_kind=1, attention=att)
     assert calls == [q.shape]
+
+
+def _oracle_backward(q, k, v, o, lse, dout, mask_kind, scale):
+    """The fp64 oracle's gradients.  It recomputes P from q, k, v, so it also
+    checks that the o and lse it was handed are those of the same rows and
+    heads (the exchanges must move them with their q)."""
+    import oracle
+    ro, rl = oracle.attn_fwd(q.numpy(), k.numpy(), v.numpy(), scale, mask_kind)
+    assert np.array_equal(o.numpy(), ro) and np.array_equal(lse.numpy(), rl), "o / lse routed to the wrong rows"
+    dq, dk, dv = oracle.attn_bwd(q.numpy(), k.numpy(), v.numpy(), dout.numpy(), scale, mask_kind)
+    return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv)
+
+
+def _bwd_rank_main(rank, world, port, shape, mask_kind, groups, out_q, lens):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+
+    import oracle
+    from exact_io_aware_sm_b200.ulysses import ulysses_attention_bwd
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, N, Hq, Hkv, d = shape
+        q, k, v = _inputs(B, N, Hq, Hkv, d)
+        dout = np.random.default_rng(78).standard_normal((B, N, Hq, d))
+        scale = 1 / math.sqrt(d)
+        o, lse = oracle.attn_fwd(q, k, v, scale, mask_kind)
+        r0 = sum(lens[:rank])
+        sl = slice(r0, r0 + lens[rank])
+        t = [torch.from_numpy(np.ascontiguousarray(x[:, sl])) for x in (q, k, v, o, dout)]
+        tl = torch.from_numpy(np.ascontiguousarray(lse[:, :, sl]))
+        dq, dk, dv = ulysses_attention_bwd(t[0], t[1], t[2], t[3], tl, t[4], mask_kind=mask_kind, scale=scale,
+                                           head_groups=groups, backward=_oracle_backward)
+        out_q.put((rank, dq.numpy(), dk.numpy(), dv.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,shape,mask_kind,groups,lens", [
+    (2, (1, 64, 4, 2, 8), 1, 1, [32, 32]),       # causal, GQA, equal shards
+    (2, (2, 40, 8, 4, 8), 0, 2, [15, 25]),       # two head groups, uneven shards
+    (3, (1, 45, 6, 3, 8), 1, 1, [20, 1, 24]),    # three ranks, one holding a single row
+])
+def test_ulysses_backward_equals_unsharded_gradients(world, shape, mask_kind, groups, lens):
+    import oracle
+    B, N, Hq, Hkv, d = shape
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bwd_rank_main, args=(r, world, port, shape, mask_kind, groups, qq, lens))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict()
+    for _ in range(world):
+        r, dq, dk, dv = qq.get(timeout=180)
+        got[r] = (dq, dk, dv)
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    dq, dk, dv = (np.concatenate([got[r][i] for r in range(world)], axis=1) for i in range(3))
+    q, k, v = _inputs(B, N, Hq, Hkv, d)
+    dout = np.random.default_rng(78).standard_normal((B, N, Hq, d))
+    rq, rk, rv = oracle.attn_bwd(q, k, v, dout, 1 / math.sqrt(d), mask_kind)
+    for got_, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        assert got_.shape == ref.shape
+        np.testing.assert_allclose(got_, ref, atol=1e-12, rtol=0)
