@@ -261,3 +261,31 @@ def ulysses_attention_bwd(q, k, v, o, lse, dout, group=None, mask_kind=0, scale=
     if ragged:
         dq, dk, dv = (t[:, :Nl].contiguous() for t in (dq, dk, dv))
     return dq, dk, dv
+
+
+def ulysses_attention_autograd(q, k, v, group=None, mask_kind=0, scale=None, head_groups=1, attention=None,
+                               backward=None, shard_lens=None):
+    """ulysses_attention as a differentiable op: its backward is
+    ulysses_attention_bwd with the O and LSE the forward returned.  Returns o
+    for this rank's rows (the LSE carries no gradient and is not returned).
+    attention / backward replace the whole-sequence calls as in the two
+    functions above."""
+    import torch
+
+    class _Ulysses(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, q_, k_, v_):
+            o, lse = ulysses_attention(q_.contiguous(), k_.contiguous(), v_.contiguous(), group=group,
+                                       mask_kind=mask_kind, scale=scale, head_groups=head_groups,
+                                       attention=attention, shard_lens=shard_lens)
+            ctx.save_for_backward(q_, k_, v_, o, lse)
+            return o
+
+        @staticmethod
+        def backward(ctx, dout):
+            q_, k_, v_, o, lse = ctx.saved_tensors
+            return ulysses_attention_bwd(q_.contiguous(), k_.contiguous(), v_.contiguous(), o, lse, dout.contiguous(),
+                                         group=group, mask_kind=mask_kind, scale=scale, head_groups=head_groups,
+                                         backward=backward, shard_lens=shard_lens)
+
+    return _Ulysses.apply(q, k, v)
