@@ -75,6 +75,27 @@ def prefill_flops(w) -> int:
     return 4 * w["d"] * allowed_pairs(w) * w["B"] * w["Hq"]
 
 
+def plan_stats(w) -> dict:
+    """The tile plan of a prefill workload (host only, per head): Q tiles, KV
+    tile visits and how many of those carry an element predicate, before the
+    pair builder's two-segment re-cut; beside it, the classes of a plain
+    128 x 128 grid over the same mask.  The share of partial tiles among live
+    ones is the figure step 3 of the TPU attention guide measures and removes
+    by choosing the tile boundaries."""
+    import exact_io_aware_sm_b200 as eio
+    mk, bm = mask_of(w)
+    N = w["N"]
+    qt, kt = eio.plan(mk, bm, N, N)
+    visits = int(qt[:, 3].sum())
+    partial = sum(int(kt[r[2]:r[2] + r[3], 2].sum()) for r in qt)
+    cls = eio.classify(mk, bm, N, N, 128, 128)
+    full, part = int((cls == 1).sum()), int((cls == 2).sum())
+    return {"q_tiles": len(qt), "kv_tile_visits": visits, "partial_visits": partial,
+            "partial_share": partial / max(visits, 1),
+            "grid128_live": full + part, "grid128_partial": part,
+            "grid128_partial_share": part / max(full + part, 1)}
+
+
 def decode_kv_bytes(lens, Hkv, d, elem=2) -> int:
     return int(np.sum(lens)) * Hkv * d * elem * 2
 
@@ -839,7 +860,7 @@ def main():
                                "ms_per_step": r["ms_per_step"], "eager_ms_per_step": r["eager_ms_per_step"],
                                "config": {"workload": wx["desc"]},
                                "roofline": r["roofline"], "roofline_exp": r["roofline_exp"],
-                               "gpu_launches": r["gpu_launches"]}
+                               "gpu_launches": r["gpu_launches"], "plan": plan_stats(wx)}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -861,7 +882,7 @@ def main():
             "roofline": head["roofline"], "roofline_exp": head["roofline_exp"],
             "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
             "eager_ms_per_step": head["eager_ms_per_step"], "timing": head["timing"],
-            "clocks": sampler.summary(), "cpu_baseline": cpu,
+            "clocks": sampler.summary(), "cpu_baseline": cpu, "plan": plan_stats(w),
         }
         line.update(extra)
         print(json.dumps(line), flush=True)

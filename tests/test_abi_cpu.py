@@ -257,3 +257,17 @@ def test_binding_rejects_host_tensors():
         eio.key_stats(x)
     with pytest.raises(ValueError, match="CUDA"):
         eio.attn_decode(x[0], x, x, torch.zeros(1, dtype=torch.int32))
+
+
+def test_bench_plan_statistics():
+    """The tile-plan figures the bench line carries (host only): causal
+    counts in closed form; on the frame mask the plan has no partial tile,
+    where a plain 128 x 128 grid has 818 partial among 5023 live ones."""
+    import bench
+    g = bench.plan_stats(bench.WORKLOADS["gpt2"])
+    assert (g["q_tiles"], g["kv_tile_visits"], g["partial_visits"]) == (8, 36, 8)
+    lg = bench.plan_stats(bench.WORKLOADS["long"])
+    assert (lg["q_tiles"], lg["kv_tile_visits"], lg["partial_visits"]) == (128, 128 * 129 // 2, 128)
+    f = bench.plan_stats(bench.WORKLOADS["frame"])
+    assert f["q_tiles"] == 24 * 9 and f["partial_visits"] == 0 and f["partial_share"] == 0.0
+    assert (f["grid128_live"], f["grid128_partial"]) == (4205 + 818, 818)
