@@ -1,15 +1,20 @@
 """Benchmark: exact attention on B200 through the C-ABI library.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gpt2|long|frame|decode] [--no-extra]
+                    [--workload gpt2|long|frame|decode] [--no-extra] [--no-cpu-baseline]
+                    [--backward-only | --bound-only]
 
 Headline (one JSON line on rank 0): prefill attention TFLOP/s on the GPT-2
 shaped causal workload (B=8, H=12, N=1024, d=64, bf16).  One step is one
 attn_fwd call (tile plan lookup, TMA/tcgen05 kernel: S = QK^T, mask on
-partial tiles, online softmax, PV, O and LSE out).  The same line carries the
-decode workload (B=64, Hq=32, Hkv=8, d=128, lengths U[1024, 8192]) in KV GB/s
-and, unless --no-extra, the long-context GQA and frame block-sparse prefill
-workloads, each with its own roofline fraction.
+partial tiles, online softmax, PV, O and LSE out).  Unless --no-extra, the
+same line carries the decode workload (B=64, Hq=32, Hkv=8, d=128, lengths
+U[1024, 8192]) in KV GB/s, the backward and the bound-based forward on the
+headline shape, and the long-context GQA and frame block-sparse prefill
+workloads, each with its own roofline fraction; every prefill entry also
+carries its tile-plan figures (`plan`).  --backward-only / --bound-only time
+just that call on the chosen workload; --workload decode makes decode the
+headline.  --impl reference times the fp64 oracle on the host cores.
 
 FLOPs are algorithmic: 4*d per allowed (query, key) pair.  Bytes for decode
 are algorithmic: the K and V rows below each sequence's length, read once.
