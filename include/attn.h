@@ -27,7 +27,10 @@
  *     calling thread.
  *   - Tensors are contiguous and row-major in the layouts stated per call.
  *     Device pointers must be 16-byte aligned.  The caller owns every buffer;
- *     the library never frees or reallocates caller memory.
+ *     the library never frees or reallocates caller memory.  The library sees
+ *     pointers, not sizes: the caller guarantees that every buffer holds the
+ *     elements its layout states for the sizes passed (the Python binding
+ *     checks this before it passes a pointer).
  *   - Streams: "stream" is a cudaStream_t passed as void* (NULL = legacy
  *     default stream).  Compute calls are asynchronous on that stream.
  *     Argument errors are returned at once, before any launch.  Errors that a
