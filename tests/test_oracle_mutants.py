@@ -37,6 +37,13 @@ MUTANTS = [
      "dv[kj + t] += ds * ld(dout, dtype, q_off + t);"),
     ("key mean over Nkv + 1", "for (int t = 0; t < d; ++t) m[t] /= Nkv;",
      "for (int t = 0; t < d; ++t) m[t] /= (Nkv + 1);"),
+    ("frame rule: next frame instead of previous", "return fj == 0 || fj == fi || fj == fi - 1;",
+     "return fj == 0 || fj == fi || fj == fi + 1;"),
+    ("frame rule: reference frame dropped", "return fj == 0 || fj == fi || fj == fi - 1;",
+     "return fj == fi || fj == fi - 1;"),
+    ("radius squared", "radius[(size_t)b * Hkv + h] = sqrt(r2);", "radius[(size_t)b * Hkv + h] = r2;"),
+    ("bound rule inverted", "int use_bound = 2.0 * M * 1.4426950408889634 <= limit2;",
+     "int use_bound = 2.0 * M * 1.4426950408889634 > limit2;"),
 ]
 
 RUNNER = """
