@@ -3,8 +3,8 @@
 // kernel relies on:
 //   - every Q tile of the plan runs exactly once, in slot A or slot B of one pair;
 //   - 'heads' mode pairs a Q tile with itself (two query heads, one KV list);
-//   - slot B's tiles cover exactly the keys of its Q tile in the plan, slot A's keys are exactly
-//     those of the first nA tiles of the same list, and no tile is wider than 128 keys;
+//   - slot B's tiles cover exactly the keys of its Q tile in the plan, each once, slot A's keys are
+//     exactly those of the first nA tiles of the same list, and no tile is wider than 128 keys;
 //   - a tile of a pair kept without re-cutting carries, per slot, the partial flag of that slot's
 //     own tile in the plan; a re-cut tile has no partial flag (re-cutting is for predicate-free lists);
 //   - the visit order is a permutation of the pairs, most KV tiles first.
@@ -97,6 +97,7 @@ int main() {
         }
         if (t.nA > t.nB || (t.nrowsA == 0 && t.nA != 0)) fail("slot A's tile count", trial);
         std::set<int> kb, ka;
+        long vb = 0, va = 0;  // keys visited by each slot, with multiplicity
         bool is_recut = false;
         for (int k = 0; k < t.nB; ++k) {
           const PairKV& v = pp.kv[t.kv_first + k];
@@ -104,8 +105,14 @@ int main() {
           if ((v.flags >> 8) & 0xFF) is_recut = true;
           const std::set<int> s = tile_keys(v);
           kb.insert(s.begin(), s.end());
-          if (k < t.nA) ka.insert(s.begin(), s.end());
+          vb += v.ncols;
+          if (k < t.nA) {
+            ka.insert(s.begin(), s.end());
+            va += v.ncols;
+          }
         }
+        if (vb != static_cast<long>(kb.size()) || va != static_cast<long>(ka.size()))
+          fail("a slot visits a key twice", trial);
         if (kb != plan_keys(p, qb)) fail("slot B's keys differ from the plan", trial);
         if (ia >= 0 && ka != plan_keys(p, p.q[ia])) fail("slot A's keys differ from the plan", trial);
         // per-slot partial flags

@@ -1,5 +1,6 @@
 // Host check of the prefill pair builder: the two-segment re-cut of every pair's KV list covers
-// exactly the keys of the original plan, all allowed by the block map, in tiles of at most 128 keys.
+// exactly the keys of the original plan, each once, all allowed by the block map, in tiles of at
+// most 128 keys.
 #include "plan.h"
 #include <cstdio>
 #include <set>
@@ -18,13 +19,16 @@ int main() {
       PairPlan pp; build_pairs(p, rm == 1, &pp);
       for (const auto& t : pp.pairs) {
         std::set<int> got;
+        long visits = 0;  // keys visited, counted with multiplicity: each must be visited once
         for (int k = 0; k < t.nB; ++k) {
           const PairKV& v = pp.kv[t.kv_first + k];
           int n0 = (v.flags >> 8) & 0xFF; tiles++;
           if (v.ncols > 128 || v.ncols % 16) bad++;
+          visits += v.ncols;
           if (n0) { two++; for (int c = 0; c < n0; ++c) got.insert(v.col0 + c); for (int c = 0; c < v.ncols - n0; ++c) got.insert(v.col1 + c); }
           else for (int c = 0; c < v.ncols; ++c) got.insert(v.col0 + c);
         }
+        if (visits != static_cast<long>(got.size())) bad++;  // a key visited twice
         // keys of slot B's Q tile from the original plan
         const QTile* qb = nullptr;
         for (const auto& q : p.q) if (q.row0 == t.rowB) qb = &q;
