@@ -64,3 +64,46 @@ def test_survivors_collective_errors_when_a_rank_dies():
         for rank, outcome, dt in got:
             assert outcome != "returned", f"rank {rank}: the collective returned although a rank had died"
             assert dt < 60, f"rank {rank}: the error took {dt:.0f} s"
+
+
+def _ulysses_rank_main(rank, world, port, out_q):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from exact_io_aware_sm_b200.ulysses import ulysses_attention
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=20))
+    dist.barrier()
+    if rank == world - 1:
+        os._exit(3)
+    x = torch.from_numpy(np.random.default_rng(rank).standard_normal((1, 8, 4, 8)))
+
+    def att(q, k, v, mk, sc):  # never reached: the exchange before it fails
+        raise AssertionError("attention ran without every rank's rows")
+    t0 = time.time()
+    try:
+        ulysses_attention(x, x, x, attention=att, shard_lens=[8] * world)
+        out_q.put((rank, "returned", time.time() - t0))
+    except Exception as e:
+        out_q.put((rank, type(e).__name__, time.time() - t0))
+    out_q.close()
+    out_q.join_thread()
+    os._exit(0)
+
+
+def test_ulysses_exchange_errors_when_a_rank_dies():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 2
+    procs = [ctx.Process(target=_ulysses_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in range(world - 1)]
+    for p in procs:
+        p.join(60)
+    for rank, outcome, dt in got:
+        assert outcome not in ("returned", "AssertionError"), f"rank {rank}: {outcome}"
+        assert dt < 60, f"rank {rank}: the error took {dt:.0f} s"
