@@ -271,3 +271,45 @@ def test_bench_plan_statistics():
     f = bench.plan_stats(bench.WORKLOADS["frame"])
     assert f["q_tiles"] == 24 * 9 and f["partial_visits"] == 0 and f["partial_share"] == 0.0
     assert (f["grid128_live"], f["grid128_partial"]) == (4205 + 818, 818)
+
+
+def test_error_detail_is_per_thread_and_host_calls_are_thread_safe():
+    """attn_last_error_detail reports the calling thread's own last failure
+    while other threads fail differently at the same time (ctypes releases
+    the GIL during the calls); concurrent host-only planning gives the same
+    plans as serial planning."""
+    import threading
+    L = eio.lib()
+    errors = []
+
+    def failing(kind):
+        buf = ctypes.create_string_buffer(256)
+        for _ in range(2000):
+            rc = _fwd(q=None) if kind == "null" else _fwd(Hq=3, Hkv=2)
+            L.attn_last_error_detail(buf, 256)
+            text = buf.value.decode()
+            if (kind == "null" and (rc != 1 or "non-NULL" not in text)) or \
+               (kind == "shape" and (rc != 2 or "multiple" not in text)):
+                errors.append((kind, rc, text))
+                return
+
+    rng = np.random.default_rng(99)
+    maps = [(int(n), int(m), _random_map(rng, (int(n) + 15) // 16, (int(m) + 15) // 16, 0.5))
+            for n, m in rng.integers(1, 900, size=(8, 2))]
+    serial = [eio.plan(oracle.MASK_BLOCK, bm, n, m) for n, m, bm in maps]
+    planned = [None] * len(maps)
+
+    def planning(i):
+        n, m, bm = maps[i]
+        for _ in range(20):
+            planned[i] = eio.plan(oracle.MASK_BLOCK, bm, n, m)
+
+    threads = [threading.Thread(target=failing, args=(k,)) for k in ("null", "shape", "null", "shape")]
+    threads += [threading.Thread(target=planning, args=(i,)) for i in range(len(maps))]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors[:3]
+    for (qs, ks), (qp, kp) in zip(serial, planned):
+        assert np.array_equal(qs, qp) and np.array_equal(ks, kp)
