@@ -758,6 +758,7 @@ def run_reference(args, world, rank):
         return
     import oracle
     oracle.build()
+    cores = oracle.threads(cpu_cores())  # all the host's cores, whatever OMP_NUM_THREADS the launcher set
     run, desc = oracle_prefill_call(w, w["seed"])
     for _ in range(min(args.warmup, 1)):
         run()
@@ -774,7 +775,7 @@ def run_reference(args, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": w["desc"], "sample": f"{desc} per step"},
-        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"{desc} per step, {args.steps} steps, fp64"},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -871,8 +872,9 @@ def main():
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
+        cores = oracle.threads(cpu_cores())
         dt, fl, desc = oracle_prefill_sample(w, rank_seed(w["seed"], 0))
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                "sample": desc}
 
     if rank == 0:

@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.ora_key_stats.argtypes = [P, I, I, I, I, I, P, P]
         L.ora_attn_bwd_dq_rows.argtypes = [P, P, P, P, I, I, I, I, I, I, I, D, I, P, P, I, P]
         L.ora_attn_fwd_bound.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, P, P, P, D, P, P, P]
+        L.ora_threads.argtypes = [I]
+        L.ora_threads.restype = I
         _lib = L
     return _lib
 
@@ -208,6 +210,12 @@ def classify(mask_kind, block_map, Nq, Nkv, tq, tk):
 def count_allowed(mask_kind, block_map, Nq, Nkv):
     bm = _bm(block_map)
     return int(lib().ora_count_allowed(mask_kind, _ptr(bm), Nq, Nkv))
+
+
+def threads(n: int = 0) -> int:
+    """Set the oracle's OpenMP thread count for calls from this thread (if
+    n > 0) and return the count it will use."""
+    return int(lib().ora_threads(int(n)))
 
 
 def check_schedule(mask_kind, block_map, Nq, Nkv, qtiles, kvtiles):

@@ -41,6 +41,7 @@
  * stored value (bf16 bit patterns, fp32 or fp64).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -667,4 +668,14 @@ int ora_attn_bwd_dq_rows(const void *q, const void *k, const void *v, const void
     free(dP);
   }
   return bad ? -1 : 0;
+}
+
+/*
+ * Threads for the parallel loops of this file: sets the count (for parallel
+ * regions that the calling thread starts) when n > 0, and returns the count
+ * the next such region will use.  Timing code reports this number.
+ */
+int ora_threads(int n) {
+  if (n > 0) omp_set_num_threads(n);
+  return omp_get_max_threads();
 }
