@@ -868,8 +868,8 @@ def main():
                                "roofline": r["roofline"], "roofline_exp": r["roofline_exp"],
                                "gpu_launches": r["gpu_launches"], "plan": plan_stats(wx)}
 
-    cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
+    cpu = None  # the oracle baseline: rank 0 of a one-GPU run only, so scaling runs hold no GPU idle for it
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
         cores = oracle.threads(cpu_cores())
