@@ -743,6 +743,26 @@ def oracle_prefill_sample(w, seed, min_seconds=10.0, max_passes=200):
     return dt, fl, f"{desc}, {n} passes, fp64, {dt:.1f} s"
 
 
+def oracle_decode_call(w, seed, n_seq=8):
+    """A bounded sample of the decode workload for the oracle: the first
+    n_seq sequences, with the same seeded queries, caches and lengths as in
+    the full batch.  Returns (run, description, algorithmic bytes per run)."""
+    import oracle
+    B, Hq, Hkv, Lmax, d = w["B"], w["Hq"], w["Hkv"], w["Lmax"], w["d"]
+    n = min(n_seq, B)
+    lens = synthetic.seqlens(w["len_seed"], B)[:n]
+    q = synthetic.tensor(seed, synthetic.TID_Q, (n, Hq, d))
+    kc = synthetic.kv_cache(seed, synthetic.TID_K, n, Lmax, Hkv, d, lens)
+    vc = synthetic.kv_cache(seed, synthetic.TID_V, n, Lmax, Hkv, d, lens)
+    scale = 1.0 / math.sqrt(d)
+
+    def run():
+        oracle.decode(q, kc, vc, lens, scale)
+
+    nbytes = decode_kv_bytes(lens, Hkv, d) + q.nbytes * 2 + n * Hq * 4
+    return run, f"the first {n} of {B} sequences ({int(lens.sum())} cached keys)", nbytes
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -759,6 +779,9 @@ def run_reference(args, world, rank):
     import oracle
     oracle.build()
     cores = oracle.threads(cpu_cores())  # all the host's cores, whatever OMP_NUM_THREADS the launcher set
+    if w["kind"] == "decode":
+        run_reference_decode(args, w, cores)
+        return
     run, desc = oracle_prefill_call(w, w["seed"])
     for _ in range(min(args.warmup, 1)):
         run()
@@ -778,6 +801,30 @@ def run_reference(args, world, rank):
         "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"{desc} per step, {args.steps} steps, fp64"},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_decode(args, w, cores):
+    """The reference arm on the decode workload: the oracle's decode over a
+    bounded sample of sequences, in KV GB/s (algorithmic bytes)."""
+    run, desc, nbytes = oracle_decode_call(w, w["seed"])
+    for _ in range(min(args.warmup, 1)):
+        run()
+    dt = 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        run()
+        dt += time.perf_counter() - t0
+    gbs = nbytes * args.steps / dt / 1e9
+    line = {
+        "impl": "reference", "metric": "decode KV GB/s", "value": gbs, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w["desc"], "sample": f"{desc} per step"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{desc} per step, {args.steps} steps, fp64"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 

@@ -83,3 +83,16 @@ def test_reference_arm_under_torchrun_prints_one_line():
     # and reports, every core of the host
     assert d["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_on_the_decode_workload():
+    """--impl reference --workload decode: the oracle's decode over the first
+    sequences of the same seeded batch, one JSON line in KV GB/s."""
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--workload", "decode", "--steps", "1", "--warmup", "0"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == "decode KV GB/s" and d["unit"] == "GB/s" and d["value"] > 0
+    assert d["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0)) and "sequences" in d["config"]["sample"]
