@@ -763,6 +763,23 @@ def oracle_decode_call(w, seed, n_seq=8):
     return run, f"the first {n} of {B} sequences ({int(lens.sum())} cached keys)", nbytes
 
 
+def oracle_decode_baseline(w, seed, min_seconds=5.0):
+    """The cpu_baseline of a decode line: the oracle's decode of a sample of
+    the batch (oracle_decode_call), repeated for at least min_seconds."""
+    import oracle
+    oracle.build()
+    cores = oracle.threads(cpu_cores())
+    run, desc, nbytes = oracle_decode_call(w, seed)
+    n, dt = 0, 0.0
+    while dt < min_seconds:
+        t0 = time.perf_counter()
+        run()
+        dt += time.perf_counter() - t0
+        n += 1
+    return {"value": nbytes * n / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{desc}, {n} passes, fp64, {dt:.1f} s"}
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -884,12 +901,15 @@ def main():
     if args.workload == "decode":
         with sampler:
             d = bench_decode(w, args, world, rank, peaks)
+        cpu = None
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cpu = oracle_decode_baseline(w, rank_seed(w["seed"], 0))
         if rank == 0:
             line = {"metric": d["metric"], "value": d["value"], "unit": d["unit"], "n_gpus": world,
                     "steps": d["steps"], "warmup": args.warmup, "ms_per_step": d["ms_per_step"],
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                     "data": "synthetic", "config": d["config"], "roofline": d["roofline"], "e2e": d["e2e"],
-                    "gpu_launches": d["gpu_launches"], "clocks": sampler.summary(), "cpu_baseline": None,
+                    "gpu_launches": d["gpu_launches"], "clocks": sampler.summary(), "cpu_baseline": cpu,
                     "multi_token_2": d.get("multi_token_2")}
             print(json.dumps(line), flush=True)
         if world > 1:

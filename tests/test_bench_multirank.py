@@ -96,3 +96,11 @@ def test_reference_arm_on_the_decode_workload():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["metric"] == "decode KV GB/s" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0)) and "sequences" in d["config"]["sample"]
+
+
+def test_decode_cpu_baseline_helper():
+    import bench
+    w = bench.WORKLOADS["decode"]
+    c = bench.oracle_decode_baseline(w, bench.rank_seed(w["seed"], 0), min_seconds=0.2)
+    assert c["kind"] == "oracle" and c["unit"] == "GB/s" and c["value"] > 0
+    assert c["cores"] == len(os.sched_getaffinity(0))
