@@ -44,6 +44,10 @@ MUTANTS = [
     ("radius squared", "radius[(size_t)b * Hkv + h] = sqrt(r2);", "radius[(size_t)b * Hkv + h] = r2;"),
     ("bound rule inverted", "int use_bound = 2.0 * M * 1.4426950408889634 <= limit2;",
      "int use_bound = 2.0 * M * 1.4426950408889634 > limit2;"),
+    ("per-row dQ: D term dropped", "double ds = S[j] * (dP[j] - D);", "double ds = S[j] * dP[j];"),
+    ("per-row dQ: K row misindexed",
+     "for (int t = 0; t < d; ++t) out[t] += scale * ds * ld(k, dtype, kv_base + (size_t)j * kv_stride + t);",
+     "for (int t = 0; t < d; ++t) out[t] += scale * ds * ld(k, dtype, kv_base + (size_t)(Nkv - 1 - j) * kv_stride + t);"),
 ]
 
 RUNNER = """
