@@ -17,6 +17,11 @@ Entry points mirror include/attn.h:
     plan(mask_kind, block_map, Nq, Nkv)
     sync_status(stream=None)
 
+Above these: exact_io_aware_sm_b200.autograd.attention (the differentiable op,
+attn_fwd forward and attn_bwd backward) and exact_io_aware_sm_b200.ulysses
+(sequence-parallel forward, backward and differentiable op over
+torch.distributed).
+
 The C ABI takes plain pointers and cannot see buffer sizes, so every tensor
 and block map is checked here (device, contiguity, dtype, shape) before a
 pointer is passed: a mis-shaped output or map raises ValueError instead of
