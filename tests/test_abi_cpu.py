@@ -313,3 +313,14 @@ def test_error_detail_is_per_thread_and_host_calls_are_thread_safe():
     assert not errors, errors[:3]
     for (qs, ks), (qp, kp) in zip(serial, planned):
         assert np.array_equal(qs, qp) and np.array_equal(ks, kp)
+
+
+def test_io_complexity_worked_example(golden):
+    """bench.io_elements against the FlashAttention page's section-5 numbers:
+    standard attention ~N^2 element accesses, the tiled kernel ~N^2 d^2 / M."""
+    import bench
+    g = golden("io_complexity_flashattention_sec5.txt")
+    std, tiled = bench.io_elements(int(g["N"]), int(g["d"]), g["M"])
+    assert round(std / 1e4) == g["standard_1e4"]
+    assert round(tiled / 1e4, 1) == g["tiled_1e4"]
+    assert round(std / tiled) == g["ratio"]
