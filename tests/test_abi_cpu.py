@@ -324,3 +324,20 @@ def test_io_complexity_worked_example(golden):
     assert round(std / 1e4) == g["standard_1e4"]
     assert round(tiled / 1e4, 1) == g["tiled_1e4"]
     assert round(std / tiled) == g["ratio"]
+
+
+def test_kv_cache_and_attention_matrix_worked_examples(golden):
+    """bench's size helpers against the pages' worked numbers: the inference
+    page's KV cache example (per token, for 128 users x 2048 tokens, and with
+    MQA's single KV head) and the FlashAttention page's size of S."""
+    import bench
+    g = golden("kv_cache_size_inference_page.txt")
+    per = bench.kv_cache_bytes_per_token(int(g["layers"]), int(g["heads"]), int(g["head_dim"]))
+    assert per == g["bytes_per_token"] and per / 2 ** 20 == g["mb_per_token"]
+    total = per * int(g["users"]) * int(g["tokens"])
+    assert total / 2 ** 30 == g["gb_total"]
+    mqa = bench.kv_cache_bytes_per_token(int(g["layers"]), 1, int(g["head_dim"])) * int(g["users"]) * int(g["tokens"])
+    assert mqa / 2 ** 30 == g["gb_total_mqa"]
+    s = golden("attention_matrix_size_flashattention_sec1.txt")
+    n = bench.attention_matrix_elements(int(s["N"]), int(s["heads"]), int(s["batch"]))
+    assert round(n / 1e8, 1) == s["elements_1e8"] and round(2 * n / 1e9, 1) == s["gb_16bit"]
