@@ -124,7 +124,8 @@ def _bm(block_map, Nq=None, Nkv=None):
 def _need(t, name, shape, dtypes, device=None):
     """Check a tensor handed to the library: a contiguous CUDA tensor of one
     of the given dtypes whose shape matches `shape` (None entries match any
-    size), on `device` if given."""
+    size), on `device` if given, else (the call's first tensor) on the
+    current CUDA device, where the library launches."""
     if not getattr(t, "is_cuda", False):
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
@@ -136,6 +137,12 @@ def _need(t, name, shape, dtypes, device=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}; expected {want}")
     if device is not None and t.device != device:
         raise ValueError(f"{name} is on {t.device}; expected {device}")
+    if device is None:  # the call's first tensor: the library runs on the current device
+        import torch
+        cur = torch.cuda.current_device()
+        if t.device.index is not None and t.device.index != cur:
+            raise ValueError(f"{name} is on {t.device} but the current CUDA device is {cur}; "
+                             f"call inside torch.cuda.device({t.device.index})")
 
 
 def attn_fwd(q, k, v, o=None, lse=None, scale=None, mask_kind=MASK_NONE, block_map=None,
