@@ -278,3 +278,36 @@ def test_ulysses_autograd_gradients(world, shape, mask_kind, lens):
     rq, rk, rv = oracle.attn_bwd(q, k, v, w, 1 / math.sqrt(d), mask_kind)
     for got_, ref in ((dq, rq), (dk, rk), (dv, rv)):
         np.testing.assert_allclose(got_, ref, atol=1e-12, rtol=0)
+
+
+def _bad_lens_rank_main(rank, world, port, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+
+    from exact_io_aware_sm_b200.ulysses import ulysses_attention
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        x = torch.zeros((1, 4, 2, 8), dtype=torch.float64)
+        try:
+            ulysses_attention(x, x, x, attention=_oracle_attention, shard_lens=[5, 3])  # this rank holds 4 rows
+            out_q.put((rank, "returned"))
+        except ValueError as e:
+            out_q.put((rank, "ValueError" if "shard_lens" in str(e) else str(e)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ulysses_rejects_shard_lengths_that_do_not_match():
+    """shard_lens that disagree with the rows a rank holds raise ValueError on
+    every rank before any exchange starts (so nothing waits on a peer)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bad_lens_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    assert got == {0: "ValueError", 1: "ValueError"}
