@@ -338,6 +338,8 @@ int check_mask_args(int mask_kind, const uint8_t* block_map) {
 
 void eio::set_error_detail(const char* msg) { std::snprintf(g_err, sizeof g_err, "%s", msg); }
 
+int eio::require_sm100() { return check_device_sm100(); }
+
 bool eio::encode_bf16_map(CUtensorMap* m, const void* base, int B, int N, int H, int d, int box_rows) {
   const CUresult r = encode_map(m, base, B, N, H, d, box_rows);
   if (r != CUDA_SUCCESS) {
@@ -719,6 +721,7 @@ int attn_last_error_detail(char* buf, int len) {
 }
 
 int attn_shutdown(void) {
+  noalloc_forget();
   std::lock_guard<std::mutex> lk(g_mu);
   int cur = 0;
   cudaGetDevice(&cur);

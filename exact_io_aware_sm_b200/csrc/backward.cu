@@ -1032,17 +1032,20 @@ __global__ void __launch_bounds__(kBThreads, 1)
 template <int D, bool BLK>
 cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   using C = BCfg<D>;
-  static int attr_dev = -1, n_sm = 0;
-  int dev = 0;
+  static DeviceOnce attr_set;
+  int dev = 0, n_sm = 0;
   cudaGetDevice(&dev);
-  if (attr_dev != dev) {
+  if (!attr_set.test(dev)) {
     cudaError_t e =
         cudaFuncSetAttribute(bwd_dq_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemQ);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemKV);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    attr_dev = dev;
+    attr_set.set(dev);
+  }
+  {
+    const cudaError_t e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
   }
   CUtensorMap tq, tdo, tk, tv, to, tdq, tdk, tdv;
   if (!encode_bf16_map(&tq, a.q, a.B, a.Nq, a.Hq, D, kT) || !encode_bf16_map(&tdo, a.dout, a.B, a.Nq, a.Hq, D, kT) ||

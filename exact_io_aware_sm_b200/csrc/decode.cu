@@ -381,14 +381,14 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
 
 template <int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
-  static int attr_dev = -1;
+  static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (attr_dev != dev) {
+  if (!attr_set.test(dev)) {
     cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          DCfg<D>::kSmem);
     if (e != cudaSuccess) return e;
-    attr_dev = dev;
+    attr_set.set(dev);
   }
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -41,11 +41,12 @@ int fail(int code, const char* msg) {
 }
 
 // Device address of the scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached until attn_shutdown.
 int scratch_on_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return fail(ATTN_ERR_CUDA, "attn_decode_noalloc: no usable current device");
+  if (int rc = eio::require_sm100()) return rc;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_addr[dev]) {
     void* p = nullptr;
@@ -61,6 +62,11 @@ int scratch_on_device(void** out) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+void eio::noalloc_forget() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (void*& p : g_addr) p = nullptr;
+}
 
 extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                    const int32_t* seqlens, void* o, float* lse, int B, int Hq,
@@ -91,10 +97,10 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
   void* base = nullptr;
   if (int rc = scratch_on_device(&base)) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The error word is zero when the module loads and stays latched until
+  // attn_decode_noalloc_status reads and clears it; the partials are written
+  // before they are read.
   int* err = static_cast<int*>(base);
-  // The error word must start at zero; the partials are written before they are read.
-  if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess)
-    return fail(ATTN_ERR_CUDA, "attn_decode_noalloc: clearing the error word failed");
 
   eio::DecodeArgs a{};
   a.q = q;
@@ -117,4 +123,23 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
   const cudaError_t e = eio::launch_decode(d, G, a, s);
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, cudaGetErrorString(e));
   return ATTN_OK;
+}
+
+extern "C" int attn_decode_noalloc_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t es = cudaStreamSynchronize(s);
+  if (es != cudaSuccess) return fail(ATTN_ERR_CUDA, cudaGetErrorString(es));
+  void* base = nullptr;
+  if (int rc = scratch_on_device(&base)) return rc;
+  int h = 0;
+  if (cudaMemcpy(&h, base, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return fail(ATTN_ERR_CUDA, "attn_decode_noalloc_status: reading the error word failed");
+  if (h == 0) return ATTN_OK;
+  const int zero = 0;
+  if (cudaMemcpy(base, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return fail(ATTN_ERR_CUDA, "attn_decode_noalloc_status: clearing the error word failed");
+  if (h == eio::kErrDeviceTimeout)
+    return fail(h, "attn_decode_noalloc: a bounded wait ran out; O and LSE of that call are undefined");
+  if (h == eio::kErrDeviceArg) return fail(h, "attn_decode_noalloc: a seqlens entry was outside [0, Lmax]");
+  return fail(h, "attn_decode_noalloc: device error");
 }

@@ -4,9 +4,24 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 namespace eio {
+
+// Per-device record of one-time launch set-up (kernel attributes), safe to
+// test and set from several host threads.  The set-up it guards is
+// idempotent, so two threads that both find a device's bit clear both run it,
+// which is harmless; a bit is set only after the set-up succeeded.
+struct DeviceOnce {
+  std::atomic<unsigned long long> done{0};
+  bool test(int dev) const {
+    return dev >= 0 && dev < 64 && ((done.load(std::memory_order_acquire) >> dev) & 1ull) != 0;
+  }
+  void set(int dev) {
+    if (dev >= 0 && dev < 64) done.fetch_or(1ull << dev, std::memory_order_release);
+  }
+};
 
 // Device error codes latched by kernels (same values as attn_status).
 constexpr int kErrDeviceTimeout = 7;
@@ -126,5 +141,13 @@ bool encode_bf16_map(CUtensorMap* m, const void* base, int B, int N, int H, int 
 
 // Sets the text returned by attn_last_error_detail() on this thread.
 void set_error_detail(const char* msg);
+
+// ATTN_OK if the current device is sm_100, else ATTN_ERR_UNSUPPORTED (or
+// ATTN_ERR_CUDA) with the error detail set.
+int require_sm100();
+
+// Forgets the cached device addresses of attn_decode_noalloc's scratch array
+// (called by attn_shutdown, so that a device reset after it starts afresh).
+void noalloc_forget();
 
 }  // namespace eio

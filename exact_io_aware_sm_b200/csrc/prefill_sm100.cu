@@ -718,10 +718,10 @@ template <int D, bool STAGGER, bool BOUND>
 cudaError_t launch_ds(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const CUtensorMap& to, const CUtensorMap& tk16, const CUtensorMap& tv16,
                       const PrefillArgs& a, cudaStream_t s) {
-  static int attr_dev = -1;
+  static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (attr_dev != dev) {
+  if (!attr_set.test(dev)) {
     // The warpgroup register split is only safe when every thread starts with
     // exactly kLaunchRegs registers.
     cudaFuncAttributes fa;
@@ -731,7 +731,7 @@ cudaError_t launch_ds(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
     e = cudaFuncSetAttribute(prefill_bf16_kernel<D, STAGGER, BOUND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg<D>::kSmem);
     if (e != cudaSuccess) return e;
-    attr_dev = dev;
+    attr_set.set(dev);
   }
   if (a.n_items == 0) return cudaSuccess;
   const long long grid = a.n_items < a.num_ctas ? a.n_items : a.num_ctas;

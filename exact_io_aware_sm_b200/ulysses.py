@@ -57,14 +57,32 @@ def default_attention(q, k, v, mask_kind, scale):
     return attn_fwd(q.contiguous(), k.contiguous(), v.contiguous(), scale=scale, mask_kind=mask_kind)
 
 
-def _shard_lens(Nl, P, group, device):
-    """Every rank's shard length (one small all-gather)."""
+def _shard_lens(Nl, P, group, device, given=None):
+    """Every rank's shard length, agreed by all ranks with one small
+    all-gather before any exchange.  Each rank sends its row count and the
+    shard_lens it was given (if any); every rank then checks every given list
+    against the gathered counts, so all ranks reach the same verdict and raise
+    together (no rank goes on into an all-to-all that another one left)."""
     import torch
     import torch.distributed as dist
-    mine = torch.tensor([Nl], dtype=torch.int64, device=device)
-    allv = [torch.zeros_like(mine) for _ in range(P)]
-    dist.all_gather(allv, mine, group=group)
-    return [int(t.item()) for t in allv]
+    row = torch.full((P + 2,), -1, dtype=torch.int64)
+    row[0] = Nl
+    if given is None:
+        row[1] = 0
+    elif len(given) != P:
+        row[1] = 2  # malformed: wrong number of entries
+    else:
+        row[1] = 1
+        row[2:] = torch.tensor([int(n) for n in given], dtype=torch.int64)
+    row = row.to(device)
+    allv = [torch.zeros_like(row) for _ in range(P)]
+    dist.all_gather(allv, row, group=group)
+    rows = [t.cpu().tolist() for t in allv]
+    actual = [r[0] for r in rows]
+    bad = [i for i, r in enumerate(rows) if r[1] == 2 or (r[1] == 1 and r[2:] != actual)]
+    if bad:
+        raise ValueError(f"shard_lens given on rank(s) {bad} do not match the ranks' rows {actual}")
+    return actual
 
 
 def _pad_rows(x, n):
@@ -85,8 +103,10 @@ def ulysses_attention(q, k, v, group=None, mask_kind=0, scale=None, head_groups=
     whole sequences; the default is this package's attn_fwd (bf16 CUDA
     tensors).  mask_kind is NONE or CAUSAL: the whole sequence is present on
     every rank, so a causal mask needs no change.  shard_lens: every rank's
-    number of rows, in rank order, if the caller knows them (else they are
-    gathered; shards of equal length need no padding)."""
+    number of rows, in rank order, if the caller knows them; the lengths are
+    gathered either way, and a given list that does not match them raises
+    ValueError on every rank before any exchange (shards of equal length need
+    no padding)."""
     import torch
     import torch.distributed as dist
 
@@ -99,10 +119,7 @@ def ulysses_attention(q, k, v, group=None, mask_kind=0, scale=None, head_groups=
     _check(B, Nl, Hq, Hkv, P, head_groups)
     if P == 1:
         return attention(q, k, v, mask_kind, scale)
-    lens = list(shard_lens) if shard_lens is not None else _shard_lens(Nl, P, group, q.device)
-    me = dist.get_rank(group)
-    if len(lens) != P or lens[me] != Nl:
-        raise ValueError(f"shard_lens {lens} does not match this rank's {Nl} rows")
+    lens = _shard_lens(Nl, P, group, q.device, None if shard_lens is None else list(shard_lens))
     Np = max(lens)  # every shard padded to this many rows for the exchanges
     ragged = any(n != Np for n in lens)
     # rows of the padded, gathered sequence that hold real rows, in sequence order
@@ -204,10 +221,7 @@ def ulysses_attention_bwd(q, k, v, o, lse, dout, group=None, mask_kind=0, scale=
     _check(B, Nl, Hq, Hkv, P, head_groups)
     if P == 1:
         return backward(q, k, v, o, lse, dout, mask_kind, scale)
-    lens = list(shard_lens) if shard_lens is not None else _shard_lens(Nl, P, group, q.device)
-    me = dist.get_rank(group)
-    if len(lens) != P or lens[me] != Nl:
-        raise ValueError(f"shard_lens {lens} does not match this rank's {Nl} rows")
+    lens = _shard_lens(Nl, P, group, q.device, None if shard_lens is None else list(shard_lens))
     Np = max(lens)
     ragged = any(n != Np for n in lens)
     keep = None

@@ -231,18 +231,31 @@ int attn_shutdown(void);
  *   (attn_last_error_detail says how much it needed), before any GPU work.
  *   Set-up: the first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture.
+ *   first call before any stream capture.  attn_shutdown forgets the cached
+ *   addresses: call it before a cudaDeviceReset, so that the next call looks
+ *   the array up again in the new context.
  *   Sharing: every call on a device uses the same array, and the array keeps
- *   the previous call's contents (each call clears the error word and writes
- *   every partial it reads).  Calls that overlap on the GPU (different
- *   streams, or other host threads) race on the array: order them.
- *   Errors: as attn_decode for arguments.  A seqlens entry outside [0, Lmax]
- *   gives that sequence O = 0 and LSE = -inf; this variant does not report it
- *   through attn_sync_status.
+ *   the previous call's contents (each call writes every partial it reads).
+ *   Calls that overlap on the GPU (different streams, or other host threads)
+ *   race on the array: order them.
+ *   Errors: as attn_decode for arguments (a device that is not sm_100 gives
+ *   ATTN_ERR_UNSUPPORTED).  Errors found on the device go to an error word
+ *   inside the array, not to the one attn_sync_status reads: a seqlens entry
+ *   outside [0, Lmax] (that sequence gets O = 0 and LSE = -inf) and a bounded
+ *   wait that ran out (O and LSE of that call are then undefined).  The word
+ *   stays latched until attn_decode_noalloc_status reads and clears it.
  */
 int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                         const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
                         int Lmax, int d, float scale, void* stream);
+
+/*
+ * attn_decode_noalloc_status -- synchronise `stream`, then return (and clear)
+ * the error word of attn_decode_noalloc on the current device: ATTN_OK,
+ * ATTN_ERR_DEVICE_TIMEOUT or ATTN_ERR_DEVICE_ARG (see above).  Allocates
+ * nothing.  The source pages have no counterpart for it either.
+ */
+int attn_decode_noalloc_status(void* stream);
 
 /*
  * attn_bwd -- gradients of attn_fwd (bf16) for an upstream gradient dO.

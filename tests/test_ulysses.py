@@ -280,30 +280,48 @@ def test_ulysses_autograd_gradients(world, shape, mask_kind, lens):
         np.testing.assert_allclose(got_, ref, atol=1e-12, rtol=0)
 
 
-def _bad_lens_rank_main(rank, world, port, out_q):
+def _bad_lens_rank_main(rank, world, port, out_q, lens_per_rank, backward=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import torch.distributed as dist
 
-    from exact_io_aware_sm_b200.ulysses import ulysses_attention
+    from exact_io_aware_sm_b200.ulysses import ulysses_attention, ulysses_attention_bwd
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        x = torch.zeros((1, 4, 2, 8), dtype=torch.float64)
+        x = torch.zeros((1, 4, 2, 8), dtype=torch.float64)  # every rank holds 4 rows
+        lse = torch.zeros((1, 2, 4), dtype=torch.float64)
         try:
-            ulysses_attention(x, x, x, attention=_oracle_attention, shard_lens=[5, 3])  # this rank holds 4 rows
+            if backward:
+                ulysses_attention_bwd(x, x, x, x, lse, x, backward=lambda *a: None,
+                                      shard_lens=lens_per_rank[rank])
+            else:
+                ulysses_attention(x, x, x, attention=_oracle_attention, shard_lens=lens_per_rank[rank])
             out_q.put((rank, "returned"))
         except ValueError as e:
             out_q.put((rank, "ValueError" if "shard_lens" in str(e) else str(e)))
+        # The group is still usable: a collective after the refusal completes.
+        t = torch.ones(1)
+        dist.all_reduce(t)
+        assert t.item() == world
     finally:
         dist.destroy_process_group()
 
 
-def test_ulysses_rejects_shard_lengths_that_do_not_match():
-    """shard_lens that disagree with the rows a rank holds raise ValueError on
-    every rank before any exchange starts (so nothing waits on a peer)."""
+@pytest.mark.parametrize("lens_per_rank,backward", [
+    ([[5, 3], [5, 3]], False),   # every rank's own entry is wrong
+    ([[4, 3], [4, 3]], False),   # only rank 1's entry is wrong: rank 0 must raise too
+    ([[4, 4], [4, 3]], False),   # the ranks pass different lists
+    ([[4, 4], [4, 4, 0]], False),  # one rank's list has the wrong length
+    ([[4, 3], [4, 3]], True),    # the same agreement in the backward
+])
+def test_ulysses_rejects_shard_lengths_that_do_not_match(lens_per_rank, backward):
+    """shard_lens that disagree with the rows the ranks hold raise ValueError
+    on every rank before any exchange starts (so nothing waits on a peer),
+    even when a rank's own entry is right or the ranks pass different lists."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_bad_lens_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_bad_lens_rank_main, args=(r, 2, port, q, lens_per_rank, backward))
+             for r in range(2)]
     for p in procs:
         p.start()
     got = dict(q.get(timeout=120) for _ in range(2))

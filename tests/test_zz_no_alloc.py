@@ -36,7 +36,14 @@ def lib():
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     L.attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P]
     L.attn_decode_noalloc.restype = I
+    L.attn_decode_noalloc_status.argtypes = [P]
+    L.attn_decode_noalloc_status.restype = I
     return L
+
+
+def _status(L):
+    """The no-allocation decode's own error word (read and cleared)."""
+    return L.attn_decode_noalloc_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
 def _inputs(seed, B, Hq, Hkv, Lmax, d):
@@ -74,7 +81,25 @@ def test_noalloc_matches_attn_decode_on_two_calls(lib, shape):
         err = (o.float() - ref_o.float()).abs()
         assert err.max().item() <= O_MAX and err.mean().item() <= O_MEAN
         assert (lse - ref_l).abs().max().item() <= LSE_TOL
+        assert _status(lib) == 0, eio.last_error()  # its own error word: nothing latched
     eio.sync_status()
+
+
+def test_noalloc_reports_device_errors_through_its_own_status(lib):
+    """A seqlens entry above Lmax is found on the device: that sequence gets
+    O = 0 and LSE = -inf, and the error goes to the array's own error word,
+    which attn_decode_noalloc_status returns once and then clears."""
+    B, Hq, Hkv, Lmax, d = 3, 8, 2, 300, 128
+    q, kc, vc, _ = _inputs(903, B, Hq, Hkv, Lmax, d)
+    bad = torch.tensor([7, Lmax + 5, 300], dtype=torch.int32, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    _noalloc(lib, q, kc, vc, bad, o, lse, B, Hq, Hkv, Lmax, d)
+    assert _status(lib) == 9  # ATTN_ERR_DEVICE_ARG
+    assert "seqlens" in eio.last_error()
+    assert _status(lib) == 0  # cleared
+    assert torch.all(o[1].float() == 0) and torch.isneginf(lse[1]).all()
+    eio.sync_status()  # the library workspace's word is untouched
 
 
 def test_noalloc_rejects_oversized_shape(lib):
