@@ -1,30 +1,34 @@
 """Benchmark: exact attention on B200 through the C-ABI library.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gpt2|long|frame|decode] [--no-extra] [--no-cpu-baseline]
-                    [--backward-only | --bound-only]
+                    [--workload long|gpt2|frame|decode] [--no-extra] [--no-cpu-baseline]
+                    [--backward-only | --bound-only] [--verbose]
 
-Headline (one JSON line on rank 0): prefill attention TFLOP/s on the GPT-2
-shaped causal workload (B=8, H=12, N=1024, d=64, bf16).  One step is one
-attn_fwd call (tile plan lookup, TMA/tcgen05 kernel: S = QK^T, mask on
-partial tiles, online softmax, PV, O and LSE out).  Unless --no-extra, the
-same line carries the decode workload (B=64, Hq=32, Hkv=8, d=128, lengths
-U[1024, 8192]) in KV GB/s, the backward and the bound-based forward on the
-headline shape, and the long-context GQA and frame block-sparse prefill
-workloads, each with its own roofline fraction; every prefill entry also
-carries its tile-plan figures (`plan`).  --backward-only / --bound-only time
-just that call on the chosen workload; --workload decode makes decode the
-headline.  --impl reference times the fp64 oracle on the host cores.
+Headline (one JSON line on rank 0): prefill attention TFLOP/s on the largest
+single-GPU workload, long-context GQA causal prefill (B=1, Hq=32, Hkv=8,
+N=16384, d=128, bf16; 2.2 TFLOP per step).  One step is one attn_fwd call
+(tile plan lookup, TMA/tcgen05 kernel: S = QK^T, mask on partial tiles,
+online softmax, PV, O and LSE out).  Unless --no-extra, the same line carries
+one entry per other workload -- GPT-2 causal prefill (B=8, H=12, N=1024,
+d=64), frame block-sparse prefill (24 heads, 24 frames x 1040 tokens, d=128),
+GQA decode (B=64, Hq=32, Hkv=8, d=128, lengths U[1024, 8192]) in KV GB/s --
+each with its roofline fraction, the fp64 oracle's rate on the host cores
+(cpu_baseline) and the end-to-end rate with host buffers (e2e), plus the
+backward on the GPT-2 shape and the bound-based forward on the long-context
+workload.  The main legs come last in the line.  --verbose prints every
+leg's full record to stderr.  --impl reference times the fp64 oracle on the
+host cores.
 
 FLOPs are algorithmic: 4*d per allowed (query, key) pair.  Bytes for decode
 are algorithmic: the K and V rows below each sequence's length, read once.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
 device synchronise on both sides; each step is bracketed by CUDA events on the
-launching stream, and L2 is flushed (a 256 MiB write) before every prefill
-step; the decode cache (1.26 GB) is larger than L2.  Multi-GPU: one process
-per GPU, each rank runs its own copy of the workload (weak scaling), the
-reported time is the max over ranks.
+launching stream (the mean and the median per step are reported), and L2 is
+flushed (a 256 MiB write) before every prefill step; the decode cache
+(1.26 GB) is larger than L2.  Multi-GPU: one process per GPU, each rank runs
+its own copy of the workload (weak scaling), the reported time is the max over
+ranks.
 """
 from __future__ import annotations
 
@@ -318,7 +322,8 @@ def mask_of(w):
 
 # ------------------------------------------------------------------ timing core
 def time_steps(step, K, W, world, flush=None):
-    """W warm-ups, then K steps each bracketed by events on the current stream."""
+    """W warm-ups, then K steps each bracketed by events on the current stream.
+    Returns (mean ms, median ms, wall seconds of the timed region)."""
     import torch
     for _ in range(W):
         if flush:
@@ -340,7 +345,7 @@ def time_steps(step, K, W, world, flush=None):
     barrier(world)
     wall = time.perf_counter() - t0
     ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    return sum(ms) / K, wall
+    return sum(ms) / K, statistics.median(ms), wall
 
 
 def time_e2e_pipelined(h2d, run, d2h, steps, warmup, world, flush=None):
@@ -436,17 +441,17 @@ def bench_prefill(w, args, world, rank, peaks, with_e2e=True):
     # Eager calls first (warms the plan cache), then the same call replayed
     # from a CUDA graph: the graph time is the kernel's, the eager time adds
     # the host-side call overhead when the GPU would otherwise idle.
-    eager_ms, _ = time_steps(step, args.steps, args.warmup, world, flush)
+    eager_ms, _, _ = time_steps(step, args.steps, args.warmup, world, flush)
     graph = capture_graph(step)
-    ms, wall = time_steps(graph.replay, args.steps, args.warmup, world, flush)
+    ms, med, wall = time_steps(graph.replay, args.steps, args.warmup, world, flush)
     eio.sync_status()
-    ms = max_over_ranks(ms, world)
+    ms, med = max_over_ranks(ms, world), max_over_ranks(med, world)
     eager_ms = max_over_ranks(eager_ms, world)
     flops = prefill_flops(w)
     tflops = whole_job_rate(flops, ms, world) / 1e12
     peak = peaks["bf16_tflops"]
     out = {
-        "ms_per_step": ms, "tflops": tflops, "flops_per_step": flops,
+        "ms_per_step": ms, "ms_median": med, "tflops": tflops, "flops_per_step": flops,
         "roofline": {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak,
                      "unit": "TFLOP/s", "frac": flops / (ms * 1e-3) / 1e12 / peak,
                      "peak_source": f"{peaks['source']} bf16 burst",
@@ -482,7 +487,7 @@ def bench_prefill(w, args, world, rank, peaks, with_e2e=True):
             eio.attn_fwd(dq[i], dk[i], dv[i], o=do[i], lse=dl[i], scale=scale, mask_kind=mk, block_map=bm)
 
         ems = time_e2e_pipelined([(hq_, dq), (hk_, dk), (hv_, dv)], run, [(do, ho), (dl, hl)],
-                                 max(8, args.steps // 2), 3, world, flush)
+                                 args.steps, 3, world, flush)
         eio.sync_status()
         ems = max_over_ranks(ems, world)
         out["e2e"] = {"value": whole_job_rate(flops, ems, world) / 1e12, "unit": "TFLOP/s",
@@ -523,21 +528,22 @@ def bench_backward(w, args, world, rank, peaks):
     flush = make_flush()
     time_steps(step, 3, args.warmup, world, flush)
     graph = capture_graph(step)
-    ms, _ = time_steps(graph.replay, max(5, args.steps // 2), args.warmup, world, flush)
+    ms, med, _ = time_steps(graph.replay, args.steps, args.warmup, world, flush)
     eio.sync_status()
-    ms = max_over_ranks(ms, world)
+    ms, med = max_over_ranks(ms, world), max_over_ranks(med, world)
     flops = 2.5 * prefill_flops(w)
     tflops = whole_job_rate(flops, ms, world) / 1e12
     peak = peaks["bf16_tflops"]
     # The kernels run seven products (S and dP in both), 3.5x the forward.
     out = {"metric": "attention backward TFLOP/s", "value": tflops, "unit": "TFLOP/s", "ms_per_step": ms,
+           "ms_median": med,
            "config": {"workload": w["desc"] + ", backward (dQ, dK, dV)"},
            "roofline": {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
                         "frac": flops / (ms * 1e-3) / 1e12 / peak, "peak_source": f"{peaks['source']} bf16 burst",
                         "executed_frac": 1.4 * flops / (ms * 1e-3) / 1e12 / peak,
                         "kernel": "bwd_dq + bwd_dkdv (one call)",
                         "traffic": recorded_traffic(f"backward_{args_key(w)}")},
-           "gpu_launches": 2 * max(5, args.steps // 2)}
+           "gpu_launches": 2 * args.steps}
     del tq, tk, tv, tdo, o, lse, dq, dk, dv
     torch.cuda.empty_cache()
     return out
@@ -570,12 +576,13 @@ def bench_bound(w, args, world, rank, peaks):
                            n_fallback=nfb)
 
     flush = make_flush()
-    steps = max(5, args.steps // 2)
+    steps = args.steps
     stats()
     time_steps(fwd, 3, args.warmup, world, flush)
     g_stats, g_fwd = capture_graph(stats), capture_graph(fwd)
-    ms_stats, _ = time_steps(g_stats.replay, steps, args.warmup, world, flush)
-    ms_fwd, _ = time_steps(g_fwd.replay, steps, args.warmup, world, flush)
+    ms_stats, _, _ = time_steps(g_stats.replay, steps, args.warmup, world, flush)
+    ms_fwd, med_fwd, _ = time_steps(g_fwd.replay, steps, args.warmup, world, flush)
+    med_fwd = max_over_ranks(med_fwd, world)
     eio.sync_status()
     ms_stats, ms_fwd = max_over_ranks(ms_stats, world), max_over_ranks(ms_fwd, world)
     nfb.zero_()
@@ -584,7 +591,7 @@ def bench_bound(w, args, world, rank, peaks):
     flops = prefill_flops(w)
     peak = peaks["bf16_tflops"]
     out = {"metric": "prefill attn TFLOP/s (bound-based softmax)", "value": whole_job_rate(flops, ms_fwd, world) / 1e12,
-           "unit": "TFLOP/s", "ms_per_step": ms_fwd, "key_stats_ms": ms_stats,
+           "unit": "TFLOP/s", "ms_per_step": ms_fwd, "ms_median": med_fwd, "key_stats_ms": ms_stats,
            "value_with_key_stats": whole_job_rate(flops, ms_fwd + ms_stats, world) / 1e12,
            "fallback_rows": int(nfb.item()),
            "config": {"workload": w["desc"] + ", attn_fwd_bound (key statistics precomputed)"},
@@ -622,18 +629,18 @@ def bench_decode(w, args, world, rank, peaks, with_e2e=True):
         eio.attn_decode(tq, tk, tv, tl, o=o, lse=lse, scale=scale)
 
     steps = max(args.steps, 20)
-    eager_ms, _ = time_steps(step, steps, args.warmup, world)
+    eager_ms, _, _ = time_steps(step, steps, args.warmup, world)
     graph = capture_graph(step)
-    ms, wall = time_steps(graph.replay, steps, args.warmup, world)
+    ms, med, wall = time_steps(graph.replay, steps, args.warmup, world)
     eio.sync_status()
-    ms = max_over_ranks(ms, world)
+    ms, med = max_over_ranks(ms, world), max_over_ranks(med, world)
     eager_ms = max_over_ranks(eager_ms, world)
     kvb = decode_kv_bytes(lens, Hkv, d)
     alg = kvb + q.nbytes * 2 + B * Hq * 4
     gbs = whole_job_rate(alg, ms, world) / 1e9
     peak = peaks["hbm_gbs"]
     out = {
-        "metric": "decode KV GB/s", "value": gbs, "unit": "GB/s", "ms_per_step": ms,
+        "metric": "decode KV GB/s", "value": gbs, "unit": "GB/s", "ms_per_step": ms, "ms_median": med,
         "config": {"workload": w["desc"], "sum_len": int(lens.sum()), "kv_bytes": kvb,
                    "l2": "cache (1.26 GB) larger than L2; no flush"},
         "roofline": {"bound": "hbm", "achieved": alg / (ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
@@ -656,7 +663,7 @@ def bench_decode(w, args, world, rank, peaks, with_e2e=True):
     if w["Hq"] // w["Hkv"] * 2 <= 8:
         time_steps(step2, 3, args.warmup, world)
         g2 = capture_graph(step2)
-        ms2, _ = time_steps(g2.replay, steps, args.warmup, world)
+        ms2, _, _ = time_steps(g2.replay, steps, args.warmup, world)
         eio.sync_status()
         ms2 = max_over_ranks(ms2, world)
         out["multi_token_2"] = {"metric": "decode KV GB/s, 2 new tokens per sequence",
@@ -730,7 +737,7 @@ def oracle_prefill_call(w, seed, row_budget_flops=2e10):
     return run, f"{n} sampled (batch, head, query) rows of the workload"
 
 
-def oracle_prefill_sample(w, seed, min_seconds=10.0, max_passes=200):
+def oracle_prefill_sample(w, seed, min_seconds=8.0, max_passes=200):
     """Repeat bounded oracle passes until `min_seconds` of CPU work; returns
     (seconds, flops, description)."""
     run, desc = oracle_prefill_call(w, seed)
@@ -763,7 +770,7 @@ def oracle_decode_call(w, seed, n_seq=8):
     return run, f"the first {n} of {B} sequences ({int(lens.sum())} cached keys)", nbytes
 
 
-def oracle_decode_baseline(w, seed, min_seconds=5.0):
+def oracle_decode_baseline(w, seed, min_seconds=6.0):
     """The cpu_baseline of a decode line: the oracle's decode of a sample of
     the batch (oracle_decode_call), repeated for at least min_seconds."""
     import oracle
@@ -777,7 +784,7 @@ def oracle_decode_baseline(w, seed, min_seconds=5.0):
         dt += time.perf_counter() - t0
         n += 1
     return {"value": nbytes * n / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{desc}, {n} passes, fp64, {dt:.1f} s"}
+            "sample": f"{desc}, {n} passes, fp64, {dt:.1f} s", "cpu": cpu_model()}
 
 
 def cpu_cores():
@@ -785,6 +792,30 @@ def cpu_cores():
         return len(os.sched_getaffinity(0))
     except Exception:
         return os.cpu_count()
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), for the CPU baselines."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_prefill_baseline(w, seed, min_seconds=8.0):
+    """The cpu_baseline of a prefill leg: the oracle on a bounded sample of
+    the workload (oracle_prefill_call), repeated for at least min_seconds."""
+    import oracle
+    oracle.build()
+    cores = oracle.threads(cpu_cores())
+    dt, fl, desc = oracle_prefill_sample(w, seed, min_seconds=min_seconds)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+            "cpu": cpu_model()}
 
 
 def run_reference(args, world, rank):
@@ -816,7 +847,7 @@ def run_reference(args, world, rank):
         "data": "synthetic",
         "config": {"workload": w["desc"], "sample": f"{desc} per step"},
         "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{desc} per step, {args.steps} steps, fp64"},
+                         "sample": f"{desc} per step, {args.steps} steps, fp64", "cpu": cpu_model()},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -840,25 +871,64 @@ def run_reference_decode(args, w, cores):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w["desc"], "sample": f"{desc} per step"},
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{desc} per step, {args.steps} steps, fp64"},
+                         "sample": f"{desc} per step, {args.steps} steps, fp64", "cpu": cpu_model()},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
+def sig(x, n=4):
+    """x rounded to n significant digits (keeps the JSON line short)."""
+    if not isinstance(x, float) or x == 0 or not math.isfinite(x):
+        return x
+    return round(x, -int(math.floor(math.log10(abs(x)))) + n - 1)
+
+
+def short(d, keys):
+    return {k: sig(d[k]) for k in keys if k in d and d[k] is not None}
+
+
+ROOF_KEYS = ("bound", "achieved", "peak", "unit", "frac", "traffic")
+
+
+def leg(workload, r, value, unit, cpu=None):
+    """One workload's entry in the JSON line: the rate (the unit names the
+    metric: TFLOP/s of prefill or backward attention, KV GB/s of decode), mean
+    and median step times, the roofline of its dominant kernel, the oracle
+    baseline and the end-to-end rate (both when measured)."""
+    out = {"workload": workload, "value": sig(value), "unit": unit,
+           "ms": sig(r["ms_per_step"]), "ms_median": sig(r.get("ms_median")),
+           "roofline": short(r["roofline"], ROOF_KEYS)}
+    if "executed_frac" in r["roofline"]:
+        out["roofline"]["executed_frac"] = sig(r["roofline"]["executed_frac"])
+    if cpu is not None:
+        out["cpu_baseline"] = short(cpu, ("value", "unit", "cores", "kind"))
+    if r.get("e2e"):
+        out["e2e"] = short(r["e2e"], ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"))
+    return out
+
+
+SHORT_NAMES = {"gpt2": "GPT-2 causal B=8 H=12 N=1024 d=64",
+               "long": "long GQA causal B=1 Hq=32 Hkv=8 N=16384 d=128",
+               "frame": "frame block-sparse H=24 24x1040 d=128",
+               "decode": "GQA decode B=64 Hq=32 Hkv=8 d=128 len U[1024,8192]"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="gpt2", choices=["gpt2", "long", "frame", "decode"])
-    ap.add_argument("--no-extra", action="store_true", help="skip the decode / other prefill workloads")
+    ap.add_argument("--workload", default="long", choices=["gpt2", "long", "frame", "decode"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only attn_bwd on the chosen prefill workload (one JSON line)")
     ap.add_argument("--bound-only", action="store_true",
                     help="time only attn_fwd_bound (and attn_key_stats) on the chosen prefill workload")
+    ap.add_argument("--verbose", action="store_true",
+                    help="also print every leg's full record (plans, eager times, second rooflines) to stderr")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -882,6 +952,7 @@ def main():
     eio.lib()
     peaks = measured_peaks()
     w = WORKLOADS[args.workload]
+    one = rank == 0 and world == 1 and not args.no_cpu_baseline  # the oracle baselines: one-GPU runs only
 
     sampler = ClockSampler(torch.cuda.current_device())
     if args.backward_only or args.bound_only:
@@ -890,7 +961,7 @@ def main():
         with sampler:
             d = (bench_backward if args.backward_only else bench_bound)(w, args, world, rank, peaks)
         if rank == 0:
-            d.update({"n_gpus": world, "steps": max(5, args.steps // 2), "warmup": args.warmup,
+            d.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                       "higher_is_better": True, "scaling": "weak",
                       "dtype": "bf16", "data": "synthetic", "clocks": sampler.summary()})
             print(json.dumps(d), flush=True)
@@ -898,68 +969,85 @@ def main():
             import torch.distributed as dist
             dist.destroy_process_group()
         return
-    if args.workload == "decode":
-        with sampler:
-            d = bench_decode(w, args, world, rank, peaks)
-        cpu = None
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            cpu = oracle_decode_baseline(w, rank_seed(w["seed"], 0))
-        if rank == 0:
-            line = {"metric": d["metric"], "value": d["value"], "unit": d["unit"], "n_gpus": world,
-                    "steps": d["steps"], "warmup": args.warmup, "ms_per_step": d["ms_per_step"],
-                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-                    "data": "synthetic", "config": d["config"], "roofline": d["roofline"], "e2e": d["e2e"],
-                    "gpu_launches": d["gpu_launches"], "clocks": sampler.summary(), "cpu_baseline": cpu,
-                    "multi_token_2": d.get("multi_token_2")}
-            print(json.dumps(line), flush=True)
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        return
+
+    detail = {}
+    legs = {}
     with sampler:
-        head = bench_prefill(w, args, world, rank, peaks)
-        extra = {}
+        if args.workload == "decode":
+            head = bench_decode(w, args, world, rank, peaks)
+        else:
+            head = bench_prefill(w, args, world, rank, peaks)
+        detail[args.workload] = head
         if not args.no_extra:
-            extra["decode"] = bench_decode(WORKLOADS["decode"], args, world, rank, peaks)
-            extra["backward"] = bench_backward(w, args, world, rank, peaks)
-            extra["bound"] = bench_bound(w, args, world, rank, peaks)
-            for name in ("long", "frame"):
+            for name in ("gpt2", "long", "frame", "decode"):
                 if name == args.workload:
                     continue
                 wx = WORKLOADS[name]
-                r = bench_prefill(wx, argparse.Namespace(steps=max(5, args.steps // 5), warmup=3),
-                                  world, rank, peaks, with_e2e=False)
-                extra[name] = {"metric": "prefill attn TFLOP/s", "value": r["tflops"], "unit": "TFLOP/s",
-                               "ms_per_step": r["ms_per_step"], "eager_ms_per_step": r["eager_ms_per_step"],
-                               "config": {"workload": wx["desc"]},
-                               "roofline": r["roofline"], "roofline_exp": r["roofline_exp"],
-                               "gpu_launches": r["gpu_launches"], "plan": plan_stats(wx)}
+                r = (bench_decode if name == "decode" else bench_prefill)(wx, args, world, rank, peaks)
+                detail[name] = r
+            g = WORKLOADS["gpt2"]
+            detail["backward"] = bench_backward(g, args, world, rank, peaks)
+            detail["bound"] = bench_bound(WORKLOADS["long"], args, world, rank, peaks)
+    if args.verbose:
+        for name, r in detail.items():
+            if name in WORKLOADS and WORKLOADS[name]["kind"] == "prefill":
+                r["plan"] = plan_stats(WORKLOADS[name])
 
-    cpu = None  # the oracle baseline: rank 0 of a one-GPU run only, so scaling runs hold no GPU idle for it
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        oracle.build()
-        cores = oracle.threads(cpu_cores())
-        dt, fl, desc = oracle_prefill_sample(w, rank_seed(w["seed"], 0))
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-               "sample": desc}
+    cpu = {}  # the oracle on a bounded sample of each workload, on the host cores, after the GPU legs
+    if one:
+        for name in detail:
+            if name in WORKLOADS:
+                seed = rank_seed(WORKLOADS[name]["seed"], 0)
+                cpu[name] = (oracle_decode_baseline(WORKLOADS[name], seed) if name == "decode"
+                             else oracle_prefill_baseline(WORKLOADS[name], seed))
 
     if rank == 0:
+        if args.verbose:
+            print("bench detail: " + json.dumps(detail), file=sys.stderr, flush=True)
+        for name in ("gpt2", "frame", "long", "decode"):
+            if name in detail and name != args.workload:
+                r = detail[name]
+                if name == "decode":
+                    legs[name] = leg(SHORT_NAMES[name], r, r["value"], "GB/s", cpu.get(name))
+                    if r.get("multi_token_2"):
+                        legs[name]["multi_token_2"] = short(r["multi_token_2"], ("value", "unit", "ms_per_step"))
+                else:
+                    legs[name] = leg(SHORT_NAMES[name], r, r["tflops"], "TFLOP/s", cpu.get(name))
+        if "backward" in detail:
+            legs["backward"] = leg(SHORT_NAMES["gpt2"] + ", backward dQ dK dV, FLOPs 2.5x forward",
+                                   detail["backward"], detail["backward"]["value"], "TFLOP/s")
+        if "bound" in detail:
+            b = detail["bound"]
+            legs["bound"] = leg(SHORT_NAMES["long"] + ", bound-based softmax", b, b["value"], "TFLOP/s")
+            legs["bound"]["key_stats_ms"] = sig(b["key_stats_ms"])
+        order = ["backward", "bound", "gpt2", "frame", "long", "decode"]  # the main legs last
+        if args.workload == "decode":
+            metric, unit, value = "decode KV GB/s", "GB/s", head["value"]
+            l2 = "cache (1.26 GB) larger than L2; no flush"
+            launches = head["gpu_launches"]
+        else:
+            metric, unit, value = "prefill attn TFLOP/s", "TFLOP/s", head["tflops"]
+            l2 = "flushed before every step (256 MiB write)"
+            launches = head["gpu_launches"]
+        hc = cpu.get(args.workload)
         line = {
-            "metric": "prefill attn TFLOP/s", "value": head["tflops"], "unit": "TFLOP/s",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w["desc"], "parallelism": f"replicas x{world} (independent batches)",
-                       "l2": "flushed before every step (256 MiB write)",
-                       "flops_per_step_per_gpu": head["flops_per_step"]},
-            "roofline": head["roofline"], "roofline_exp": head["roofline_exp"],
-            "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
-            "eager_ms_per_step": head["eager_ms_per_step"], "timing": head["timing"],
-            "clocks": sampler.summary(), "cpu_baseline": cpu, "plan": plan_stats(w),
+            "metric": metric, "value": sig(value), "unit": unit, "n_gpus": world,
+            "steps": head.get("steps", args.steps), "warmup": args.warmup,
+            "ms_per_step": sig(head["ms_per_step"]), "ms_median": sig(head.get("ms_median")),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w["desc"], "parallelism": f"replicas x{world}", "l2": l2},
+            "roofline": dict(short(head["roofline"], ROOF_KEYS), peak_source=head["roofline"]["peak_source"]),
+            "cpu_baseline": hc, "e2e": short(head["e2e"], ("value", "unit", "h2d_bytes_per_step",
+                                                            "d2h_bytes_per_step")),
+            "gpu_launches": launches, "clocks": short(sampler.summary(), ("sm_mhz", "sm_max_mhz", "reasons")),
         }
-        line.update(extra)
-        print(json.dumps(line), flush=True)
+        if hc is not None:
+            line["cpu_baseline"] = dict(short(hc, ("value", "unit", "cores", "kind")), sample=hc["sample"],
+                                        cpu=hc["cpu"])
+        for name in order:
+            if name in legs:
+                line[name] = legs[name]
+        print(json.dumps(line, separators=(",", ":")), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
