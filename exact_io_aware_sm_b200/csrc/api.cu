@@ -531,8 +531,8 @@ int attn_decode_multi(const void* q, const void* k_cache, const void* v_cache, c
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8)
     return set_err(ATTN_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1, 2, 4, 8}, got %d", G);
-  if (G * Sq > 8)
-    return set_err(ATTN_ERR_UNSUPPORTED, "decode needs (Hq/Hkv) * Sq <= 8, got %d * %d", G, Sq);
+  if (G * Sq > 16)
+    return set_err(ATTN_ERR_UNSUPPORTED, "decode needs (Hq/Hkv) * Sq <= 16, got %d * %d", G, Sq);
   if (static_cast<long long>(B) * Sq * Hq > (1ll << 30)) return set_err(ATTN_ERR_SHAPE, "too many query rows");
   if (d != 64 && d != 128) return set_err(ATTN_ERR_UNSUPPORTED, "decode needs d in {64, 128}");
   if (!(scale > 0.f) || !std::isfinite(scale))

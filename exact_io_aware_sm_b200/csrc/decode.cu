@@ -18,10 +18,12 @@
 //     Each warp is its own pipeline: a ring of 32-key stages (K and V tiles
 //     brought in by TMA, 128-byte swizzle) that it refills as it consumes, so
 //     every warp keeps up to 48 KB of loads in flight.  The G query heads x Sq
-//     tokens of the item (at most 8) share every K/V tile:
+//     tokens of the item (at most 16) share every K/V tile; they fill one or
+//     two groups of 8 MMA columns (NCG):
 //       S^T (16 keys x 8 columns) = K (16 x d) q^T     mma.m16n8k16, K by ldmatrix
 //       online softmax on the fragment (max over the 16 keys by 3 shuffles)
 //       O^T (d x 8 columns) += V^T (d x 16) P^T       V by ldmatrix.trans, P^T by movmatrix
+//     per column group, the K and V fragments loaded once for both groups.
 //     Columns past G * Sq are zero.  The output is a normalised partial O
 //     and its log2-sum-exp per (sequence, query head, split).
 //   decode_combine_kernel  one CTA per (sequence, token, query head): merges the
@@ -72,14 +74,14 @@ struct Cursor {
   int b, hkv, split, k, kend;
 };
 
-template <int D, int G>
+template <int D, int G, int NCG>
 __global__ void __launch_bounds__(kWarps * 32, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const DecodeArgs a) {
   using C = DCfg<D>;
   constexpr int R = C::R, KB = C::KB;
   constexpr int NK = D / 16;  // k-steps of S, m-tiles of O
-  const int NC = G * a.Sq;    // live columns of the 8: (head, token) pairs of the group
+  const int NC = G * a.Sq;    // live columns of the 8 * NCG: (head, token) pairs of the group
   extern __shared__ uint8_t dsmem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
 
@@ -178,9 +180,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   __syncwarp();
 
   const float sl2 = a.scale_log2;
-  uint32_t qf[NK][2];
-  float acc[NK][4];
-  float m[2], l[2];
+  uint32_t qf[NCG][NK][2];
+  float acc[NCG][NK][4];
+  float m[NCG][2], l[NCG][2];
   bool ok = true;
 
   while (consumed < produced) {
@@ -198,23 +200,27 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     const uint32_t vt = kt + C::kTileBytes;
 
     if (flags & 1) {  // first stage of an item: this item's queries, fresh state
-      // Column g of q^T is (head g / Sq, token g % Sq) of this KV group.
-      const bool live = g < NC;
-      const int gc = live ? g : 0;
-      const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                                  ((static_cast<size_t>(b) * a.Sq + gc % a.Sq) * a.Hq + hkv * G + gc / a.Sq) * D +
-                                  2 * t;
 #pragma unroll
-      for (int ks = 0; ks < NK; ++ks) {
-        qf[ks][0] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks) : 0u;
-        qf[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8) : 0u;
+      for (int cg = 0; cg < NCG; ++cg) {
+        // Column cg*8 + g of q^T is (head c / Sq, token c % Sq) of this KV group.
+        const int c = cg * 8 + g;
+        const bool live = c < NC;
+        const int gc = live ? c : 0;
+        const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(a.q) +
+                                    ((static_cast<size_t>(b) * a.Sq + gc % a.Sq) * a.Hq + hkv * G + gc / a.Sq) * D +
+                                    2 * t;
+#pragma unroll
+        for (int ks = 0; ks < NK; ++ks) {
+          qf[cg][ks][0] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks) : 0u;
+          qf[cg][ks][1] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8) : 0u;
+        }
+#pragma unroll
+        for (int mt = 0; mt < NK; ++mt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[cg][mt][i] = 0.f;
+        m[cg][0] = m[cg][1] = -INFINITY;
+        l[cg][0] = l[cg][1] = 0.f;
       }
-#pragma unroll
-      for (int mt = 0; mt < NK; ++mt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
-      m[0] = m[1] = -INFINITY;
-      l[0] = l[1] = 0.f;
     }
     if (nvalid < kStageKeys) {
       // V rows past the sequence (read by the last box, or stale) must be
@@ -228,19 +234,21 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     }
 
     const int nch = nvalid > 16 ? 2 : 1;
-    // Keys of this stage visible to the lane's two columns 2t, 2t+1: token s
+    // Keys of this stage visible to the lane's columns cg*8 + 2t + j: token s
     // (of Sq, the last at position len - 1) sees keys 0 .. len - Sq + s.
-    int lim[2] = {nvalid, nvalid};
-    if (a.Sq > 1) {
-      const int len = lens[b];
+    int lim[NCG][2];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) lim[j] = min(nvalid, len - a.Sq + (2 * t + j) % a.Sq + 1 - k0);
-    }
-    float s[2][4];
+    for (int cg = 0; cg < NCG; ++cg)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        lim[cg][j] = a.Sq > 1 ? min(nvalid, lens[b] - a.Sq + (cg * 8 + 2 * t + j) % a.Sq + 1 - k0) : nvalid;
+    float s[2][NCG][4];
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) s[ch][i] = 0.f;
+      for (int cg = 0; cg < NCG; ++cg)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[ch][cg][i] = 0.f;
       if (ch < nch) {
         const int r = ch * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
@@ -248,85 +256,99 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
           const int cc = (ks & 3) * 2 + (lane >> 4);
           uint32_t af[4];
           ldsm_x4(kt + (ks >> 2) * C::kBlockBytes + r * 128 + ((cc ^ (r & 7)) << 4), af);
-          mma_16816(s[ch], af, qf[ks][0], qf[ks][1]);
+#pragma unroll
+          for (int cg = 0; cg < NCG; ++cg) mma_16816(s[ch][cg], af, qf[cg][ks][0], qf[cg][ks][1]);
         }
       }
       // keys past the valid ones, and past each token's own position, carry no weight
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int key = ch * 16 + g + (i >> 1) * 8;
-        if (key >= lim[i & 1]) s[ch][i] = -INFINITY;
-      }
+      for (int cg = 0; cg < NCG; ++cg)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int key = ch * 16 + g + (i >> 1) * 8;
+          if (key >= lim[cg][i & 1]) s[ch][cg][i] = -INFINITY;
+        }
     }
 
-    // Running max per head (2t and 2t+1), over the 32 keys of the stage.
+    // Running max per column (cg*8 + 2t and + 1), over the 32 keys of the stage.
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      float v = fmaxf(fmaxf(s[0][j], s[0][j + 2]), fmaxf(s[1][j], s[1][j + 2]));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-      v *= sl2;
-      if (v > m[j] + kRebase) {  // move the base (always on the first stage)
-        const float alpha = wm_ex2(m[j] - v);
-        l[j] *= alpha;
+    for (int cg = 0; cg < NCG; ++cg)
 #pragma unroll
-        for (int mt = 0; mt < NK; ++mt) {
-          acc[mt][j] *= alpha;
-          acc[mt][j + 2] *= alpha;
+      for (int j = 0; j < 2; ++j) {
+        float v = fmaxf(fmaxf(s[0][cg][j], s[0][cg][j + 2]), fmaxf(s[1][cg][j], s[1][cg][j + 2]));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        v *= sl2;
+        if (v > m[cg][j] + kRebase) {  // move the base (always on the first stage)
+          const float alpha = wm_ex2(m[cg][j] - v);
+          l[cg][j] *= alpha;
+#pragma unroll
+          for (int mt = 0; mt < NK; ++mt) {
+            acc[cg][mt][j] *= alpha;
+            acc[cg][mt][j + 2] *= alpha;
+          }
+          m[cg][j] = v;
         }
-        m[j] = v;
       }
-    }
 
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
       if (ch < nch) {
-        float p[4];
+        uint32_t pb[NCG][2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          // a column that has seen no key yet keeps m = -inf: its p are 0
-          p[i] = wm_ex2(fmaf(s[ch][i], sl2, m[i & 1] == -INFINITY ? 0.f : -m[i & 1]));
-          l[i & 1] += p[i];
+        for (int cg = 0; cg < NCG; ++cg) {
+          float p[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            // a column that has seen no key yet keeps m = -inf: its p are 0
+            const float mb = m[cg][i & 1];
+            p[i] = wm_ex2(fmaf(s[ch][cg][i], sl2, mb == -INFINITY ? 0.f : -mb));
+            l[cg][i & 1] += p[i];
+          }
+          pb[cg][0] = movmatrix_trans(wm_pack_bf16x2(p[0], p[1]));
+          pb[cg][1] = movmatrix_trans(wm_pack_bf16x2(p[2], p[3]));
         }
-        const uint32_t b0 = movmatrix_trans(wm_pack_bf16x2(p[0], p[1]));
-        const uint32_t b1 = movmatrix_trans(wm_pack_bf16x2(p[2], p[3]));
         const int r = ch * 16 + (lane >> 4) * 8 + (lane & 7);
 #pragma unroll
         for (int mt = 0; mt < NK; ++mt) {
           const int cc = (mt & 3) * 2 + ((lane >> 3) & 1);
           uint32_t af[4];
           ldsm_x4_trans(vt + (mt >> 2) * C::kBlockBytes + r * 128 + ((cc ^ (r & 7)) << 4), af);
-          mma_16816(acc[mt], af, b0, b1);
+#pragma unroll
+          for (int cg = 0; cg < NCG; ++cg) mma_16816(acc[cg][mt], af, pb[cg][0], pb[cg][1]);
         }
       }
     }
 
     if (flags & 2) {  // last stage of the item: normalise and write the partial
-      float lt[2];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float v = l[j];
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
-        lt[j] = v;
-      }
+      for (int cg = 0; cg < NCG; ++cg) {
+        float lt[2];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int col = 2 * t + j;
-        if (col < NC) {
-          const size_t row = (static_cast<size_t>(b) * a.Sq + col % a.Sq) * a.Hq + hkv * G + col / a.Sq;
-          const size_t p = row * a.nsplit + split;
-          // a token may see no key of this split (its position precedes it)
-          const float inv = lt[j] > 0.f ? 1.f / lt[j] : 0.f;
-          float* op = a.opart + p * D;
+        for (int j = 0; j < 2; ++j) {
+          float v = l[cg][j];
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
+          lt[j] = v;
+        }
 #pragma unroll
-          for (int mt = 0; mt < NK; ++mt) {
-            op[16 * mt + g] = acc[mt][j] * inv;
-            op[16 * mt + g + 8] = acc[mt][j + 2] * inv;
+        for (int j = 0; j < 2; ++j) {
+          const int col = cg * 8 + 2 * t + j;
+          if (col < NC) {
+            const size_t row = (static_cast<size_t>(b) * a.Sq + col % a.Sq) * a.Hq + hkv * G + col / a.Sq;
+            const size_t p = row * a.nsplit + split;
+            // a token may see no key of this split (its position precedes it)
+            const float inv = lt[j] > 0.f ? 1.f / lt[j] : 0.f;
+            float* op = a.opart + p * D;
+#pragma unroll
+            for (int mt = 0; mt < NK; ++mt) {
+              op[16 * mt + g] = acc[cg][mt][j] * inv;
+              op[16 * mt + g + 8] = acc[cg][mt][j + 2] * inv;
+            }
+            if (g == 0) a.lpart[p] = lt[j] > 0.f ? m[cg][j] + __log2f(lt[j]) : -INFINITY;
           }
-          if (g == 0) a.lpart[p] = lt[j] > 0.f ? m[j] + __log2f(lt[j]) : -INFINITY;
         }
       }
     }
@@ -379,13 +401,13 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
 
 
 
-template <int D, int G>
+template <int D, int G, int NCG>
 cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
   static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set.test(dev)) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G, NCG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          DCfg<D>::kSmem);
     if (e != cudaSuccess) return e;
     attr_set.set(dev);
@@ -413,7 +435,7 @@ cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
     const long long items = static_cast<long long>(c.B) * a.nsplit * a.Hkv;
     const long long want = (items + kWarps - 1) / kWarps;
     const int grid = static_cast<int>(want < sms ? want : sms);
-    decode_split_kernel<D, G><<<grid, kWarps * 32, DCfg<D>::kSmem, s>>>(tk, tv, c);
+    decode_split_kernel<D, G, NCG><<<grid, kWarps * 32, DCfg<D>::kSmem, s>>>(tk, tv, c);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -423,11 +445,13 @@ cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
 
 template <int D>
 cudaError_t launch_d(int G, const DecodeArgs& a, cudaStream_t s) {
+  // One group of 8 MMA columns holds up to 8 (head, token) pairs, two up to 16.
+  const bool two = G * a.Sq > 8;
   switch (G) {
-    case 1: return launch_dg<D, 1>(a, s);
-    case 2: return launch_dg<D, 2>(a, s);
-    case 4: return launch_dg<D, 4>(a, s);
-    case 8: return launch_dg<D, 8>(a, s);
+    case 1: return two ? launch_dg<D, 1, 2>(a, s) : launch_dg<D, 1, 1>(a, s);
+    case 2: return two ? launch_dg<D, 2, 2>(a, s) : launch_dg<D, 2, 1>(a, s);
+    case 4: return two ? launch_dg<D, 4, 2>(a, s) : launch_dg<D, 4, 1>(a, s);
+    case 8: return two ? launch_dg<D, 8, 2>(a, s) : launch_dg<D, 8, 1>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -97,7 +97,7 @@ struct DecodeArgs {
   int* err;
   int* counter;     // work-item counters, one per group of 2048 sequences; zero before the call, zeroed after
   int B, Hq, Hkv, Lmax, nsplit;
-  int Sq;           // query tokens per sequence (the newest Sq positions); G * Sq <= 8
+  int Sq;           // query tokens per sequence (the newest Sq positions); G * Sq <= 16
   float scale_log2;
 };
 constexpr int kDecodeMaxCounters = 63;  // sequence groups one call may need (B <= 65535)

@@ -35,8 +35,9 @@
 // base, so the result is exactly softmax(S) V while most rescales vanish.
 //
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+d), O_B after O_A.
-// d = 128: P_X overwrites the first 64 columns of S_X, so the MMA issuer
-// orders S_X(j+1) after PV_X(j) has completed.  d = 64 leaves 128 columns
+// d = 128: P_X overwrites the first 64 columns of S_X; the MMA issuer issues
+// S_X(j+1) right after PV_X(j), and the tensor core's in-order execution of
+// one thread's MMAs keeps the overwrite behind that PV's read of P.  d = 64 leaves 128 columns
 // free: P_A [384,448) and P_B [448,512) have their own, and S_X(j+1) is
 // issued as soon as the softmax threads have loaded S_X(j) into registers,
 // so it overlaps their exponentials.
@@ -312,8 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             &q_full[x * QB + qb], ch * 64, headX[x], rowX[x], it.b);
         qcnt[x]++;
       }
+      int4 kt_next = it.nB > 0 ? a.kvtiles[it.kv_first] : make_int4(0, 0, 0, 0);
       for (int j = 0; ok && j < it.nB; ++j) {
-        const int4 kt = a.kvtiles[it.kv_first + j];
+        const int4 kt = kt_next;  // read one tile ahead of its use
+        if (j + 1 < it.nB) kt_next = a.kvtiles[it.kv_first + j + 1];
         for (int t = 0; t < 2; ++t) {
           const uint32_t slot = seq % R;
           if (seq >= R && !wwait(&ring_empty[slot], ((seq / R) + 1) & 1)) {
@@ -382,12 +385,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // S_X = Q_X K^T for the K tile in ring slot kslot; releases the stage.
     auto issue_s = [&](uint32_t qbase, int ncols, uint32_t kslot) {
-      if (scnt > 0) {
-        // S_X is rewritten: the softmax must have loaded it (separate P) or
-        // the PV that read P from its columns must have completed.
-        if (C::kSepP ? !wait_bar(&s_free[x], (scnt - 1) & 1) : !wait_bar(&pv_done[x], (pcnt - 1) & 1))
-          return;
-      }
+      // S_X is rewritten.  Separate P: the softmax must have loaded S_X.  P in
+      // S's columns: the PV that reads P was issued just before by this
+      // thread, and the tensor core executes one thread's MMAs in issue
+      // order, so this S overwrites P only after that PV has read it.
+      if (C::kSepP && scnt > 0 && !wait_bar(&s_free[x], (scnt - 1) & 1)) return;
       tc_fence_after();
       const uint32_t id = idesc_bf16_f32(128, static_cast<uint32_t>(ncols), 0, 0);
       const uint32_t kbase = sRing + kslot * C::kTileBytes;
@@ -424,6 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nX = x == 0 ? it.nA : it.nB;
       const int nB = it.nB;
       const int4* kv = a.kvtiles + it.kv_first;
+      // Tile widths are read one tile ahead of their use.
+      int nc_cur = nX > 0 ? kv[0].y : 0, nc_next = nX > 1 ? kv[1].y : 0;
       uint32_t qbuf = 0;
       if (nX > 0) {
         qbuf = qcnt % QB;
@@ -431,20 +435,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         qcnt++;
         const uint32_t qbase = sQ + (x * QB + qbuf) * C::kTileBytes;
         if (!wait_bar(&ring_full[seq % R], (seq / R) & 1)) break;
-        issue_s(qbase, kv[0].y, seq % R);
+        issue_s(qbase, nc_cur, seq % R);
         for (int j = 0; ok && j < nX; ++j) {
           const uint32_t vseq = seq + 2 * j + 1, kseq = vseq + 1;
           const bool next = j + 1 < nX;
+          const int nc_after = j + 2 < nX ? kv[j + 2].y : 0;
           if (C::kSepP && next) {  // next S as soon as the softmax has loaded this one
             if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
-            issue_s(qbase, kv[j + 1].y, kseq % R);
+            issue_s(qbase, nc_next, kseq % R);
           }
           if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
-          issue_pv(j, kv[j].y, vseq % R);
-          if (!C::kSepP && next) {  // P shares S's columns: after this PV
+          issue_pv(j, nc_cur, vseq % R);
+          if (!C::kSepP && next) {  // P shares S's columns: right after this PV
             if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
-            issue_s(qbase, kv[j + 1].y, kseq % R);
+            issue_s(qbase, nc_next, kseq % R);
           }
+          nc_cur = nc_next;
+          nc_next = nc_after;
         }
         ocnt++;
       }
@@ -524,9 +531,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (stagger) bcnt++;
       const int4* kv = a.kvtiles + it.kv_first;
       float l = 0.f;
+      int4 kt_next = nX > 0 ? kv[0] : make_int4(0, 0, 0, 0);
 
       for (int t = 0; t < nX; ++t) {
-        const int4 kt = kv[t];
+        const int4 kt = kt_next;
+        if (t + 1 < nX) kt_next = kv[t + 1];
         const int nc = kt.y;
         if (!warp_wait(&s_full[x], tcnt & 1)) {
           ok = false;

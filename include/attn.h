@@ -147,9 +147,9 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
  *   o         device, [B, Sq, Hq, d] bf16 (written)
  *   lse       device, [B, Hq, Sq] fp32 (written); may be NULL
  * A token that sees no row (seqlens[b] - Sq + s < 0) gets O = 0, LSE = -inf.
- * Limits: as attn_decode, and (Hq / Hkv) * Sq <= 8 (the query heads of a KV
- * group times the tokens share one 8-column MMA operand), else
- * ATTN_ERR_UNSUPPORTED.  Sq = 1 is attn_decode.
+ * Limits: as attn_decode, and (Hq / Hkv) * Sq <= 16 (the query heads of a KV
+ * group times the tokens fill one or two 8-column MMA operands that share
+ * every K/V fragment), else ATTN_ERR_UNSUPPORTED.  Sq = 1 is attn_decode.
  * Scratch: B*Sq*Hq*ceil(Lmax/512)*(d+1) floats of library workspace.
  */
 int attn_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,

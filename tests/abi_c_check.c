@@ -80,8 +80,8 @@ int main(void) {
                   NULL) == ATTN_ERR_MASK); /* BLOCK without a map */
   EXPECT(attn_decode(fake, fake, fake, (const int32_t*)fake, fake, NULL, 1, 12, 4, 64, 128, 0.1f, NULL) ==
          ATTN_ERR_UNSUPPORTED); /* 3 query heads per KV head */
-  EXPECT(attn_decode_multi(fake, fake, fake, (const int32_t*)fake, fake, NULL, 1, 3, 8, 2, 64, 128, 0.1f, NULL) ==
-         ATTN_ERR_UNSUPPORTED); /* (Hq/Hkv) * Sq = 12 > 8 */
+  EXPECT(attn_decode_multi(fake, fake, fake, (const int32_t*)fake, fake, NULL, 1, 5, 8, 2, 64, 128, 0.1f, NULL) ==
+         ATTN_ERR_UNSUPPORTED); /* (Hq/Hkv) * Sq = 20 > 16 */
   EXPECT(attn_bwd(fake, fake, fake, fake, (const float*)fake, fake, fake, fake, fake, 1, 2, 2, 16, 16, 64, 0.125f,
                   9, NULL, NULL) == ATTN_ERR_MASK);
   EXPECT(attn_key_stats(fake, (float*)fake, (float*)fake, 1, 0, 2, 64, NULL) == ATTN_ERR_SHAPE);

@@ -110,7 +110,7 @@ def _decode_cases(n, seed, base):
     for i in range(n):
         d = int(rng.choice([64, 128]))
         G = int(rng.choice([1, 2, 4, 8]))
-        Sq = int(rng.choice([s for s in (1, 2, 4, 8) if G * s <= 8]))
+        Sq = int(rng.choice([s for s in (1, 2, 3, 4, 8, 16) if G * s <= 16]))
         Hkv = int(rng.integers(1, 4))
         B = int(rng.integers(1, 7))
         Lmax = int(rng.integers(1, 3000))

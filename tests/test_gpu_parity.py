@@ -348,6 +348,11 @@ DECODE_MULTI = [
     (4, 4, 4, 2, 700, 64, [700, 3, 512, 2]),
     (2, 8, 2, 2, 600, 64, [600, 5]),
     (3, 2, 2, 1, 64, 128, [64, 0, 33]),
+    # two groups of 8 MMA columns: (Hq/Hkv) * Sq in 9..16
+    (3, 2, 16, 2, 1100, 128, [1100, 513, 1]),   # G = 8, MTP-2
+    (2, 4, 8, 2, 700, 64, [700, 3]),            # G = 4, four tokens
+    (2, 16, 2, 2, 600, 128, [600, 7]),          # G = 1, sixteen tokens, a sequence shorter than Sq
+    (2, 3, 8, 2, 333, 64, [333, 2]),            # G = 4, three tokens: 12 live columns of 16
 ]
 
 
@@ -405,8 +410,13 @@ def test_decode_multi_equals_single_at_sq1():
     assert torch.equal(o1, o2.reshape(B, Hq, d)) and torch.equal(l1, l2.reshape(B, Hq))
 
 
-def test_decode_multi_full_size_mtp2():
-    B, Sq, Hq, Hkv, Lmax, d = 64, 2, 32, 8, 8192, 128
+@pytest.mark.parametrize("Sq,Hq", [(2, 32), (2, 64)], ids=["G4-mtp2", "G8-mtp2"])
+def test_decode_multi_full_size_mtp2(Sq, Hq):
+    """The decode workload (64 sequences, lengths U[1024, 8192], 8 KV heads,
+    d = 128) with two new tokens per sequence, every element against the
+    oracle's causal prefill; with 64 query heads (G = 8) the 16 (head, token)
+    pairs of a KV group fill two groups of MMA columns."""
+    B, Hkv, Lmax, d = 64, 8, 8192, 128
     lens = synthetic.seqlens(2005, B)
     q = synthetic.tensor(1005, synthetic.TID_Q, (B, Sq, Hq, d))
     kc = synthetic.kv_cache(1005, synthetic.TID_K, B, Lmax, Hkv, d, lens, fill_bits=0x7FC0)
@@ -414,7 +424,7 @@ def test_decode_multi_full_size_mtp2():
     o, lse = eio.attn_decode_multi(dev_bf16(q), dev_bf16(kc), dev_bf16(vc), torch.from_numpy(lens).cuda())
     eio.sync_status()
     ro, rl = oracle_decode_multi(q, kc, vc, lens, 1 / math.sqrt(d))
-    check(o, lse, ro, rl, "mtp2 full size")
+    check(o, lse, ro, rl, f"attn_decode_multi Sq={Sq} Hq={Hq} full size", log=True)
 
 
 def test_decode_more_sequences_than_one_launch_holds():
