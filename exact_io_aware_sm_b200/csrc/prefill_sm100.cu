@@ -65,7 +65,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kBoundLimit2 = 100.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D>
+template <int D, bool BOUND = false>
 struct Cfg {
   // Of every 8 column pairs of a tile, this many take the polynomial exp2
   // on the FMA pipe instead of the MUFU unit.  At d = 64, where the MUFU is
@@ -76,6 +76,15 @@ struct Cfg {
   // d = 64 leaves 128 TMEM columns free: P gets its own columns, so the next
   // S of a slot can be computed while the softmax of the current tile runs.
   static constexpr bool kSepP = D == 64;
+  // Half-tile pipeline (d = 128, bound-based softmax): d = 128 has no free
+  // TMEM columns for a separate P, so S is computed in halves of 64 keys into
+  // two alternating 64-column buffers per slot, and the S of the next
+  // half-tile runs on the tensor core while the softmax works on the current
+  // one (P overwrites its own S half).  It pays where the softmax is short
+  // (no row max: +16 % on the long-context workload); with the running max
+  // the fixed per-step costs of twice as many steps cancel the overlap, so
+  // that softmax keeps whole 128-key tiles.
+  static constexpr bool kHalf = D == 128 && BOUND;
   static constexpr int kRing = (D == 64) ? 8 : 4;         // K/V tiles in flight
   static constexpr int kChunkBytes = 128 * 128;           // 128 rows x 64 bf16 (one swizzle span)
   static constexpr int kTileBytes = 128 * D * 2;          // Q, K or V tile (128 rows)
@@ -87,8 +96,8 @@ struct Cfg {
   static constexpr int kOffStage = kOffRing + kRing * kTileBytes;
   static constexpr int kOffBar = kOffStage + (kStageO ? 2 * 128 * D * 2 : 0);
   // q_full[2*QB] q_empty[2*QB] ring_full[R] ring_empty[R] s_full[2] p_full[2]
-  // pv_done[2] o_free[2] mma_idle
-  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 2 + 2 + 1;  // + mma_idle[2], s_free[2], b_first
+  // pv_done[2] o_free[2] mma_idle[2] s_free[2] b_first o_ready[2] p_fullb[2]
+  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 2 + 2 + 1 + 2 + 2;
   static constexpr int kSmem = kOffBar + 8 * kNumBars + 16 + 1024;  // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -206,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmO,
                         const __grid_constant__ CUtensorMap tmK16,
                         const __grid_constant__ CUtensorMap tmV16, const PrefillArgs a) {
-  using C = Cfg<D>;
+  using C = Cfg<D, BOUND>;
   constexpr int R = C::kRing;
   constexpr int NCH = D / 64;  // 64-element swizzle chunks per row
 
@@ -226,6 +235,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_idle = o_free + 2;    // [2]
   uint64_t* s_free = mma_idle + 2;    // [2] (separate-P layout): S loaded by the softmax
   uint64_t* b_first = s_free + 2;     // slot B finished the exponentials of an item's first tile
+  // Half-tile layout (d = 128): s_full[x] and s_free[x] signal S in buffer 0
+  // and 1 of slot x, p_full[x] and p_fullb[x] the P of buffer 0 and 1 (one
+  // barrier per buffer: the softmax can finish the step after the next
+  // before the issuer waits, and a parity wait must never be two phases
+  // behind), and o_ready[x] the last PV of an item.
+  uint64_t* o_ready = b_first + 1;    // [2]
+  uint64_t* p_fullb = o_ready + 2;    // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -242,7 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[x], 4);
       mbar_init(&pv_done[x], 1);
       mbar_init(&o_free[x], 4);
-      mbar_init(&s_free[x], 4);
+      mbar_init(&s_free[x], C::kHalf ? 1 : 4);
+      mbar_init(&o_ready[x], 1);
+      mbar_init(&p_fullb[x], 4);
     }
     for (int i = 0; i < R; ++i) {
       mbar_init(&ring_full[i], 1);
@@ -423,6 +441,96 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = it_next;  // decoded one item ahead
       w = item_index(++wk, n_items);
       if (w >= 0) it_next = decode_item(a, w);
+      if constexpr (C::kHalf) {
+        // Half-tile steps: each KV tile of up to 128 keys is one or two steps
+        // of up to 64 keys (h = 0, 1).  Step s writes S into buffer s & 1 of
+        // this slot; the issue order S(0), S(1), then per step PV(s), S(s + 2)
+        // lets S(s + 2) overwrite the buffer of P(s) only after PV(s) has read
+        // it (one thread's MMAs execute in order).
+        const int nX = x == 0 ? it.nA : it.nB;
+        const int nB = it.nB;
+        const int4* kv = a.kvtiles + it.kv_first;
+        uint32_t qbuf = 0;
+        if (nX > 0) {
+          qbuf = qcnt % QB;
+          if (!wait_bar(&q_full[x * QB + qbuf], (qcnt / QB) & 1)) break;
+          qcnt++;
+          const uint32_t qbase = sQ + (x * QB + qbuf) * C::kTileBytes;
+          int sj = 0, sh = 0, snc = kv[0].y;  // next S step: tile, half, tile width
+          int pj = 0, ph = 0, pnc = snc;      // next PV step
+          auto issue_sh = [&]() {
+            const uint32_t kpos = seq + 2 * sj;
+            if (sh == 0 && !wait_bar(&ring_full[kpos % R], (kpos / R) & 1)) return;
+            tc_fence_after();
+            const uint32_t ncols = static_cast<uint32_t>(min(64, snc - 64 * sh));
+            const uint32_t b = scnt & 1;
+            const uint32_t id = idesc_bf16_f32(128, ncols, 0, 0);
+            const uint32_t kbase = sRing + (kpos % R) * C::kTileBytes + sh * 64 * 128;  // rows 64h.. of K
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t koff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+              mma_bf16_ss_elect(s_col + b * 64, sdesc_sw128(qbase + koff, 16, 1024),
+                                sdesc_sw128(kbase + koff, 16, 1024), id, kk > 0 ? 1u : 0u);
+            }
+            mma_commit_elect(b == 0 ? &s_full[x] : &s_free[x]);
+            const bool last = sh == 1 || snc <= 64;
+            if (last) mma_commit_elect(&ring_empty[kpos % R]);  // K tile read by both halves
+            scnt++;
+            if (last) {
+              ++sj;
+              sh = 0;
+              snc = sj < nX ? kv[sj].y : 0;
+            } else {
+              sh = 1;
+            }
+          };
+          auto issue_pvh = [&]() {
+            const uint32_t vpos = seq + 2 * pj + 1;
+            if (!wait_bar((pcnt & 1) == 0 ? &p_full[x] : &p_fullb[x], (pcnt >> 1) & 1)) return;
+            if (pj == 0 && ph == 0 && ocnt > 0 && !wait_bar(&o_free[x], (ocnt - 1) & 1)) return;
+            if (ph == 0 && !wait_bar(&ring_full[vpos % R], (vpos / R) & 1)) return;
+            tc_fence_after();
+            const int nk = min(64, pnc - 64 * ph);
+            const uint32_t b = pcnt & 1;
+            const uint32_t vbase = sRing + (vpos % R) * C::kTileBytes;
+            for (int i = 0; i < (nk >> 4); ++i)
+              mma_bf16_ts_elect(o_col, s_col + b * 64 + i * 8,
+                                sdesc_sw128(vbase + (4 * ph + i) * 2048, C::kChunkBytes, 1024), idO,
+                                (pj > 0 || ph > 0 || i > 0) ? 1u : 0u);
+            mma_commit_elect(&pv_done[x]);
+            const bool last = ph == 1 || pnc <= 64;
+            if (last) mma_commit_elect(&ring_empty[vpos % R]);
+            pcnt++;
+            if (last) {
+              ++pj;
+              ph = 0;
+              pnc = pj < nX ? kv[pj].y : 0;
+            } else {
+              ph = 1;
+            }
+          };
+          issue_sh();
+          if (ok && sj < nX) issue_sh();
+          while (ok && pj < nX) {
+            issue_pvh();
+            if (ok && sj < nX) issue_sh();
+          }
+          if (ok) mma_commit_elect(&o_ready[x]);  // the item's last PV
+          ocnt++;
+        }
+        // Stages of tiles this slot does not visit: release once filled.
+        for (int j = nX; ok && j < nB; ++j) {
+          const uint32_t kseq = seq + 2 * j, vseq = kseq + 1;
+          if (!wait_bar(&ring_full[kseq % R], (kseq / R) & 1)) break;
+          mbar_arrive_elect(&ring_empty[kseq % R]);
+          if (!wait_bar(&ring_full[vseq % R], (vseq / R) & 1)) break;
+          mbar_arrive_elect(&ring_empty[vseq % R]);
+        }
+        seq += 2 * nB;
+        if (!ok) break;
+        if (nX > 0) mma_commit_elect(&q_empty[x * QB + qbuf]);
+        continue;
+      }
       const int nX = x == 0 ? it.nA : it.nB;
       const int nB = it.nB;
       const int4* kv = a.kvtiles + it.kv_first;
@@ -483,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_tmem = tmem + lane_off + static_cast<uint32_t>(256 + x * D);
     const uint32_t p_tmem = C::kSepP ? tmem + lane_off + static_cast<uint32_t>(256 + 2 * D + x * 64) : s_tmem;
     const float sl2 = a.scale_log2;
-    uint32_t tcnt = 0, bcnt = 0;
+    uint32_t tcnt = 0, bcnt = 0, icnt = 0;
     bool ok = true;
     // Waits and the abort decision are made warp-uniform, because the warp
     // then executes .sync.aligned tcgen05 instructions together.
@@ -533,6 +641,96 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;
       int4 kt_next = nX > 0 ? kv[0] : make_int4(0, 0, 0, 0);
 
+      if constexpr (C::kHalf) {
+      // Half-tile steps (see the MMA issuer): step t of this slot reads S from
+      // buffer t & 1 (64 columns), writes its P over the first 32 of them.
+      const uint32_t tcnt0 = tcnt;
+      for (int j = 0; j < nX && ok; ++j) {
+        const int4 kt = kt_next;
+        if (j + 1 < nX) kt_next = kv[j + 1];
+        const int nh = kt.y > 64 ? 2 : 1;
+        for (int h = 0; h < nh; ++h) {
+          const uint32_t b = tcnt & 1;
+          if (!warp_wait(b == 0 ? &s_full[x] : &s_free[x], (tcnt >> 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // Columns at or past `lim` are masked: past the half's width always,
+          // and on partial tiles past Nkv and past the causal diagonal.
+          int lim = min(64, kt.y - 64 * h);
+          if ((kt.z >> x) & 1) {
+            lim = min(lim, a.Nkv - kt.x - 64 * h);
+            if (a.causal) lim = min(lim, grow + a.causal_off + 1 - kt.x - 64 * h);
+          }
+          uint32_t sr[64];
+          tmem_ld32(s_tmem + b * 64, sr);
+          tmem_ld32(s_tmem + b * 64 + 32, sr + 32);
+          tmem_wait_ld();
+          if (__any_sync(0xffffffffu, lim < 64)) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
+          }
+          float mx_s = -INFINITY;
+          if (!BOUND || !skip_max) {
+            float mx4[4];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              float m = __uint_as_float(sr[q4 * 16]);
+#pragma unroll
+              for (int c = 1; c < 15; c += 2)
+                m = max3f(m, __uint_as_float(sr[q4 * 16 + c]), __uint_as_float(sr[q4 * 16 + c + 1]));
+              mx4[q4] = fmaxf(m, __uint_as_float(sr[q4 * 16 + 15]));
+            }
+            mx_s = max3f(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * sl2;
+          }
+          const bool upd = (!BOUND || !fixed) && mx_s > m_b + kRescaleThreshold;
+          const float alpha = upd ? ex2(m_b - mx_s) : 1.f;  // 0 when m_b was -inf
+          if (upd) m_b = mx_s;
+          const float base = m_b == -INFINITY ? 0.f : m_b;
+          float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+          const float2 sl = make_float2(sl2, sl2), nb = make_float2(-base, -base);
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float2 e = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl, nb);
+            const float2 p = make_float2(ex2(e.x), ex2(e.y));
+            acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], p);
+            sr[c >> 1] = pack_bf16x2(p.x, p.y);
+          }
+          if (stagger && x == 1 && tcnt == tcnt0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_first);
+          }
+          if (tcnt > tcnt0 && __any_sync(0xffffffffu, upd)) {
+            // O holds the earlier steps: the previous step's PV must have
+            // completed before O is rescaled.
+            if (!warp_wait(&pv_done[x], (tcnt - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              uint32_t orr[32];
+              tmem_ld32(o_tmem + c, orr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+              tmem_st32(o_tmem + c, orr);
+            }
+          }
+          const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+          l = l * alpha + (s01.x + s01.y);
+          tmem_st32(s_tmem + b * 64, sr);  // P: 64 keys as 32 columns of bf16 pairs
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b == 0 ? &p_full[x] : &p_fullb[x]);
+          tcnt++;
+        }
+      }
+      } else {
       for (int t = 0; t < nX; ++t) {
         const int4 kt = kt_next;
         if (t + 1 < nX) kt_next = kv[t + 1];
@@ -626,15 +824,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&p_full[x]);
         tcnt++;
       }
+      }
       if (!ok) break;
 
       // ---------------------------------------------------------- epilogue
       if (nX > 0) {
-        if (!warp_wait(&pv_done[x], (tcnt - 1) & 1)) {
+        // the item's last PV has completed
+        if (!warp_wait(C::kHalf ? &o_ready[x] : &pv_done[x], C::kHalf ? (icnt & 1) : ((tcnt - 1) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        icnt++;
       }
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
       const bool valid = row < nrows;
@@ -738,14 +939,14 @@ cudaError_t launch_ds(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kLaunchRegs || fa.maxThreadsPerBlock < kThreads) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(prefill_bf16_kernel<D, STAGGER, BOUND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg<D>::kSmem);
+                             Cfg<D, BOUND>::kSmem);
     if (e != cudaSuccess) return e;
     attr_set.set(dev);
   }
   if (a.n_items == 0) return cudaSuccess;
   const long long grid = a.n_items < a.num_ctas ? a.n_items : a.num_ctas;
   prefill_bf16_kernel<D, STAGGER, BOUND>
-      <<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmem, s>>>(tq, tk, tv, to, tk16, tv16, a);
+      <<<static_cast<unsigned>(grid), kThreads, Cfg<D, BOUND>::kSmem, s>>>(tq, tk, tv, to, tk16, tv16, a);
   return cudaGetLastError();
 }
 
