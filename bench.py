@@ -597,7 +597,8 @@ def bench_bound(w, args, world, rank, peaks):
            "config": {"workload": w["desc"] + ", attn_fwd_bound (key statistics precomputed)"},
            "roofline": {"bound": "tensor", "achieved": flops / (ms_fwd * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
                         "frac": flops / (ms_fwd * 1e-3) / 1e12 / peak, "peak_source": f"{peaks['source']} bf16 burst",
-                        "kernel": "prefill_bf16_kernel (bound mode)"},
+                        "kernel": "prefill_bf16_kernel (bound mode)",
+                        "traffic": recorded_traffic(f"prefill_bound_{args_key(w)}")},
            "gpu_launches": 3 * steps}
     del tq, tk, tv, o, lse
     torch.cuda.empty_cache()
