@@ -203,6 +203,11 @@ __device__ __forceinline__ long long item_index(long long k, long long n_items) 
 }
 
 constexpr bool kFirstLoadsFirst = true;
+// Q tiles and O rows are each touched once: load and store them as
+// evict_first in L2, so that they do not push out K/V tiles that the items
+// of later rounds read again.
+constexpr bool kStreamHintQ = true;
+constexpr bool kStreamHintO = true;
 
 // STAGGER: both slots of every pair visit the same number of KV tiles, and
 // slot A starts each item after slot B's first exponentials (see below).
@@ -326,9 +331,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx_elect(&q_full[x * QB + qb], C::kTileBytes);
 #pragma unroll
-        for (int ch = 0; ch < NCH; ++ch)
-          tma_load_4d_elect(smem + C::kOffQ + (x * QB + qb) * C::kTileBytes + ch * C::kChunkBytes, &tmQ,
-                            &q_full[x * QB + qb], ch * 64, headX[x], rowX[x], it.b);
+        for (int ch = 0; ch < NCH; ++ch) {
+          uint8_t* qdst = smem + C::kOffQ + (x * QB + qb) * C::kTileBytes + ch * C::kChunkBytes;
+          if constexpr (kStreamHintQ)
+            tma_load_4d_elect_hint(qdst, &tmQ, &q_full[x * QB + qb], ch * 64, headX[x], rowX[x], it.b,
+                                   l2_policy_evict_first());
+          else
+            tma_load_4d_elect(qdst, &tmQ, &q_full[x * QB + qb], ch * 64, headX[x], rowX[x], it.b);
+        }
         qcnt[x]++;
       }
       int4 kt_next = it.nB > 0 ? a.kvtiles[it.kv_first] : make_int4(0, 0, 0, 0);
@@ -874,9 +884,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            if (quarter * 32 + 16 * h < nrows)
-              tma_store_4d(&tmO, stg + (quarter * 32 + 16 * h) * (D * 2), 0, head, row0 + quarter * 32 + 16 * h,
-                           it.b);
+            if (quarter * 32 + 16 * h < nrows) {
+              if constexpr (kStreamHintO)
+                tma_store_4d_hint(&tmO, stg + (quarter * 32 + 16 * h) * (D * 2), 0, head,
+                                  row0 + quarter * 32 + 16 * h, it.b, l2_policy_evict_first());
+              else
+                tma_store_4d(&tmO, stg + (quarter * 32 + 16 * h) * (D * 2), 0, head, row0 + quarter * 32 + 16 * h,
+                             it.b);
+            }
           bulk_commit();
         }
       } else {
@@ -894,12 +909,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (valid) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            *reinterpret_cast<uint4*>(orow + 2 * (c + u * 8)) = make_uint4(
+          for (int u = 0; u < 4; ++u) {
+            const uint4 v = make_uint4(
                 pack_bf16x2(__uint_as_float(orr[u * 8 + 0]) * inv_l, __uint_as_float(orr[u * 8 + 1]) * inv_l),
                 pack_bf16x2(__uint_as_float(orr[u * 8 + 2]) * inv_l, __uint_as_float(orr[u * 8 + 3]) * inv_l),
                 pack_bf16x2(__uint_as_float(orr[u * 8 + 4]) * inv_l, __uint_as_float(orr[u * 8 + 5]) * inv_l),
                 pack_bf16x2(__uint_as_float(orr[u * 8 + 6]) * inv_l, __uint_as_float(orr[u * 8 + 7]) * inv_l));
+            if constexpr (kStreamHintO)
+              st_global_v4_hint(orow + 2 * (c + u * 8), v, l2_policy_evict_first());
+            else
+              *reinterpret_cast<uint4*>(orow + 2 * (c + u * 8)) = v;
+          }
         }
       }
       }

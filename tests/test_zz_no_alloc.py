@@ -5,9 +5,10 @@ device memory through its own pool, a serving process with a memory budget
 fixed at start-up, or code that cannot take the device synchronisation an
 allocation may cause).  attn_decode_noalloc keeps its scratch in a fixed
 device array inside the library instead.  These tests call it through the C
-ABI and compare it with attn_decode, on two calls in a row (the second with
-new inputs, so stale contents of the shared array would show), and check that
-an oversized shape is refused before any GPU work.
+ABI and compare it with attn_decode and with the fp64 oracle, on two calls in
+a row (the second with new inputs, so stale contents of the shared array would
+show), check that its own error word reports a device-side error, and that an
+oversized shape is refused before any GPU work.
 
 This file is named so that pytest collects it last.
 """
@@ -19,6 +20,7 @@ import pytest
 import torch
 
 import exact_io_aware_sm_b200 as eio
+import oracle
 import synthetic
 
 pytestmark = pytest.mark.gpu
@@ -46,11 +48,16 @@ def _status(L):
     return L.attn_decode_noalloc_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-def _inputs(seed, B, Hq, Hkv, Lmax, d):
+def _host_inputs(seed, B, Hq, Hkv, Lmax, d):
     lens = synthetic.seqlens(seed, B, 1, Lmax)
     q = synthetic.tensor(seed, synthetic.TID_Q, (B, Hq, d))
     kc = synthetic.kv_cache(seed, synthetic.TID_K, B, Lmax, Hkv, d, lens)
     vc = synthetic.kv_cache(seed, synthetic.TID_V, B, Lmax, Hkv, d, lens)
+    return q, kc, vc, lens
+
+
+def _inputs(seed, B, Hq, Hkv, Lmax, d):
+    q, kc, vc, lens = _host_inputs(seed, B, Hq, Hkv, Lmax, d)
 
     def dev(x):
         return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
@@ -82,6 +89,12 @@ def test_noalloc_matches_attn_decode_on_two_calls(lib, shape):
         assert err.max().item() <= O_MAX and err.mean().item() <= O_MEAN
         assert (lse - ref_l).abs().max().item() <= LSE_TOL
         assert _status(lib) == 0, eio.last_error()  # its own error word: nothing latched
+        # and against the fp64 oracle directly, every element
+        hq, hkc, hvc, hlens = _host_inputs(seed + d, B, Hq, Hkv, Lmax, d)
+        ro, rl = oracle.decode(hq, hkc, hvc, hlens, 1.0 / math.sqrt(d))
+        oerr = np.abs(o.float().cpu().numpy().astype(np.float64) - ro)
+        assert oerr.max() <= O_MAX and oerr.mean() <= O_MEAN
+        assert np.abs(lse.cpu().numpy().astype(np.float64) - rl).max() <= LSE_TOL
     eio.sync_status()
 
 
