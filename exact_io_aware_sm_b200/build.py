@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libattn_b200.so")
 SOURCES = ["api.cu", "plan.cpp", "prefill_sm100.cu", "prefill_f32.cu", "decode.cu", "decode_noalloc.cu",
            "backward.cu", "key_stats.cu"]
-HEADERS = ["kernels.h", "plan.h", "ptx_sm100.cuh", "warp_mma.cuh", "fastmath.cuh", os.path.join("..", "..", "include", "attn.h")]
+HEADERS = ["kernels.h", "plan.h", "ptx_sm100.cuh", "pdl.cuh", "warp_mma.cuh", "fastmath.cuh", os.path.join("..", "..", "include", "attn.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -66,6 +66,7 @@
 
 #include "fastmath.cuh"
 #include "kernels.h"
+#include "pdl.cuh"
 #include "ptx_sm100.cuh"
 #include "warp_mma.cuh"
 
@@ -403,7 +404,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tma_prefetch_desc(&tmV);
     }
     uint32_t g = 0, nfix = 0;
-    bool ok = true;
+    bool ok = true, vec_ready = false;
     for (long long k = 0; ok; ++k) {
       const long long w = bwd_item(k, n_items);
       if (w < 0) break;
@@ -437,6 +438,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         // the tile's 128 -lse2 and -D values (padded rows: -lse2 = -inf, D = 0)
         const size_t vrow = (static_cast<size_t>(it.b) * a.Hq + hq) * nq_pad + static_cast<size_t>(qt) * kT;
+        // -lse2 and -D are written by the dQ kernel, which may still be
+        // running (programmatic dependent launch): wait for it before the
+        // first copy of them.
+        if (!vec_ready) {
+          pdl_wait();
+          vec_ready = true;
+        }
         bulk_load_elect(vec + s * 2 * kT, a.neg_lse2 + vrow, kT * 4, &br.full[s]);
         bulk_load_elect(vec + s * 2 * kT + kT, a.neg_d + vrow, kT * 4, &br.full[s]);
       }
@@ -704,6 +712,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const int off = a.Nkv - a.Nq;
   const int nq_pad = (a.Nq + kT - 1) / kT * kT;
   const long long n_items = static_cast<long long>((a.Nq + kT - 1) / kT) * a.Hq * a.B;
+  // The dK/dV kernel may be scheduled as this kernel's CTAs finish; it
+  // waits for this grid before it reads -lse2 and -D.
+  if (threadIdx.x == 0) pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     mbar_init(br.fixed_full, 1);
@@ -1060,9 +1071,8 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
                                                                                                  tdq, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dkdv_kernel<D, BLK><<<static_cast<unsigned>(n_kv < n_sm ? n_kv : n_sm), kBThreads, C::kSmemKV, s>>>(tq, tdo, tk, tv,
-                                                                                                     tdk, tdv, a);
-  return cudaGetLastError();
+  return launch_after_pdl(bwd_dkdv_kernel<D, BLK>, dim3(static_cast<unsigned>(n_kv < n_sm ? n_kv : n_sm)),
+                          dim3(kBThreads), C::kSmemKV, s, tq, tdo, tk, tv, tdk, tdv, a);
 }
 
 }  // namespace

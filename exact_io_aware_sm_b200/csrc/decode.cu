@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 
 #include "kernels.h"
+#include "pdl.cuh"
 #include "ptx_sm100.cuh"
 #include "warp_mma.cuh"
 
@@ -100,6 +101,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
+  // The combine kernel may be scheduled as this kernel's CTAs finish; it
+  // waits for this grid before it reads the partials.
+  if (threadIdx.x == 0) pdl_launch_dependents();
   if (warp == 0) {
     int carry = 0;
     if (lane == 0) pre[0] = 0;
@@ -374,8 +378,8 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
   const int b = bh / (a.Sq * a.Hq);
   const int lse_at = (b * a.Hq + bh % a.Hq) * a.Sq + (bh / a.Hq) % a.Sq;  // LSE is [B, Hq, Sq]
   const int t = threadIdx.x;
-  // The split kernels of this call have finished: zero their item counters
-  // for the next call.
+  pdl_wait();  // the split kernels of this call have finished and their partials are visible
+  // Zero their item counters for the next call.
   if (bh == 0 && t < (a.B + kMaxB - 1) / kMaxB) a.counter[t] = 0;
   const int len = checked_len(a, b);
   const int ns = (len + kDecodeChunk - 1) / kDecodeChunk;
@@ -439,8 +443,7 @@ cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  decode_combine_kernel<D><<<a.B * a.Sq * a.Hq, D, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_after_pdl(decode_combine_kernel<D>, dim3(a.B * a.Sq * a.Hq), dim3(D), 0, s, a);
 }
 
 template <int D>
