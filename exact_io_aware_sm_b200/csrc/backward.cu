@@ -101,8 +101,8 @@ struct BCfg {
   static constexpr int kOffStgQ = kOffX + kTile;
   static constexpr int kOffBarQ = kOffStgQ + (kStage ? kTile : 0);
   // fixed_full, fixed_empty, full[R], empty[R], s_full[2], dp_full, p_full, ds_full,
-  // mma_done, acc_free[2], mma_idle, stg_full, stg_free
-  static constexpr int kNumBars = 2 * R + 13;
+  // mma_done, acc_free[2], mma_idle, stg_full, stg_free, p_full1
+  static constexpr int kNumBars = 2 * R + 14;
   static constexpr int kSmemKV = kOffBarKV + 8 * kNumBars + 16 + 1024;
   static constexpr int kSmemQ = kOffBarQ + 8 * kNumBars + 16 + 1024;
   static_assert(kSmemKV <= 227 * 1024 && kSmemQ <= 227 * 1024, "shared memory per CTA");
@@ -112,14 +112,26 @@ struct BCfg {
   static constexpr int kAccQ = D == 64 ? 2 : 1;  // dQ accumulators in TMEM
 };
 
-// Barriers shared by both kernels' layouts (p_full is unused by the dQ kernel).
+// Barriers shared by both kernels' layouts (p_full0/1 are unused by the dQ
+// kernel).  With two S buffers (dK/dV kernel at d = 64) P of step t is
+// signalled on p_full(t), alternating between two barriers: the issuer puts
+// S(t+1) on the tensor core before it waits for P(t), so the element-wise
+// warps may finish P(t) and P(t+1) before that wait, and a parity wait must
+// never fall two phases behind its barrier.  With one S buffer, S(t+1)
+// follows dK(t), which follows the wait for P(t), and p_full0 serves every
+// step.
 struct BBars {
-  uint64_t *fixed_full, *fixed_empty, *full, *empty, *s_full, *dp_full, *p_full, *ds_full, *mma_done, *acc_free,
-      *mma_idle, *stg_full, *stg_free;
+  uint64_t *fixed_full, *fixed_empty, *full, *empty, *s_full, *dp_full, *p_full0, *ds_full, *mma_done, *acc_free,
+      *mma_idle, *stg_full, *stg_free, *p_full1;
   __device__ BBars(uint64_t* b, int R)
       : fixed_full(b), fixed_empty(b + 1), full(b + 2), empty(b + 2 + R), s_full(b + 2 + 2 * R),
-        dp_full(b + 4 + 2 * R), p_full(b + 5 + 2 * R), ds_full(b + 6 + 2 * R), mma_done(b + 7 + 2 * R),
-        acc_free(b + 8 + 2 * R), mma_idle(b + 10 + 2 * R), stg_full(b + 11 + 2 * R), stg_free(b + 12 + 2 * R) {}
+        dp_full(b + 4 + 2 * R), p_full0(b + 5 + 2 * R), ds_full(b + 6 + 2 * R), mma_done(b + 7 + 2 * R),
+        acc_free(b + 8 + 2 * R), mma_idle(b + 10 + 2 * R), stg_full(b + 11 + 2 * R), stg_free(b + 12 + 2 * R),
+        p_full1(b + 13 + 2 * R) {}
+  template <int NB>
+  __device__ uint64_t* p_full(uint32_t t) const { return (NB == 2 && (t & 1)) ? p_full1 : p_full0; }
+  template <int NB>
+  __device__ static uint32_t p_parity(uint32_t t) { return NB == 2 ? (t >> 1) & 1 : t & 1; }
 };
 
 // One element-wise thread's NC TMEM columns (times mul) as bf16 into a
@@ -365,7 +377,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(&br.s_full[0], 1);
     mbar_init(&br.s_full[1], 1);
     mbar_init(br.dp_full, 1);
-    mbar_init(br.p_full, kEW);
+    mbar_init(br.p_full0, kEW);
+    mbar_init(br.p_full1, kEW);
     mbar_init(br.ds_full, kEW);
     mbar_init(br.mma_done, 1);
     mbar_init(&br.acc_free[0], kEW);
@@ -498,7 +511,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
           mma_commit_elect(&br.s_full[(g + 1) % NB]);
         }
         // dV / dK of the previous item have been read out of TMEM
-        if (!wwait(br.p_full, g & 1) || (u == 0 && k > 0 && !wwait(&br.acc_free[0], (k - 1) & 1))) {
+        if (!wwait(br.p_full<NB>(g), BBars::p_parity<NB>(g)) ||
+            (u == 0 && k > 0 && !wwait(&br.acc_free[0], (k - 1) & 1))) {
           ok = false;
           break;
         }
@@ -619,7 +633,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(br.p_full);
+        if (lane == 0) mbar_arrive(br.p_full<NB>(g));
         if (!wwait(br.dp_full, g & 1)) {
           ok = false;
           break;
