@@ -96,8 +96,8 @@ struct Cfg {
   static constexpr int kOffStage = kOffRing + kRing * kTileBytes;
   static constexpr int kOffBar = kOffStage + (kStageO ? 2 * 128 * D * 2 : 0);
   // q_full[2*QB] q_empty[2*QB] ring_full[R] ring_empty[R] s_full[2] p_full[2]
-  // pv_done[2] o_free[2] mma_idle[2] s_free[2] b_first o_ready[2] p_fullb[2]
-  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 2 + 2 + 1 + 2 + 2;
+  // pv_done[2] o_free[2] mma_idle[2] s_free[2] b_first[kQBuf] o_ready[2] p_fullb[2]
+  static constexpr int kNumBars = 4 * kQBuf + 2 * kRing + 8 + 2 + 2 + kQBuf + 2 + 2;
   static constexpr int kSmem = kOffBar + 8 * kNumBars + 16 + 1024;  // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
@@ -239,13 +239,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_free = pv_done + 2;     // [2]
   uint64_t* mma_idle = o_free + 2;    // [2]
   uint64_t* s_free = mma_idle + 2;    // [2] (separate-P layout): S loaded by the softmax
-  uint64_t* b_first = s_free + 2;     // slot B finished the exponentials of an item's first tile
+  // b_first[i]: slot B has finished the exponentials of the first tile of an
+  // offset item, item n on b_first[n % QB].  Slot B can start an item only
+  // once the in-order producer has loaded slot A's Q for it, which needs slot
+  // A's Q buffer of QB offset items earlier, freed only after slot A's wait
+  // for that item; so slot B is at most QB - 1 items ahead of that wait, and
+  // with QB barriers in turn no parity wait falls two phases behind.
+  uint64_t* b_first = s_free + 2;     // [QB]
   // Half-tile layout (d = 128): s_full[x] and s_free[x] signal S in buffer 0
   // and 1 of slot x, p_full[x] and p_fullb[x] the P of buffer 0 and 1 (one
   // barrier per buffer: the softmax can finish the step after the next
   // before the issuer waits, and a parity wait must never be two phases
   // behind), and o_ready[x] the last PV of an item.
-  uint64_t* o_ready = b_first + 1;    // [2]
+  uint64_t* o_ready = b_first + QB;   // [2]
   uint64_t* p_fullb = o_ready + 2;    // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -271,9 +277,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ring_full[i], 1);
       mbar_init(&ring_empty[i], 2);  // released by both slot issuers
     }
-    mbar_init(b_first, 4);
     mbar_init(&mma_idle[0], 1);
     mbar_init(&mma_idle[1], 1);
+    for (int i = 0; i < QB; ++i) mbar_init(&b_first[i], 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -641,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool skip_max = BOUND && __all_sync(0xffffffffu, fixed);
       const bool stagger = STAGGER && it.nA > 0;
       if (stagger && x == 0) {
-        if (!warp_wait(b_first, bcnt & 1)) {
+        if (!warp_wait(&b_first[bcnt % QB], (bcnt / QB) & 1)) {
           ok = false;
           break;
         }
@@ -710,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (stagger && x == 1 && tcnt == tcnt0) {
             __syncwarp();
-            if (lane == 0) mbar_arrive(b_first);
+            if (lane == 0) mbar_arrive(&b_first[(bcnt - 1) % QB]);  // bcnt counts this item already
           }
           if (tcnt > tcnt0 && __any_sync(0xffffffffu, upd)) {
             // O holds the earlier steps: the previous step's PV must have
@@ -801,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (stagger && x == 1 && t == 0) {
           __syncwarp();
-          if (lane == 0) mbar_arrive(b_first);
+          if (lane == 0) mbar_arrive(&b_first[(bcnt - 1) % QB]);  // bcnt counts this item already
         }
         if (C::kSepP && t > 0) {
           // P_X and O_X are free once PV_{t-1} has completed.

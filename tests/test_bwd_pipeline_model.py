@@ -18,61 +18,7 @@ import random
 
 import pytest
 
-
-class Bar:
-    def __init__(self, count):
-        self.count, self.pending, self.phase = count, count, 0
-
-    def arrive(self):
-        self.pending -= 1
-        assert self.pending >= 0
-        if self.pending == 0:
-            self.phase += 1
-            self.pending = self.count
-
-
-def run(roles, bars, queue, rng, max_rounds=400000):
-    waiting = {k: None for k in roles}
-    finished = set()
-    for _ in range(max_rounds):
-        if len(finished) == len(roles):
-            return "ok"
-        progressed = False
-        order = list(roles)
-        rng.shuffle(order)
-        for k in order:
-            if k in finished:
-                continue
-            for _ in range(rng.randint(1, 3)):
-                w = waiting[k]
-                if w is not None:
-                    name, index = w
-                    if bars[name].phase > index + 1:
-                        return f"parity ambiguous: {k} waits for phase {index} of {name}, at {bars[name].phase}"
-                    if bars[name].phase <= index:
-                        break
-                    waiting[k] = None
-                try:
-                    waiting[k] = next(roles[k])
-                except StopIteration:
-                    finished.add(k)
-                    progressed = True
-                    break
-                progressed = True
-        for _ in range(rng.randint(0, 3)):
-            if queue:
-                entry = queue.pop(0)
-                if entry != "op":
-                    bars[entry].arrive()
-                progressed = True
-        if not progressed:
-            if queue:
-                entry = queue.pop(0)
-                if entry != "op":
-                    bars[entry].arrive()
-                continue
-            return "deadlock: " + ", ".join(f"{k} waits {waiting[k]}" for k in roles if k not in finished)
-    return "did not finish"
+from protocol_model import Bar, run
 
 
 def dkdv_model(steps, R, NB, n_ew, rng, p_alternate=None):
