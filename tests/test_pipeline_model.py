@@ -15,7 +15,8 @@ The kernel's roles and barriers, as the model has them (one CTA):
   softmax x  per step: wait for S(s), write P(s), arrive on p_full[x][s & 1];
              per item: the epilogue waits for o_ready and frees O; slot A
              starts each item after slot B's first step (the stagger).
-A tensor-core operation completes in issue order at a random later time.
+A tensor-core operation completes in issue order at a random later time, and
+any role can be held back for a while (the shared engine in protocol_model.py).
 
 An mbarrier wait names only the parity of the phase it waits for, so a waiter
 must never fall two phases behind its barrier (it would then wait for a phase
@@ -28,26 +29,14 @@ import random
 
 import pytest
 
-
-class Bar:
-    def __init__(self, name, count):
-        self.name, self.count, self.pending, self.phase = name, count, count, 0
-
-    def arrive(self):
-        self.pending -= 1
-        if self.pending == 0:
-            self.phase += 1
-            self.pending = self.count
-
-    def complete(self, index):
-        return self.phase > index
+from protocol_model import Bar, run
 
 
-def simulate(items, rng, R=4, stagger=True, p_per_buffer=True, max_rounds=200000):
+def simulate(items, rng, R=4, stagger=True, p_per_buffer=True, max_rounds=400000):
     bars = {}
 
     def bar(name, count):
-        bars[name] = Bar(name, count)
+        bars[name] = Bar(count)
 
     for x in (0, 1):
         for n, c in (("q_full", 1), ("q_empty", 1), ("s_full0", 1), ("s_full1", 1), ("p_full0", 4),
@@ -57,7 +46,11 @@ def simulate(items, rng, R=4, stagger=True, p_per_buffer=True, max_rounds=200000
         bar(f"ring_full{i}", 1)
         bar(f"ring_empty{i}", 2)
     bar("b_first", 4)
-    tensor_queue = []  # commit lists of issued tensor-core operations, in issue order
+    tensor_queue = []  # issued tensor-core operations ("op") and their commits, in issue order
+
+    def op(*commits):
+        tensor_queue.append("op")
+        tensor_queue.extend(commits)
 
     def p_bar(x, step):
         return f"p_full{step & 1}{x}" if p_per_buffer else f"p_full0{x}"
@@ -98,8 +91,7 @@ def simulate(items, rng, R=4, stagger=True, p_per_buffer=True, max_rounds=200000
                     kpos = seq + 2 * j
                     if h == 0:
                         yield (f"ring_full{kpos % R}", kpos // R)
-                    commits = [f"s_full{scnt & 1}{x}"] + ([f"ring_empty{kpos % R}"] if last_half[(j, h)] else [])
-                    tensor_queue.append(commits)
+                    op(f"s_full{scnt & 1}{x}", *([f"ring_empty{kpos % R}"] if last_half[(j, h)] else []))
                     scnt += 1
                     s_next += 1
 
@@ -113,11 +105,11 @@ def simulate(items, rng, R=4, stagger=True, p_per_buffer=True, max_rounds=200000
                     vpos = seq + 2 * j + 1
                     if h == 0:
                         yield (f"ring_full{vpos % R}", vpos // R)
-                    tensor_queue.append([f"pv_done{x}"] + ([f"ring_empty{vpos % R}"] if last_half[(j, h)] else []))
+                    op(f"pv_done{x}", *([f"ring_empty{vpos % R}"] if last_half[(j, h)] else []))
                     pcnt += 1
                     if s_next < len(steps):
                         yield from issue_s()
-                tensor_queue.append([f"o_ready{x}"])
+                tensor_queue.append(f"o_ready{x}")
                 ocnt += 1
             for j in range(nX, nB):  # stages of tiles past slot A's prefix
                 for t in (0, 1):
@@ -126,7 +118,7 @@ def simulate(items, rng, R=4, stagger=True, p_per_buffer=True, max_rounds=200000
                     bars[f"ring_empty{pos % R}"].arrive()
             seq += 2 * nB
             if nX > 0:
-                tensor_queue.append([f"q_empty{x}"])
+                tensor_queue.append(f"q_empty{x}")
 
     def softmax(x):
         tcnt = bcnt = icnt = 0
@@ -156,45 +148,7 @@ def simulate(items, rng, R=4, stagger=True, p_per_buffer=True, max_rounds=200000
     for x in (0, 1):
         for q in range(4):
             roles[f"softmax{x}{q}"] = softmax(x)
-    waiting = {k: None for k in roles}
-    finished = set()
-    for _ in range(max_rounds):
-        if len(finished) == len(roles):
-            return "ok"
-        progressed = False
-        order = list(roles)
-        rng.shuffle(order)
-        for k in order:
-            if k in finished:
-                continue
-            for _ in range(rng.randint(1, 3)):
-                w = waiting[k]
-                if w is not None:
-                    name, index = w
-                    if bars[name].phase > index + 1:
-                        return f"parity ambiguous: {k} waits for phase {index} of {name}, which is at {bars[name].phase}"
-                    if not bars[name].complete(index):
-                        break
-                    waiting[k] = None
-                try:
-                    waiting[k] = next(roles[k])
-                except StopIteration:
-                    finished.add(k)
-                    progressed = True
-                    break
-                progressed = True
-        for _ in range(rng.randint(0, 2)):
-            if tensor_queue:
-                for c in tensor_queue.pop(0):
-                    bars[c].arrive()
-                progressed = True
-        if not progressed:
-            if tensor_queue:
-                for c in tensor_queue.pop(0):
-                    bars[c].arrive()
-                continue
-            return "deadlock: " + ", ".join(f"{k} waits {waiting[k]}" for k in roles if k not in finished)
-    return "did not finish"
+    return run(roles, bars, tensor_queue, rng, max_rounds)
 
 
 def random_items(rng):
