@@ -7,20 +7,26 @@
 // Three launches over 128-key chunks, each thread moving 16 bytes (eight
 // keys' columns) per load with several loads in flight:
 //   key_sum_kernel     per-chunk column sums into scratch;
-//   key_mean_kernel    kbar = (sum of the chunk sums, in chunk order) / Nkv,
-//                      so the result does not depend on scheduling;
+//   key_mean_kernel    kbar = (sum of the chunk sums) / Nkv, eight runs of
+//                      consecutive chunks summed in parallel and then added in
+//                      run order, so the result does not depend on scheduling;
 //   key_radius_kernel  the largest centred norm of each chunk, folded into
 //                      `radius` with an integer atomicMax on the float's bits
 //                      (non-negative floats order like their bit patterns).
+// The second and third are programmatic dependents of the one before them:
+// they start while it drains, and the radius kernel loads its keys (an input
+// of the call) before it waits for the mean.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
+#include "pdl.cuh"
 
 namespace eio {
 namespace {
 
 constexpr int kChunkKeys = 128;
 constexpr int kStatThreads = 256;
+constexpr int kMeanRuns = 8;  // runs of chunks summed in parallel per column
 
 __device__ __forceinline__ void add8(float* acc, const uint4& u) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -40,6 +46,7 @@ __global__ void __launch_bounds__(kStatThreads) key_sum_kernel(const KeyStatsArg
   const int c8 = threadIdx.x % TPR, r = threadIdx.x / TPR;
   const int j0 = split * kChunkKeys, j1 = min(a.Nkv, j0 + kChunkKeys);
   const uint4* k = reinterpret_cast<const uint4*>(a.k);
+  if (threadIdx.x == 0) pdl_launch_dependents();
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int p = 0; p < kChunkKeys / RPI; ++p) {
@@ -59,13 +66,26 @@ __global__ void __launch_bounds__(kStatThreads) key_sum_kernel(const KeyStatsArg
 }
 
 template <int D>
-__global__ void __launch_bounds__(D) key_mean_kernel(const KeyStatsArgs a) {
+__global__ void __launch_bounds__(kMeanRuns * D) key_mean_kernel(const KeyStatsArgs a) {
   const size_t bh = static_cast<size_t>(blockIdx.y) * a.Hkv + blockIdx.x;
-  const float* p = a.part + bh * a.nsplit * D + threadIdx.x;
+  const int c = threadIdx.x % D, run = threadIdx.x / D;
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  const int per = (a.nsplit + kMeanRuns - 1) / kMeanRuns;
+  const int i0 = run * per, i1 = min(a.nsplit, i0 + per);
+  pdl_wait();  // the chunk sums are complete
+  const float* p = a.part + bh * a.nsplit * D + c;
   float s = 0.f;
 #pragma unroll 8
-  for (int i = 0; i < a.nsplit; ++i) s += p[static_cast<size_t>(i) * D];
-  a.kbar[bh * D + threadIdx.x] = s / static_cast<float>(a.Nkv);
+  for (int i = i0; i < i1; ++i) s += p[static_cast<size_t>(i) * D];
+  __shared__ float runs[kMeanRuns][D];
+  runs[run][c] = s;
+  __syncthreads();
+  if (run == 0) {
+    float t = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMeanRuns; ++r) t += runs[r][c];
+    a.kbar[bh * D + c] = t / static_cast<float>(a.Nkv);
+  }
 }
 
 template <int D>
@@ -74,18 +94,26 @@ __global__ void __launch_bounds__(kStatThreads) key_radius_kernel(const KeyStats
   const size_t bh = static_cast<size_t>(b) * a.Hkv + h;
   constexpr int TPR = D / 8, RPI = kStatThreads / TPR;
   const int c8 = threadIdx.x % TPR, r = threadIdx.x / TPR;
+  const int j0 = split * kChunkKeys, j1 = min(a.Nkv, j0 + kChunkKeys);
+  const uint4* k = reinterpret_cast<const uint4*>(a.k);
+  constexpr int NP = kChunkKeys / RPI;
+  uint4 kv[NP];  // this thread's keys, loaded while the mean is still being formed
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int j = j0 + r + p * RPI;
+    kv[p] = j < j1 ? k[((static_cast<size_t>(b) * a.Nkv + j) * a.Hkv + h) * TPR + c8] : make_uint4(0, 0, 0, 0);
+  }
+  pdl_wait();  // kbar is complete
   float kb[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) kb[i] = a.kbar[bh * D + c8 * 8 + i];
-  const int j0 = split * kChunkKeys, j1 = min(a.Nkv, j0 + kChunkKeys);
-  const uint4* k = reinterpret_cast<const uint4*>(a.k);
   float mx = 0.f;
 #pragma unroll
-  for (int p = 0; p < kChunkKeys / RPI; ++p) {
+  for (int p = 0; p < NP; ++p) {
     const int j = j0 + r + p * RPI;
     float ss = 0.f;
     if (j < j1) {
-      const uint4 u = k[((static_cast<size_t>(b) * a.Nkv + j) * a.Hkv + h) * TPR + c8];
+      const uint4 u = kv[p];
       const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -119,11 +147,9 @@ cudaError_t launch_d(const KeyStatsArgs& a, cudaStream_t s) {
   key_sum_kernel<D><<<grid, kStatThreads, 0, s>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  key_mean_kernel<D><<<dim3(a.Hkv, a.B), D, 0, s>>>(a);
-  e = cudaGetLastError();
+  e = launch_after_pdl(key_mean_kernel<D>, dim3(a.Hkv, a.B), dim3(kMeanRuns * D), 0, s, a);
   if (e != cudaSuccess) return e;
-  key_radius_kernel<D><<<grid, kStatThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_after_pdl(key_radius_kernel<D>, grid, dim3(kStatThreads), 0, s, a);
 }
 
 }  // namespace
