@@ -11,8 +11,9 @@
 //                      consecutive chunks summed in parallel and then added in
 //                      run order, so the result does not depend on scheduling;
 //   key_radius_kernel  the largest centred norm of each chunk, folded into
-//                      `radius` with an integer atomicMax on the float's bits
-//                      (non-negative floats order like their bit patterns).
+//                      `radius` (zeroed by the mean kernel) with an integer
+//                      atomicMax on the float's bits (non-negative floats
+//                      order like their bit patterns).
 // The second and third are programmatic dependents of the one before them:
 // they start while it drains, and the radius kernel loads its keys (an input
 // of the call) before it waits for the mean.
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(kMeanRuns * D) key_mean_kernel(const KeyStatsA
   __shared__ float runs[kMeanRuns][D];
   runs[run][c] = s;
   __syncthreads();
+  if (threadIdx.x == 0) a.radius[bh] = 0.f;  // folded into the maximum by the radius kernel
   if (run == 0) {
     float t = 0.f;
 #pragma unroll
@@ -141,11 +143,9 @@ __global__ void __launch_bounds__(kStatThreads) key_radius_kernel(const KeyStats
 
 template <int D>
 cudaError_t launch_d(const KeyStatsArgs& a, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(a.radius, 0, sizeof(float) * static_cast<size_t>(a.B) * a.Hkv, s);
-  if (e != cudaSuccess) return e;
   const dim3 grid(a.nsplit, a.Hkv, a.B);
   key_sum_kernel<D><<<grid, kStatThreads, 0, s>>>(a);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_after_pdl(key_mean_kernel<D>, dim3(a.Hkv, a.B), dim3(kMeanRuns * D), 0, s, a);
   if (e != cudaSuccess) return e;
