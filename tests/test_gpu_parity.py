@@ -572,6 +572,33 @@ def test_key_stats_and_bound_forward(case):
     assert int(nfb.item()) == int((flags == 0).sum()) == 0
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_key_stats_repeatable_and_reset_on_every_call(d):
+    """The chunk sums are added in a fixed order, so repeated calls agree bit
+    for bit; the radius starts from zero on every call, so statistics of wide
+    keys followed by narrow keys into the same buffers give the narrow keys'
+    radius.  129 chunks: not a multiple of the mean's eight runs."""
+    B, Hkv, N = 2, 3, 128 * 128 + 77
+    _, k, _ = make_inputs(3500 + d, B, Hkv, Hkv, 1, N, d)
+    kf = synthetic.bf16_bits_to_f32(k) + np.float32(0.5)
+    k = synthetic.f32_to_bf16_bits(kf)
+    wide = synthetic.f32_to_bf16_bits(kf * np.float32(8.0))
+    kbar = torch.empty((B, Hkv, d), dtype=torch.float32, device="cuda")
+    radius = torch.empty((B, Hkv), dtype=torch.float32, device="cuda")
+    eio.key_stats(dev_bf16(wide), kbar=kbar, radius=radius)
+    r_wide = radius.clone()
+    tk = dev_bf16(k)
+    eio.key_stats(tk, kbar=kbar, radius=radius)
+    kb1, r1 = kbar.clone(), radius.clone()
+    kb2, r2 = eio.key_stats(tk)
+    eio.sync_status()
+    assert torch.equal(kb1, kb2) and torch.equal(r1, r2)
+    assert (r1 < r_wide).all()
+    rk, rr = oracle.key_stats(k)
+    np.testing.assert_allclose(kb1.cpu().numpy(), rk, atol=2e-5, rtol=1e-5)
+    np.testing.assert_allclose(r1.cpu().numpy(), rr, rtol=1e-5)
+
+
 def test_bound_forward_falls_back_on_long_queries():
     """Every fifth query 40x longer: those rows' bounds exceed the limit and
     keep the running max; the count matches the oracle's and O is exact."""
