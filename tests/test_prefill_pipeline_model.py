@@ -13,11 +13,10 @@ under random schedules, for both layouts:
 with and without the slot offset (slot A starts an item once slot B has
 finished the exponentials of its first tile; slot B can be up to QB - 1
 short items ahead of slot A's wait, so the kernel signals offset item n on
-barrier n % QB).  Items are pairs as the
-planner makes them: equal slots, slot A one tile shorter (causal pairs, not
-offset), a lone tile in slot B, and a slot B with no key tile at all.  The
-half-tile pipeline of the bound-based form has its own model
-(test_pipeline_model.py).
+barrier n % QB).  Items are pairs as the planner makes them: equal slots,
+slot A one tile shorter (causal pairs, not offset), a lone tile in slot B,
+and a slot B with no key tile at all.  The half-tile pipeline of the
+bound-based form has its own model (test_pipeline_model.py).
 """
 import random
 
