@@ -13,7 +13,7 @@
 // other slot's GEMMs.
 //
 // Roles (384 threads, three warpgroups; the first gives registers to the
-// two softmax warpgroups with setmaxnreg: 128 x 72 + 256 x 216 = 384 x 168):
+// two softmax warpgroups with setmaxnreg: 128 x 72 + 256 x 216 <= 384 x 168, or 80 and 208):
 //   warp 0        TMA producer: Q_A, Q_B once per item (double-buffered for
 //                 d = 64, whose items are short), then K_j, V_j into a ring of
 //                 shared-memory stages.
@@ -55,10 +55,17 @@ constexpr int kThreads = 384;
 // exactly kLaunchRegs registers per thread: the host refuses to launch it
 // otherwise, since an increase that the pool cannot cover never returns.
 constexpr int kLaunchRegs = 168;
-constexpr int kRegsControl = 72;   // warpgroup 0: producer, MMA issuer
-constexpr int kRegsSoftmax = 216;  // warpgroups 1 and 2
-static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
-              "register split must fit in the launch allocation");
+// Warpgroup 0 (producer, MMA issuers) and warpgroups 1 and 2 (softmax).  The
+// d = 128 running-max softmax (128 scores per thread) needs 216 to run without
+// spills; the d = 64 forms and the bound-based half-tile forms fit their
+// softmax in 208, and their issuers (more per-item state) spill at 72.
+template <int D, bool BOUND>
+struct RegSplit {
+  static constexpr int kControl = (D == 64 || BOUND) ? 80 : 72;
+  static constexpr int kSoftmax = (D == 64 || BOUND) ? 208 : 216;
+  static_assert(128 * kControl + 256 * kSoftmax <= kThreads * kLaunchRegs,
+                "register split must fit in the launch allocation");
+};
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Bound-based softmax: a row keeps the bound as its base only if no P can fall
 // below 2^-kBoundLimit2 (every centred score lies within +-bound).
@@ -302,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long n_items = a.n_items;
 
   if (warp < 4) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<D, BOUND>::kControl));
   // The producer and MMA warps run converged; elect.sync picks the lane that
   // issues each TMA copy, MMA and commit.
   auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -597,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait(&mma_idle[x], 0);
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<D, BOUND>::kSoftmax));
     // ------------------------------------------------------------ softmax
     const int x = (warp - 4) >> 2;  // slot
     const int quarter = warp & 3;
