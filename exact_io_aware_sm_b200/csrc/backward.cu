@@ -74,8 +74,27 @@ namespace eio {
 namespace {
 
 constexpr int kT = 128;  // rows of a Q tile, keys of a KV tile: the MMA's M
-constexpr int kBThreads = 320;
+constexpr int kBThreads = 320;  // dQ: warp 0 producer, warp 1 MMA, warps 2-9 element-wise
 constexpr int kEW = 8;   // element-wise warps
+// dK/dV at d = 64: 384 threads.  Warpgroup 0: warp 0 the producer, warp 1
+// the MMA issuer (and TMEM owner), warps 2 and 3 idle; warps 4-11
+// (warpgroups 1 and 2) element-wise.  setmaxnreg moves registers from
+// warpgroup 0 to the element-wise warps, which spilled at the 168 every
+// thread gets otherwise.  The split is only safe when the kernel starts with
+// exactly kKVLaunchRegs registers per thread; the host checks this before the
+// first launch.  At d = 128 the dK/dV kernel keeps the dQ kernel's layout (it
+// measured slower with the split).
+template <int D>
+constexpr bool kKVSplit = D == 64;
+template <int D>
+constexpr int kKVThreads = kKVSplit<D> ? 384 : kBThreads;
+template <int D>
+constexpr int kKVFirstEW = kKVSplit<D> ? 4 : 2;
+constexpr int kKVLaunchRegs = 168;
+constexpr int kKVRegsControl = 80;
+constexpr int kKVRegsEW = 208;
+static_assert(128 * kKVRegsControl + 256 * kKVRegsEW <= kKVThreads<64> * kKVLaunchRegs,
+              "register split must fit in the launch allocation");
 constexpr float kLog2e = 1.4426950408889634f;
 // Of every 8 column pairs, this many take the polynomial 2^x on the FMA pipe
 // instead of the MUFU unit (measured: 1 at d = 64 and 2 at d = 128 were
@@ -345,7 +364,7 @@ __device__ __forceinline__ void write_ds(uint32_t t_dp, uint32_t t_ds, const flo
 // BLK: block-sparse mask (tile lists with block bitmaps); otherwise no mask
 // or causal.
 template <int D, bool BLK>
-__global__ void __launch_bounds__(kBThreads, 1)
+__global__ void __launch_bounds__(kKVThreads<D>, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
@@ -408,6 +427,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
   };
   auto stage = [&](uint32_t t) { return smem + C::kOffRing + (t % R) * 2 * C::kTile; };
 
+  constexpr int kFirstEW = kKVFirstEW<D>;
+  if (warp < kFirstEW) {
+  if constexpr (kKVSplit<D>) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kKVRegsControl));
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -547,9 +569,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
     // Every MMA issued above has finished before TMEM is released.
     mma_commit_elect(br.mma_idle);
     mbar_wait(br.mma_idle, 0);
+  }  // d = 64: warps 2 and 3 have no role
   } else {
+    if constexpr (kKVSplit<D>) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kKVRegsEW));
     // ------------------------------------------------------------ element-wise
-    const int h = (warp - 2) >> 2;  // column half
+    const int h = (warp - kFirstEW) >> 2;  // column half
     const int quarter = warp & 3;
     const uint32_t lo = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t t_row = tmem + lo;
@@ -557,12 +581,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
     constexpr int STG = C::kOffStgKV;
     // Staged output of the k-th item: wait until the previous item's TMA
     // stores have read the staging tiles, write this thread's rows (fill),
-    // and have warp 2 store the tiles (issue) once every element-wise warp
+    // and have the first element-wise warp store the tiles (issue) once every element-wise warp
     // has written.  All waits are bounded.
     auto stage_out = [&](long long k, auto fill, auto issue) -> bool {
       uint8_t* stg = smem + STG;
       if (k > 0) {
-        if (warp == 2) {
+        if (warp == kFirstEW) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
           if (lane == 0) mbar_arrive(br.stg_free);
@@ -573,7 +597,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(br.stg_full);
-      if (warp == 2) {
+      if (warp == kFirstEW) {
         if (!wwait(br.stg_full, k & 1)) return false;
         if (lane == 0) {
           issue(stg);
@@ -695,7 +719,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       }
     }
     if (!ok && lane == 0) fail(kErrDeviceTimeout);
-    if (C::kStage && warp == 2 && lane == 0) bulk_wait_all();  // stores done before the CTA retires
+    if (C::kStage && warp == kFirstEW && lane == 0) bulk_wait_all();  // stores done before the CTA retires
   }
 
   tc_fence_before();
@@ -1061,8 +1085,14 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   int dev = 0, n_sm = 0;
   cudaGetDevice(&dev);
   if (!attr_set.test(dev)) {
-    cudaError_t e =
-        cudaFuncSetAttribute(bwd_dq_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemQ);
+    // The dK/dV kernel's warpgroup register split needs every thread to start
+    // with exactly kKVLaunchRegs registers.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, bwd_dkdv_kernel<D, BLK>);
+    if (e != cudaSuccess) return e;
+    if (kKVSplit<D> && (fa.numRegs != kKVLaunchRegs || fa.maxThreadsPerBlock < kKVThreads<D>))
+      return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(bwd_dq_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemQ);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemKV);
     if (e != cudaSuccess) return e;
@@ -1086,7 +1116,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_after_pdl(bwd_dkdv_kernel<D, BLK>, dim3(static_cast<unsigned>(n_kv < n_sm ? n_kv : n_sm)),
-                          dim3(kBThreads), C::kSmemKV, s, tq, tdo, tk, tv, tdk, tdv, a);
+                          dim3(kKVThreads<D>), C::kSmemKV, s, tq, tdo, tk, tv, tdk, tdv, a);
 }
 
 }  // namespace
